@@ -1,0 +1,190 @@
+/*
+ * zha.h -- C-ABI of libzha: the Zyphra Hierarchical Attention (ZHA) hot path
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The method (lefilia.fr page "Zyphra presente Zyphra Hierarchical Attention
+ * (ZHA), une voie vers une attention vraiment sous-quadratique", paragraph 1):
+ * the KV cache stays complete and a tree over it only decides which keys each
+ * query reads. Keys are cut into contiguous blocks of b tokens; each block gets
+ * one summary key derived from 16 learned reference queries; blocks are grouped
+ * level by level (a level-l node covers b^l tokens). A query scores the top
+ * nodes, keeps the smallest set covering a fraction p of the estimated
+ * attention mass, expands only the kept branches down to the raw KV entries,
+ * and always keeps the first token. Paragraph 2 gives the operating point
+ * p = 0.95 and the two geometries (b = 4, L = 6) and (b = 256, L = 1).
+ *
+ * Formulas the pages leave open are fixed by this library as:
+ *   summary   s = (1/16) sum_r sum_c softmax_c(R_r . x_c / sqrt(d)) x_c over the
+ *             node's children x_c (raw keys at level 1, stored summaries above);
+ *             R is 16 x d, shared by all KV heads;
+ *   node mass exp(q . s / sqrt(d) + ln b^l);
+ *   causal tail: tokens of [b^L T_top(t), t] with T_top(t) = floor((t+1)/b^L)
+ *             are always attended (they are not yet in a complete top node);
+ *   GQA:      q head h reads KV head h / (Hq / Hkv) and selects on its own.
+ * Selection uses a canonical fp32 arithmetic (sequential fmaf dot products, a
+ * Cody-Waite/Taylor exponential, fixed-point masses: M = trunc(e^(z-zmax) 2^40),
+ * need = ceil(T p_q / 2^32), p_q = floor(p 2^32 + 0.5), ties to the lower node
+ * index), so selected index sets are reproducible bit for bit.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller (for example
+ *     PyTorch tensors), contiguous, 16-byte aligned. The library never
+ *     allocates, never synchronises the device and keeps no state between
+ *     calls; it is re-entrant.
+ *   - `stream` is a cudaStream_t passed as void*; every call is asynchronous on
+ *     it.
+ *   - Argument errors return synchronously before any launch
+ *     (ZHA_ERR_INVALID_ARG / ZHA_ERR_UNSUPPORTED / ZHA_ERR_WORKSPACE).
+ *     Launch failures return ZHA_ERR_CUDA. Data-dependent conditions found by a
+ *     kernel (an index list longer than its capacity, a candidate list longer
+ *     than the workspace) are OR-ed as zha_status bits into *dev_status (a
+ *     device int32 the caller zeroes and reads after its own synchronisation);
+ *     outputs are then truncated safely. No kernel traps or asserts.
+ *   - dtype ZHA_BF16: K, V, Q, outputs and stored summaries are bf16.
+ *     dtype ZHA_F32: all of them are fp32. R is always fp32.
+ *   - Layouts (row-major):
+ *       K, V       [batch][n_kv_heads][capacity][head_dim]
+ *       summaries  level l (1..L) starts at element level_offsets[l-1] of
+ *                  `tree` and is [batch][n_kv_heads][capacity / b^l][head_dim];
+ *                  node (l, j) covers tokens [j b^l, (j+1) b^l)
+ *       decode Q   [batch][n_q_heads][head_dim], query position seq_len[s]-1
+ *       outputs    same shape as their queries
+ *       level_counts [query][q head][L], kept node counts, top level first
+ */
+#ifndef ZHA_H
+#define ZHA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum zha_status {
+  ZHA_OK = 0,
+  ZHA_ERR_INVALID_ARG = 1,   /* null pointer, bad size or geometry, p out of range */
+  ZHA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. head_dim not 64/128) */
+  ZHA_ERR_CUDA = 4,          /* a launch or runtime call failed */
+  ZHA_ERR_CAPACITY = 8,      /* device status bit: an index list hit idx_cap */
+  ZHA_ERR_WORKSPACE = 16,    /* workspace smaller than zha_workspace_bytes() */
+  ZHA_ERR_TIMEOUT = 32,      /* device status bit: a bounded wait gave up */
+  ZHA_ERR_INTERNAL = 64      /* device status bit: an internal consistency check failed */
+} zha_status;
+
+typedef enum zha_dtype { ZHA_F32 = 0, ZHA_BF16 = 1 } zha_dtype;
+
+typedef enum zha_op {
+  ZHA_OP_SELECT = 0,
+  ZHA_OP_ATTEND = 1,
+  ZHA_OP_DECODE = 2,
+  ZHA_OP_PREFILL = 3,
+  ZHA_OP_DENSE = 4
+} zha_op;
+
+/* Geometry and shapes. b (block) >= 2 and either divides 32 or is a multiple
+ * of 32 up to 1024; 1 <= levels <= 8; head_dim 64 or 128; n_q_heads a multiple
+ * of n_kv_heads with at most 8 query heads per KV head. */
+typedef struct zha_config {
+  int32_t head_dim;   /* d */
+  int32_t block;      /* b */
+  int32_t levels;     /* L */
+  int32_t n_q_heads;  /* Hq */
+  int32_t n_kv_heads; /* Hkv */
+  int32_t batch;      /* B */
+  int64_t capacity;   /* rows per (sequence, KV head) in K and V */
+  int32_t dtype;      /* zha_dtype */
+  int32_t reserved;   /* must be 0 */
+} zha_config;
+
+/* The cache a call works on. k, v, r are read-only; tree is written by the
+ * build/extend calls and read by the others; seq_len[b] (device int32) is the
+ * number of valid tokens of sequence b. */
+typedef struct zha_cache {
+  const void* k;
+  const void* v;
+  const float* r;          /* [16][head_dim] learned reference queries */
+  void* tree;              /* summaries, see layout above */
+  const int32_t* seq_len;  /* [batch], device */
+} zha_cache;
+
+/* Human-readable name of a status value (or of the lowest set bit). */
+const char* zha_status_string(int32_t status);
+
+/* Host-only query: bytes of the summary tree and the element offset of each
+ * level (level_offsets[l-1] for l = 1..L; may be NULL). */
+zha_status zha_tree_layout(const zha_config* cfg, size_t* tree_bytes, int64_t* level_offsets);
+
+/* Host-only query: workspace bytes the given operation needs for up to
+ * max_queries query tokens (decode/dense: ignored, the batch is used; prefill:
+ * the chunk length T). */
+zha_status zha_workspace_bytes(const zha_config* cfg, int32_t op, int64_t max_queries,
+                               size_t* bytes);
+
+/* Build every complete node of every level for the first seq_len[b] tokens of
+ * each sequence (lefilia.fr page, par. 1: blocks summarised, then grouped
+ * level by level). Nodes that are not complete are left untouched. */
+zha_status zha_build_tree(const zha_config* cfg, const zha_cache* cache, void* stream);
+
+/* Build exactly the nodes that became complete when sequence b grew from
+ * old_len[b] (device int32) to seq_len[b] tokens. max_new_tokens is a host
+ * upper bound on seq_len[b] - old_len[b] over all b (it sizes the launch);
+ * growth beyond it is left unbuilt. */
+zha_status zha_extend_tree(const zha_config* cfg, const zha_cache* cache, const int32_t* old_len,
+                           int64_t max_new_tokens, void* stream);
+
+/* Top-p traversal (lefilia.fr page, par. 1) for nq query tokens with all Hq
+ * heads each: q [nq][Hq][d]; token i belongs to sequence q_seq[i] at position
+ * q_pos[i] (device int32 arrays, q_pos[i] < seq_len[q_seq[i]]). For query
+ * (i, h) the ascending selected token list
+ *   S = tokens of kept level-1 nodes U {0} U [b^L T_top, t]
+ * is written to idx + (i*Hq + h)*idx_cap, its length to n_idx[i*Hq + h] and
+ * the kept node counts per level to level_counts (nullable). p in (0, 1];
+ * p >= 1 keeps every candidate. Lists longer than idx_cap are truncated and
+ * set ZHA_ERR_CAPACITY in *dev_status. ws/ws_bytes: ZHA_OP_SELECT workspace. */
+zha_status zha_select(const zha_config* cfg, const zha_cache* cache, const void* q,
+                      const int32_t* q_seq, const int32_t* q_pos, int64_t nq, double p,
+                      int32_t* idx, int64_t idx_cap, int32_t* n_idx, int32_t* level_counts,
+                      void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* Exact softmax attention of each query (i, h) over its list idx/n_idx (as
+ * written by zha_select, ascending token positions of sequence q_seq[i]):
+ * out[i][h] = sum_j softmax_j(q . k_j / sqrt(d)) v_j. fp32 accumulation.
+ * ws/ws_bytes: ZHA_OP_ATTEND workspace for nq queries. */
+zha_status zha_attend(const zha_config* cfg, const zha_cache* cache, const void* q,
+                      const int32_t* q_seq, int64_t nq, const int32_t* idx, int64_t idx_cap,
+                      const int32_t* n_idx, void* out, void* ws, size_t ws_bytes,
+                      int32_t* dev_status, void* stream);
+
+/* One decode step for every sequence: selection at position seq_len[b] - 1
+ * followed by attention over the selected keys, q [B][Hq][d] -> out [B][Hq][d].
+ * The query heads sharing a KV head are traversed together and their
+ * selections are read from HBM once (per-head masks). level_counts is
+ * nullable. The tree must already contain every node complete at seq_len
+ * (call zha_extend_tree after appending tokens). ws: ZHA_OP_DECODE workspace. */
+zha_status zha_decode(const zha_config* cfg, const zha_cache* cache, const void* q, double p,
+                      void* out, int32_t* level_counts, void* ws, size_t ws_bytes,
+                      int32_t* dev_status, void* stream);
+
+/* Chunked prefill of sequence `seq`: the caller has written the chunk's K and V
+ * rows [chunk_start, chunk_start + T) and set seq_len[seq] = chunk_start + T.
+ * Extends the tree over the chunk, then for every token i of the chunk
+ * (position chunk_start + i) and head h selects causally and attends:
+ * q [T][Hq][d] -> out [T][Hq][d]. level_counts ([T][Hq][L]) is nullable.
+ * ws: ZHA_OP_PREFILL workspace for max_queries = T. */
+zha_status zha_prefill_chunk(const zha_config* cfg, const zha_cache* cache, const void* q,
+                             int32_t seq, int64_t chunk_start, int64_t T, double p, void* out,
+                             int32_t* level_counts, void* ws, size_t ws_bytes,
+                             int32_t* dev_status, void* stream);
+
+/* Dense flash-decoding over every key [0, seq_len[b] - 1] (the baseline the
+ * sparse path is measured against): q [B][Hq][d] -> out [B][Hq][d].
+ * ws: ZHA_OP_DENSE workspace. */
+zha_status zha_dense_decode(const zha_config* cfg, const zha_cache* cache, const void* q,
+                            void* out, void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZHA_H */

@@ -1,0 +1,79 @@
+"""The C-ABI library loads without a GPU, exports every declared entry point,
+and rejects bad arguments on the host before any launch. CPU only."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    with open(os.path.join(ROOT, "include", "zha.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^(?:zha_status|const char\*)\s+(zha_\w+)\(", text, re.M)))
+
+
+@pytest.fixture(scope="module")
+def z():
+    import __graft_entry__
+
+    __graft_entry__.build()
+    import tree_indexed_sparse_zha_b200 as z
+
+    return z
+
+
+def test_exports_every_declared_symbol(z):
+    names = _declared_functions()
+    assert len(names) == 10, names
+    lib = z.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(z.EXPORTS)
+
+
+def test_tree_layout_host_only(z):
+    cfg = z.make_config(128, 4, 6, 16, 2, 8, 262400, torch.bfloat16)
+    nbytes, offs = z.zha_tree_layout(cfg)
+    rows = [262400 // 4 ** l for l in range(1, 7)]
+    exp_offs = [sum(8 * 2 * r * 128 for r in rows[:i]) for i in range(6)]
+    assert offs == exp_offs
+    assert nbytes == 2 * sum(8 * 2 * r * 128 for r in rows)
+
+
+def test_status_strings(z):
+    assert z.status_string(0) == "ok"
+    assert "capacity" in z.status_string(z.ZHA_ERR_CAPACITY)
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("head_dim", 96, 2), ("block", 3, 2), ("block", 48, 2), ("levels", 0, 1), ("levels", 9, 1),
+    ("n_q_heads", 15, 1), ("n_q_heads", 12, 2), ("n_q_heads", 32, 2), ("batch", 0, 1), ("capacity", 0, 1),
+    ("dtype", 7, 1), ("reserved", 1, 1),
+])
+def test_bad_geometry_rejected(z, field, value, code):
+    cfg = z.make_config(128, 4, 6, 16, 2, 8, 262400, torch.bfloat16)
+    setattr(cfg, field, value)
+    n = ctypes.c_size_t(0)
+    assert z.lib().zha_tree_layout(ctypes.byref(cfg), ctypes.byref(n), None) == code
+
+
+def test_bad_arguments_rejected_before_launch(z):
+    cfg = z.make_config(128, 4, 6, 16, 2, 1, 4096, torch.bfloat16)
+    L = z.lib()
+    # null cache / null pointers and p out of range never reach the device
+    assert L.zha_build_tree(ctypes.byref(cfg), None, None) == z.ZHA_ERR_INVALID_ARG
+    c = z.zha_cache(0, 0, 0, 0, 0)
+    assert L.zha_build_tree(ctypes.byref(cfg), ctypes.byref(c), None) == z.ZHA_ERR_INVALID_ARG
+    c = z.zha_cache(16, 16, 16, 16, 16)  # non-null dummies: p is checked first
+    for p in (0.0, -0.5, float("nan")):
+        assert L.zha_decode(ctypes.byref(cfg), ctypes.byref(c), ctypes.c_void_p(16), p,
+                            ctypes.c_void_p(16), None, ctypes.c_void_p(16), 1 << 40, None,
+                            None) == z.ZHA_ERR_INVALID_ARG
+    # workspace too small
+    assert L.zha_dense_decode(ctypes.byref(cfg), ctypes.byref(c), ctypes.c_void_p(16),
+                              ctypes.c_void_p(16), ctypes.c_void_p(16), 1, None) == \
+        z.ZHA_ERR_WORKSPACE

@@ -1,0 +1,186 @@
+"""CUDA path vs the CPU oracle, through the C-ABI.
+
+Bar: summary trees, selected index sets and per-level kept counts bit-exact;
+attention outputs within max-abs 2e-2 (bf16 I/O, fp32 accumulation) or 1e-5
+(fp32 mode) of the oracle's fp64 attention over the oracle's own selection."""
+import numpy as np
+import pytest
+import torch
+
+from tree_indexed_sparse_zha_b200 import workloads as W
+
+from _harness import TOL, Gpu, Ref, compare_tree
+
+pytestmark = pytest.mark.gpu
+
+
+def _decode_parity(wl, step_q, p, n_tokens, units=None, heads=None):
+    """zha_decode + zha_select + zha_attend on the current cache state vs oracle."""
+    c = wl.cfg
+    gpu = _decode_parity.gpu
+    ref = _decode_parity.ref
+    q = step_q.to(gpu.dev)
+    out, lc = gpu.decode(q, p)
+    t = n_tokens - 1
+    qf = q.float().cpu().numpy()
+    seqs = range(c.batch) if units is None else units
+    hs = range(c.n_q_heads) if heads is None else heads
+    cap = n_tokens + 2
+    idx, n_idx, lcs, qs = gpu.select(q, list(range(c.batch)), [t] * c.batch, p, cap)
+    att = gpu.attend(q, qs, idx, n_idx)
+    idx = idx.cpu().numpy()
+    n_idx = n_idx.cpu().numpy()
+    lcs = lcs.cpu().numpy()
+    flagged = 0
+    for s in seqs:
+        for h in hs:
+            e_idx, e_counts, _, tie = ref.select(qf[s, h], s, h, t, p)
+            flagged += tie
+            assert lc[s, h].tolist() == e_counts.tolist(), (s, h, lc[s, h], e_counts)
+            assert lcs[s, h].tolist() == e_counts.tolist()
+            assert n_idx[s, h] == len(e_idx)
+            assert np.array_equal(idx[s, h, :n_idx[s, h]], e_idx), (s, h)
+            o = ref.attend(qf[s, h], s, h, e_idx)
+            tol = TOL[c.dtype]
+            assert np.abs(out[s, h] - o).max() < tol, (s, h, np.abs(out[s, h] - o).max())
+            assert np.abs(att[s, h] - o).max() < tol
+    return flagged
+
+
+def _run_decode_case(wl, p=None, units=None, heads=None, check_tree_units=None):
+    c = wl.cfg
+    gpu = Gpu(wl)
+    ref = Ref(wl, c.n_tokens)
+    _decode_parity.gpu, _decode_parity.ref = gpu, ref
+    for (s, k) in (check_tree_units or [(s, k) for s in range(c.batch)
+                                        for k in range(c.n_kv_heads)]):
+        compare_tree(gpu, ref, s, k)
+    return _decode_parity(wl, wl.queries(0), c.p if p is None else p, c.n_tokens, units, heads)
+
+
+def test_tiny_f32():
+    _run_decode_case(W.make("tiny-f32-1k"))
+
+
+def test_decode_deep_32k():
+    _run_decode_case(W.make("decode-deep-32k"))
+
+
+@pytest.mark.parametrize("n", [300, 4095, 4096, 4097, 9000])
+def test_ragged_lengths(n):
+    # fewer tokens than one top node (dense), exactly one, one plus a tail
+    _run_decode_case(W.make("decode-deep-32k", n_tokens=n))
+
+
+def test_tiny_p_sweep():
+    wl = W.make("tiny-f32-1k")
+    for p in (1e-6, 0.3, 0.8, 0.999, 1.0):
+        _run_decode_case(wl, p=p)
+
+
+def test_decode_deep_256k_scaled_incremental():
+    """Scaled copy of the 256K decode run: 8 sequences, extend + decode every step."""
+    wl = W.make("decode-deep-256k-b8", n_tokens=16384 + 4090, steps=24)
+    c = wl.cfg
+    gpu = Gpu(wl)
+    z = __import__("tree_indexed_sparse_zha_b200")
+    final_n = c.n_tokens + c.steps
+    ref = Ref(wl, final_n)
+    _decode_parity.gpu, _decode_parity.ref = gpu, ref
+    old = gpu.cache.seq_len.clone()
+    for step in range(1, c.steps + 1):
+        old.copy_(gpu.cache.seq_len)
+        gpu.cache.seq_len.add_(1)
+        z.zha_extend_tree(gpu.cfg, gpu.cache, old, 1)
+        n = c.n_tokens + step
+        if step in (1, 6, 7, 23, 24):  # 16384+4096 = 20480 completes a top node at step 6
+            _decode_parity(wl, wl.queries(step), c.p, n)
+    torch.cuda.synchronize()
+    for s in range(c.batch):
+        for k in range(c.n_kv_heads):
+            compare_tree(gpu, ref, s, k)
+
+
+def test_decode_wide_scaled_p_sweep():
+    wl = W.make("decode-wide-256k-b8", n_tokens=16384 + 100)
+    c = wl.cfg
+    gpu = Gpu(wl)
+    ref = Ref(wl, c.n_tokens)
+    _decode_parity.gpu, _decode_parity.ref = gpu, ref
+    compare_tree(gpu, ref, 0, 0)
+    compare_tree(gpu, ref, 7, 1)
+    q = wl.queries(0)
+    for p in c.p_sweep:
+        _decode_parity(wl, q, p, c.n_tokens)
+    # p = 1 keeps everything: the sparse path equals the dense kernel
+    out1, _ = gpu.decode(q.to(gpu.dev), 1.0)
+    dense = gpu.dense(q.to(gpu.dev))
+    assert np.abs(out1 - dense).max() < TOL["bf16"]
+
+
+def test_prefill_scaled():
+    """Scaled chunked prefill: a 256-token chunk whose middle completes a top
+    node (positions 16256..16511; top node 3 ends at 16383), causal."""
+    base = W.CONFIGS["prefill-deep-1m-chunk4k"]
+    wl = W.Workload(base.scaled(16256, chunk=256))
+    c = wl.cfg
+    gpu = Gpu(wl)  # tree over the first 16384 tokens
+    z = __import__("tree_indexed_sparse_zha_b200")
+    start = c.n_tokens
+    gpu.cache.seq_len.fill_(start + c.chunk)
+    q = wl.queries(0).to(gpu.dev)
+    out = torch.empty_like(q)
+    lc = torch.full((c.chunk, c.n_q_heads, c.levels), -1, dtype=torch.int32, device=gpu.dev)
+    ws = z.alloc_workspace(gpu.cfg, z.ZHA_OP_PREFILL, c.chunk, device=gpu.dev)
+    z.zha_prefill_chunk(gpu.cfg, gpu.cache, q, 0, start, c.p, out, lc, ws, gpu.status)
+    gpu.check_status()
+    ref = Ref(wl, start + c.chunk)
+    compare_tree(gpu, ref, 0, 0)
+    compare_tree(gpu, ref, 0, 1)
+    out = out.float().cpu().numpy()
+    lc = lc.cpu().numpy()
+    qf = q.float().cpu().numpy()
+    rng = np.random.default_rng(0)
+    tokens = sorted(set([0, 1, 126, 127, 128, c.chunk - 2, c.chunk - 1])
+                    | set(rng.choice(c.chunk, 12, replace=False).tolist()))
+    for i in tokens:
+        for h in range(c.n_q_heads):
+            e_idx, e_counts, _, _ = ref.select(qf[i, h], 0, h, start + i, c.p)
+            assert lc[i, h].tolist() == e_counts.tolist(), (i, h)
+            o = ref.attend(qf[i, h], 0, h, e_idx)
+            assert np.abs(out[i, h] - o).max() < TOL["bf16"], (i, h)
+
+
+def test_capacity_overflow_sets_status():
+    wl = W.make("decode-deep-32k", n_tokens=5000)
+    gpu = Gpu(wl)
+    q = wl.queries(0).to(gpu.dev)
+    gpu.select(q, [0], [4999], 0.95, 5001)  # fits
+    z = __import__("tree_indexed_sparse_zha_b200")
+    idx = torch.zeros(1, 16, 8, dtype=torch.int32, device=gpu.dev)
+    n_idx = torch.zeros(1, 16, dtype=torch.int32, device=gpu.dev)
+    ws = z.alloc_workspace(gpu.cfg, z.ZHA_OP_SELECT, 1, device=gpu.dev)
+    qs = torch.zeros(1, dtype=torch.int32, device=gpu.dev)
+    qp = torch.full((1,), 4999, dtype=torch.int32, device=gpu.dev)
+    z.zha_select(gpu.cfg, gpu.cache, q, qs, qp, 0.95, idx, n_idx, None, ws, gpu.status)
+    torch.cuda.synchronize()
+    assert int(gpu.status.item()) & z.ZHA_ERR_CAPACITY
+    assert (n_idx > 8).all()
+
+
+@pytest.mark.slow
+def test_decode_deep_256k_full_size_sampled():
+    """The headline workload at full size, in the launch configuration the bench
+    times; the oracle checks two (sequence, KV head) units of the first step."""
+    wl = W.make("decode-deep-256k-b8", device="cuda")
+    c = wl.cfg
+    wl.K, wl.V, wl.R = wl.K.cpu(), wl.V.cpu(), wl.R.cpu()
+    _run_decode_case(wl, units=[0, 5], heads=list(range(16)),
+                     check_tree_units=[(0, 0), (0, 1), (5, 0), (5, 1)])
+
+
+@pytest.mark.slow
+def test_decode_wide_256k_full_size_sampled():
+    wl = W.make("decode-wide-256k-b8", device="cuda")
+    wl.K, wl.V, wl.R = wl.K.cpu(), wl.V.cpu(), wl.R.cpu()
+    _run_decode_case(wl, units=[3], heads=list(range(16)), check_tree_units=[(3, 0), (3, 1)])

@@ -1,1 +1,253 @@
-"""B200-native ZHA hot path (placeholder; the binding is filled in below)."""
+"""B200-native hot path of Zyphra Hierarchical Attention (ZHA).
+
+Thin ctypes binding over ``libzha.so`` (sm_100a CUDA kernels behind the C-ABI
+declared in ``include/zha.h``). The functions keep the C names and only
+marshal arguments: every step of the path runs in the library's kernels on the
+caller's current CUDA stream. PyTorch provides device memory and streams.
+
+If the library is missing or cannot be loaded, importing the binding's
+functions raises immediately: there is no CPU or eager fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libzha.so")
+
+ZHA_OK = 0
+ZHA_ERR_INVALID_ARG = 1
+ZHA_ERR_UNSUPPORTED = 2
+ZHA_ERR_CUDA = 4
+ZHA_ERR_CAPACITY = 8
+ZHA_ERR_WORKSPACE = 16
+ZHA_ERR_TIMEOUT = 32
+ZHA_ERR_INTERNAL = 64
+
+ZHA_F32 = 0
+ZHA_BF16 = 1
+
+ZHA_OP_SELECT = 0
+ZHA_OP_ATTEND = 1
+ZHA_OP_DECODE = 2
+ZHA_OP_PREFILL = 3
+ZHA_OP_DENSE = 4
+
+EXPORTS = (
+    "zha_status_string", "zha_tree_layout", "zha_workspace_bytes", "zha_build_tree",
+    "zha_extend_tree", "zha_select", "zha_attend", "zha_decode", "zha_prefill_chunk",
+    "zha_dense_decode",
+)
+
+
+class zha_config(ctypes.Structure):
+    _fields_ = [
+        ("head_dim", ctypes.c_int32),
+        ("block", ctypes.c_int32),
+        ("levels", ctypes.c_int32),
+        ("n_q_heads", ctypes.c_int32),
+        ("n_kv_heads", ctypes.c_int32),
+        ("batch", ctypes.c_int32),
+        ("capacity", ctypes.c_int64),
+        ("dtype", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+    ]
+
+
+class zha_cache(ctypes.Structure):
+    _fields_ = [
+        ("k", ctypes.c_void_p),
+        ("v", ctypes.c_void_p),
+        ("r", ctypes.c_void_p),
+        ("tree", ctypes.c_void_p),
+        ("seq_len", ctypes.c_void_p),
+    ]
+
+
+class ZhaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libzha.so (built in-tree by ``__graft_entry__.build()``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libzha.so not found at {LIB_PATH}; run __graft_entry__.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.POINTER
+        c_cfg, c_cache = P(zha_config), P(zha_cache)
+        vp, i32, i64, d, sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_double,
+                               ctypes.c_size_t)
+        sig = {
+            "zha_status_string": ([i32], ctypes.c_char_p),
+            "zha_tree_layout": ([c_cfg, P(sz), P(i64)], i32),
+            "zha_workspace_bytes": ([c_cfg, i32, i64, P(sz)], i32),
+            "zha_build_tree": ([c_cfg, c_cache, vp], i32),
+            "zha_extend_tree": ([c_cfg, c_cache, vp, i64, vp], i32),
+            "zha_select": ([c_cfg, c_cache, vp, vp, vp, i64, d, vp, i64, vp, vp, vp, sz, vp, vp],
+                           i32),
+            "zha_attend": ([c_cfg, c_cache, vp, vp, i64, vp, i64, vp, vp, vp, sz, vp, vp], i32),
+            "zha_decode": ([c_cfg, c_cache, vp, d, vp, vp, vp, sz, vp, vp], i32),
+            "zha_prefill_chunk": ([c_cfg, c_cache, vp, i32, i64, i64, d, vp, vp, vp, sz, vp, vp],
+                                  i32),
+            "zha_dense_decode": ([c_cfg, c_cache, vp, vp, vp, sz, vp], i32),
+        }
+        for name, (args, res) in sig.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().zha_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int):
+    if status != ZHA_OK:
+        raise ZhaError(fn, status)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("libzha needs contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+# ---------------------------------------------------------------------------
+# configuration / cache handles
+# ---------------------------------------------------------------------------
+
+@dataclass
+class Cache:
+    """Device tensors one call works on (all caller-owned)."""
+    k: torch.Tensor           # [B][Hkv][Ncap][d]
+    v: torch.Tensor
+    r: torch.Tensor           # [16][d] fp32
+    tree: torch.Tensor        # flat buffer of zha_tree_layout() bytes (any dtype view)
+    seq_len: torch.Tensor     # [B] int32
+
+    def c(self) -> zha_cache:
+        return zha_cache(self.k.data_ptr(), self.v.data_ptr(), self.r.data_ptr(),
+                         self.tree.data_ptr(), self.seq_len.data_ptr())
+
+
+def make_config(head_dim: int, block: int, levels: int, n_q_heads: int, n_kv_heads: int,
+                batch: int, capacity: int, dtype: torch.dtype) -> zha_config:
+    return zha_config(head_dim, block, levels, n_q_heads, n_kv_heads, batch, capacity,
+                      ZHA_BF16 if dtype == torch.bfloat16 else ZHA_F32, 0)
+
+
+def zha_tree_layout(cfg: zha_config):
+    nbytes = ctypes.c_size_t(0)
+    offs = (ctypes.c_int64 * max(cfg.levels, 1))()
+    _check("zha_tree_layout", lib().zha_tree_layout(ctypes.byref(cfg), ctypes.byref(nbytes), offs))
+    return nbytes.value, [offs[i] for i in range(cfg.levels)]
+
+
+def zha_workspace_bytes(cfg: zha_config, op: int, max_queries: int = 0) -> int:
+    n = ctypes.c_size_t(0)
+    _check("zha_workspace_bytes",
+           lib().zha_workspace_bytes(ctypes.byref(cfg), op, max_queries, ctypes.byref(n)))
+    return n.value
+
+
+def alloc_tree(cfg: zha_config, device="cuda") -> torch.Tensor:
+    nbytes, _ = zha_tree_layout(cfg)
+    dt = torch.bfloat16 if cfg.dtype == ZHA_BF16 else torch.float32
+    return torch.zeros(max(nbytes // dt.itemsize, 1), dtype=dt, device=device)
+
+
+def alloc_workspace(cfg: zha_config, op: int, max_queries: int = 0, device="cuda") -> torch.Tensor:
+    return torch.empty(zha_workspace_bytes(cfg, op, max_queries), dtype=torch.uint8, device=device)
+
+
+# ---------------------------------------------------------------------------
+# entry points (same names as the C-ABI)
+# ---------------------------------------------------------------------------
+
+def zha_build_tree(cfg: zha_config, cache: Cache, stream=None):
+    c = cache.c()
+    _check("zha_build_tree", lib().zha_build_tree(ctypes.byref(cfg), ctypes.byref(c),
+                                                  _stream(stream)))
+
+
+def zha_extend_tree(cfg: zha_config, cache: Cache, old_len: torch.Tensor, max_new_tokens: int,
+                    stream=None):
+    c = cache.c()
+    _check("zha_extend_tree", lib().zha_extend_tree(ctypes.byref(cfg), ctypes.byref(c),
+                                                    _ptr(old_len), max_new_tokens,
+                                                    _stream(stream)))
+
+
+def zha_select(cfg: zha_config, cache: Cache, q: torch.Tensor, q_seq: torch.Tensor,
+               q_pos: torch.Tensor, p: float, idx: torch.Tensor, n_idx: torch.Tensor,
+               level_counts: Optional[torch.Tensor], ws: torch.Tensor,
+               dev_status: Optional[torch.Tensor] = None, stream=None):
+    c = cache.c()
+    nq = q.shape[0]
+    _check("zha_select", lib().zha_select(
+        ctypes.byref(cfg), ctypes.byref(c), _ptr(q), _ptr(q_seq), _ptr(q_pos), nq, float(p),
+        _ptr(idx), idx.shape[-1], _ptr(n_idx), _ptr(level_counts), _ptr(ws), ws.numel(),
+        _ptr(dev_status), _stream(stream)))
+
+
+def zha_attend(cfg: zha_config, cache: Cache, q: torch.Tensor, q_seq: torch.Tensor,
+               idx: torch.Tensor, n_idx: torch.Tensor, out: torch.Tensor, ws: torch.Tensor,
+               dev_status: Optional[torch.Tensor] = None, stream=None):
+    c = cache.c()
+    _check("zha_attend", lib().zha_attend(
+        ctypes.byref(cfg), ctypes.byref(c), _ptr(q), _ptr(q_seq), q.shape[0], _ptr(idx),
+        idx.shape[-1], _ptr(n_idx), _ptr(out), _ptr(ws), ws.numel(), _ptr(dev_status),
+        _stream(stream)))
+
+
+def zha_decode(cfg: zha_config, cache: Cache, q: torch.Tensor, p: float, out: torch.Tensor,
+               level_counts: Optional[torch.Tensor], ws: torch.Tensor,
+               dev_status: Optional[torch.Tensor] = None, stream=None):
+    c = cache.c()
+    _check("zha_decode", lib().zha_decode(
+        ctypes.byref(cfg), ctypes.byref(c), _ptr(q), float(p), _ptr(out), _ptr(level_counts),
+        _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream)))
+
+
+def zha_prefill_chunk(cfg: zha_config, cache: Cache, q: torch.Tensor, seq: int, chunk_start: int,
+                      p: float, out: torch.Tensor, level_counts: Optional[torch.Tensor],
+                      ws: torch.Tensor, dev_status: Optional[torch.Tensor] = None, stream=None):
+    c = cache.c()
+    _check("zha_prefill_chunk", lib().zha_prefill_chunk(
+        ctypes.byref(cfg), ctypes.byref(c), _ptr(q), seq, chunk_start, q.shape[0], float(p),
+        _ptr(out), _ptr(level_counts), _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream)))
+
+
+def zha_dense_decode(cfg: zha_config, cache: Cache, q: torch.Tensor, out: torch.Tensor,
+                     ws: torch.Tensor, stream=None):
+    c = cache.c()
+    _check("zha_dense_decode", lib().zha_dense_decode(
+        ctypes.byref(cfg), ctypes.byref(c), _ptr(q), _ptr(out), _ptr(ws), ws.numel(),
+        _stream(stream)))
+
+
+__all__ = [n for n in globals() if n.startswith("zha_")] + [
+    "lib", "Cache", "make_config", "alloc_tree", "alloc_workspace", "ZhaError", "EXPORTS",
+]

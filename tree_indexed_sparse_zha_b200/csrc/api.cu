@@ -1,0 +1,396 @@
+// libzha C-ABI entry points: argument validation, workspace layout, dispatch.
+// Every declaration lives in include/zha.h, which documents meaning, layout,
+// ownership and error behaviour of each argument.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <string.h>
+
+#include "zha_internal.h"
+
+namespace zha {
+
+static bool pow2_le8(int g) { return g == 1 || g == 2 || g == 4 || g == 8; }
+
+zha_status make_geometry(const zha_config* cfg, Geometry* g) {
+  if (!cfg || !g) return ZHA_ERR_INVALID_ARG;
+  memset(g, 0, sizeof(*g));
+  if (cfg->reserved != 0) return ZHA_ERR_INVALID_ARG;
+  if (cfg->dtype != ZHA_F32 && cfg->dtype != ZHA_BF16) return ZHA_ERR_INVALID_ARG;
+  if (cfg->head_dim != 64 && cfg->head_dim != 128) return ZHA_ERR_UNSUPPORTED;
+  const int b = cfg->block;
+  const bool small_b = b >= 2 && b <= 32 && (32 % b) == 0;
+  const bool large_b = b >= 64 && b <= 1024 && (b % 32) == 0;
+  if (!small_b && !large_b) return ZHA_ERR_UNSUPPORTED;
+  if (cfg->levels < 1 || cfg->levels > kMaxLevelsHost) return ZHA_ERR_INVALID_ARG;
+  if (cfg->n_kv_heads < 1 || cfg->n_q_heads < 1 || cfg->n_q_heads % cfg->n_kv_heads)
+    return ZHA_ERR_INVALID_ARG;
+  if (!pow2_le8(cfg->n_q_heads / cfg->n_kv_heads)) return ZHA_ERR_UNSUPPORTED;
+  if (cfg->batch < 1 || cfg->capacity < 1) return ZHA_ERR_INVALID_ARG;
+  g->d = cfg->head_dim;
+  g->b = b;
+  g->L = cfg->levels;
+  g->Hq = cfg->n_q_heads;
+  g->Hkv = cfg->n_kv_heads;
+  g->B = cfg->batch;
+  g->G = cfg->n_q_heads / cfg->n_kv_heads;
+  g->ncap = cfg->capacity;
+  g->dtype = cfg->dtype;
+  g->elem_bytes = cfg->dtype == ZHA_BF16 ? 2 : 4;
+  g->span[0] = 1;
+  for (int l = 1; l <= g->L; ++l) {
+    g->span[l] = g->span[l - 1] * b;
+    if (g->span[l] > ((int64_t)1 << 40)) return ZHA_ERR_INVALID_ARG;
+  }
+  // node ids travel in 24 bits next to an 8-bit head mask
+  if (g->ncap / b + 1 >= ((int64_t)1 << 24)) return ZHA_ERR_UNSUPPORTED;
+  int64_t off = 0;
+  for (int l = 1; l <= g->L; ++l) {
+    g->level_rows[l - 1] = g->ncap / g->span[l];
+    g->level_off[l - 1] = off;
+    off += (int64_t)g->B * g->Hkv * g->level_rows[l - 1] * g->d;
+    g->lnsize[l - 1] = (float)((double)l * log((double)b));
+  }
+  g->tree_elems = off;
+  g->inv_sqrt_d = (float)(1.0 / sqrt((double)g->d));
+  return ZHA_OK;
+}
+
+int device_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 148;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  return n;
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+static int check_p(double p, uint64_t* p_q) {
+  if (!(p > 0.0)) return 0;  // also rejects NaN
+  const double pc = p >= 1.0 ? 1.0 : p;
+  *p_q = (uint64_t)floor(pc * 4294967296.0 + 0.5);
+  return *p_q >= 1;
+}
+
+static zha_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ZHA_OK : ZHA_ERR_CUDA; }
+
+// ---- workspace layouts ----------------------------------------------------
+
+struct DecodeLayout {
+  size_t trav, kept, n_kept, part, total;
+  int64_t units;
+};
+
+static DecodeLayout decode_layout(const Geometry& g, int64_t nq, int kind, int sms) {
+  DecodeLayout L{};
+  L.units = nq * g.Hkv;
+  const int64_t max_cand = g.level_rows[0] + 1;
+  size_t off = 0;
+  L.trav = off;
+  off = align256(off + traverse_ws_bytes(g, L.units));
+  L.kept = off;
+  off = align256(off + sizeof(uint32_t) * (size_t)max_cand * L.units);
+  L.n_kept = off;
+  off = align256(off + sizeof(int32_t) * (size_t)L.units);
+  L.part = off;
+  off = align256(off + attend_ws_bytes(g, kind, nq, sms));
+  L.total = off;
+  return L;
+}
+
+// Prefill processes the chunk in tiles of query tokens sized to fill the GPU.
+static int64_t prefill_tile(const Geometry& g, int64_t T, int sms) {
+  int64_t t = (2 * (int64_t)sms) / g.Hkv;
+  if (t < 1) t = 1;
+  if (t > T) t = T;
+  return t;
+}
+
+struct PrefillLayout {
+  size_t old_len, q_seq, q_pos, dec, total;
+  int64_t tile;
+  DecodeLayout d;
+};
+
+static PrefillLayout prefill_layout(const Geometry& g, int64_t T, int sms) {
+  PrefillLayout P{};
+  P.tile = prefill_tile(g, T, sms);
+  size_t off = 0;
+  P.old_len = off;
+  off = align256(off + sizeof(int32_t) * (size_t)g.B);
+  P.q_seq = off;
+  off = align256(off + sizeof(int32_t) * (size_t)P.tile);
+  P.q_pos = off;
+  off = align256(off + sizeof(int32_t) * (size_t)P.tile);
+  P.dec = off;
+  P.d = decode_layout(g, P.tile, kStreamTree, sms);
+  off = align256(off + P.d.total);
+  P.total = off;
+  return P;
+}
+
+__global__ void fill_prefill_kernel(int32_t* old_len, const int32_t* seq_len, int B, int seq,
+                                    int64_t chunk_start) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < B) old_len[i] = (i == seq) ? (int32_t)chunk_start : seq_len[i];
+}
+
+__global__ void fill_positions_kernel(int32_t* q_seq, int32_t* q_pos, int seq, int64_t start,
+                                      int64_t count) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < count) {
+    q_seq[i] = seq;
+    q_pos[i] = (int32_t)(start + i);
+  }
+}
+
+}  // namespace zha
+
+using namespace zha;
+
+extern "C" {
+
+const char* zha_status_string(int32_t status) {
+  if (status == ZHA_OK) return "ok";
+  if (status & ZHA_ERR_INVALID_ARG) return "invalid argument";
+  if (status & ZHA_ERR_UNSUPPORTED) return "unsupported configuration";
+  if (status & ZHA_ERR_CUDA) return "CUDA error";
+  if (status & ZHA_ERR_CAPACITY) return "index list capacity exceeded";
+  if (status & ZHA_ERR_WORKSPACE) return "workspace too small";
+  if (status & ZHA_ERR_TIMEOUT) return "bounded wait timed out";
+  if (status & ZHA_ERR_INTERNAL) return "internal consistency check failed";
+  return "unknown status";
+}
+
+zha_status zha_tree_layout(const zha_config* cfg, size_t* tree_bytes, int64_t* level_offsets) {
+  Geometry g;
+  zha_status st = make_geometry(cfg, &g);
+  if (st != ZHA_OK) return st;
+  if (tree_bytes) *tree_bytes = (size_t)g.tree_elems * g.elem_bytes;
+  if (level_offsets)
+    for (int l = 0; l < g.L; ++l) level_offsets[l] = g.level_off[l];
+  return ZHA_OK;
+}
+
+zha_status zha_workspace_bytes(const zha_config* cfg, int32_t op, int64_t max_queries,
+                               size_t* bytes) {
+  Geometry g;
+  zha_status st = make_geometry(cfg, &g);
+  if (st != ZHA_OK) return st;
+  if (!bytes) return ZHA_ERR_INVALID_ARG;
+  const int sms = device_sm_count();
+  switch (op) {
+    case ZHA_OP_SELECT:
+      if (max_queries < 1) return ZHA_ERR_INVALID_ARG;
+      *bytes = align256(traverse_ws_bytes(g, max_queries * g.Hkv));
+      return ZHA_OK;
+    case ZHA_OP_ATTEND:
+      if (max_queries < 1) return ZHA_ERR_INVALID_ARG;
+      *bytes = align256(attend_ws_bytes(g, kStreamList, max_queries, sms));
+      return ZHA_OK;
+    case ZHA_OP_DECODE:
+      *bytes = decode_layout(g, g.B, kStreamTree, sms).total;
+      return ZHA_OK;
+    case ZHA_OP_DENSE:
+      *bytes = align256(attend_ws_bytes(g, kStreamDense, g.B, sms));
+      return ZHA_OK;
+    case ZHA_OP_PREFILL:
+      if (max_queries < 1) return ZHA_ERR_INVALID_ARG;
+      *bytes = prefill_layout(g, max_queries, sms).total;
+      return ZHA_OK;
+    default:
+      return ZHA_ERR_INVALID_ARG;
+  }
+}
+
+static zha_status check_cache(const zha_cache* c, bool need_kv) {
+  if (!c || !c->tree || !c->seq_len || !c->r) return ZHA_ERR_INVALID_ARG;
+  if (need_kv && (!c->k || !c->v)) return ZHA_ERR_INVALID_ARG;
+  if (!c->k) return ZHA_ERR_INVALID_ARG;
+  return ZHA_OK;
+}
+
+zha_status zha_build_tree(const zha_config* cfg, const zha_cache* cache, void* stream) {
+  Geometry g;
+  zha_status st = make_geometry(cfg, &g);
+  if (st != ZHA_OK) return st;
+  if ((st = check_cache(cache, false)) != ZHA_OK) return st;
+  return cuda_status(launch_tree(g, cache->k, cache->tree, cache->r, cache->seq_len, nullptr, -1,
+                                 (cudaStream_t)stream));
+}
+
+zha_status zha_extend_tree(const zha_config* cfg, const zha_cache* cache, const int32_t* old_len,
+                           int64_t max_new_tokens, void* stream) {
+  Geometry g;
+  zha_status st = make_geometry(cfg, &g);
+  if (st != ZHA_OK) return st;
+  if ((st = check_cache(cache, false)) != ZHA_OK) return st;
+  if (!old_len || max_new_tokens < 0) return ZHA_ERR_INVALID_ARG;
+  if (max_new_tokens == 0) return ZHA_OK;
+  return cuda_status(launch_tree(g, cache->k, cache->tree, cache->r, cache->seq_len, old_len,
+                                 max_new_tokens, (cudaStream_t)stream));
+}
+
+zha_status zha_select(const zha_config* cfg, const zha_cache* cache, const void* q,
+                      const int32_t* q_seq, const int32_t* q_pos, int64_t nq, double p,
+                      int32_t* idx, int64_t idx_cap, int32_t* n_idx, int32_t* level_counts,
+                      void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  Geometry g;
+  zha_status st = make_geometry(cfg, &g);
+  if (st != ZHA_OK) return st;
+  if ((st = check_cache(cache, false)) != ZHA_OK) return st;
+  uint64_t p_q;
+  if (!q || !q_seq || !q_pos || nq < 1 || !idx || idx_cap < 1 || !n_idx || !ws || !check_p(p, &p_q))
+    return ZHA_ERR_INVALID_ARG;
+  if (ws_bytes < traverse_ws_bytes(g, nq * g.Hkv)) return ZHA_ERR_WORKSPACE;
+  TraverseOut out{};
+  out.idx = idx;
+  out.idx_cap = idx_cap;
+  out.n_idx = n_idx;
+  out.level_counts = level_counts;
+  return cuda_status(launch_traverse(g, cache->tree, q, cache->seq_len, q_seq, q_pos, nq, p_q, 1,
+                                     out, ws, ws_bytes, dev_status, device_sm_count(),
+                                     (cudaStream_t)stream));
+}
+
+zha_status zha_attend(const zha_config* cfg, const zha_cache* cache, const void* q,
+                      const int32_t* q_seq, int64_t nq, const int32_t* idx, int64_t idx_cap,
+                      const int32_t* n_idx, void* out, void* ws, size_t ws_bytes,
+                      int32_t* dev_status, void* stream) {
+  (void)dev_status;
+  Geometry g;
+  zha_status st = make_geometry(cfg, &g);
+  if (st != ZHA_OK) return st;
+  if ((st = check_cache(cache, true)) != ZHA_OK) return st;
+  if (!q || !q_seq || nq < 1 || !idx || idx_cap < 1 || !n_idx || !out || !ws)
+    return ZHA_ERR_INVALID_ARG;
+  const int sms = device_sm_count();
+  if (ws_bytes < attend_ws_bytes(g, kStreamList, nq, sms)) return ZHA_ERR_WORKSPACE;
+  AttendArgs a{};
+  a.kind = kStreamList;
+  a.k = cache->k;
+  a.v = cache->v;
+  a.q = q;
+  a.out = out;
+  a.seq_len = cache->seq_len;
+  a.q_seq = q_seq;
+  a.nq = nq;
+  a.idx = idx;
+  a.idx_cap = idx_cap;
+  a.n_idx = n_idx;
+  return cuda_status(launch_attend(g, a, ws, ws_bytes, sms, (cudaStream_t)stream));
+}
+
+static zha_status run_tree_decode(const Geometry& g, const zha_cache* cache, const void* q,
+                                  const int32_t* q_seq, const int32_t* q_pos, int64_t nq,
+                                  uint64_t p_q, void* out, int32_t* level_counts,
+                                  unsigned char* ws, const DecodeLayout& L, int32_t* dev_status,
+                                  int sms, cudaStream_t s) {
+  TraverseOut to{};
+  to.kept = reinterpret_cast<uint32_t*>(ws + L.kept);
+  to.n_kept = reinterpret_cast<int32_t*>(ws + L.n_kept);
+  to.level_counts = level_counts;
+  cudaError_t e = launch_traverse(g, cache->tree, q, cache->seq_len, q_seq, q_pos, nq, p_q, 0, to,
+                                  ws + L.trav, L.kept - L.trav, dev_status, sms, s);
+  if (e != cudaSuccess) return ZHA_ERR_CUDA;
+  AttendArgs a{};
+  a.kind = kStreamTree;
+  a.k = cache->k;
+  a.v = cache->v;
+  a.q = q;
+  a.out = out;
+  a.seq_len = cache->seq_len;
+  a.q_seq = q_seq;
+  a.q_pos = q_pos;
+  a.nq = nq;
+  a.kept = to.kept;
+  a.n_kept = to.n_kept;
+  a.kept_stride = g.level_rows[0] + 1;
+  return cuda_status(launch_attend(g, a, ws + L.part, L.total - L.part, sms, s));
+}
+
+zha_status zha_decode(const zha_config* cfg, const zha_cache* cache, const void* q, double p,
+                      void* out, int32_t* level_counts, void* ws, size_t ws_bytes,
+                      int32_t* dev_status, void* stream) {
+  Geometry g;
+  zha_status st = make_geometry(cfg, &g);
+  if (st != ZHA_OK) return st;
+  if ((st = check_cache(cache, true)) != ZHA_OK) return st;
+  uint64_t p_q;
+  if (!q || !out || !ws || !check_p(p, &p_q)) return ZHA_ERR_INVALID_ARG;
+  const int sms = device_sm_count();
+  const DecodeLayout L = decode_layout(g, g.B, kStreamTree, sms);
+  if (ws_bytes < L.total) return ZHA_ERR_WORKSPACE;
+  return run_tree_decode(g, cache, q, nullptr, nullptr, g.B, p_q, out, level_counts,
+                         static_cast<unsigned char*>(ws), L, dev_status, sms,
+                         (cudaStream_t)stream);
+}
+
+zha_status zha_prefill_chunk(const zha_config* cfg, const zha_cache* cache, const void* q,
+                             int32_t seq, int64_t chunk_start, int64_t T, double p, void* out,
+                             int32_t* level_counts, void* ws, size_t ws_bytes,
+                             int32_t* dev_status, void* stream) {
+  Geometry g;
+  zha_status st = make_geometry(cfg, &g);
+  if (st != ZHA_OK) return st;
+  if ((st = check_cache(cache, true)) != ZHA_OK) return st;
+  uint64_t p_q;
+  if (!q || !out || !ws || T < 1 || seq < 0 || seq >= g.B || chunk_start < 0 ||
+      chunk_start + T > g.ncap || !check_p(p, &p_q))
+    return ZHA_ERR_INVALID_ARG;
+  const int sms = device_sm_count();
+  const PrefillLayout P = prefill_layout(g, T, sms);
+  if (ws_bytes < P.total) return ZHA_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  int32_t* old_len = reinterpret_cast<int32_t*>(w + P.old_len);
+  int32_t* q_seq = reinterpret_cast<int32_t*>(w + P.q_seq);
+  int32_t* q_pos = reinterpret_cast<int32_t*>(w + P.q_pos);
+  fill_prefill_kernel<<<(g.B + 127) / 128, 128, 0, s>>>(old_len, cache->seq_len, g.B, seq,
+                                                       chunk_start);
+  if (cudaGetLastError() != cudaSuccess) return ZHA_ERR_CUDA;
+  cudaError_t e = launch_tree(g, cache->k, cache->tree, cache->r, cache->seq_len, old_len, T, s);
+  if (e != cudaSuccess) return ZHA_ERR_CUDA;
+  const size_t row_bytes = (size_t)g.Hq * g.d * g.elem_bytes;
+  for (int64_t i0 = 0; i0 < T; i0 += P.tile) {
+    const int64_t n = (T - i0) < P.tile ? (T - i0) : P.tile;
+    fill_positions_kernel<<<(unsigned)((n + 127) / 128), 128, 0, s>>>(q_seq, q_pos, seq,
+                                                                      chunk_start + i0, n);
+    if (cudaGetLastError() != cudaSuccess) return ZHA_ERR_CUDA;
+    const DecodeLayout L = decode_layout(g, n, kStreamTree, sms);
+    st = run_tree_decode(g, cache, static_cast<const unsigned char*>(q) + i0 * row_bytes, q_seq,
+                         q_pos, n, p_q, static_cast<unsigned char*>(out) + i0 * row_bytes,
+                         level_counts ? level_counts + i0 * g.Hq * g.L : nullptr, w + P.dec, L,
+                         dev_status, sms, s);
+    if (st != ZHA_OK) return st;
+  }
+  return ZHA_OK;
+}
+
+zha_status zha_dense_decode(const zha_config* cfg, const zha_cache* cache, const void* q,
+                            void* out, void* ws, size_t ws_bytes, void* stream) {
+  Geometry g;
+  zha_status st = make_geometry(cfg, &g);
+  if (st != ZHA_OK) return st;
+  if (!cache || !cache->k || !cache->v || !cache->seq_len || !q || !out || !ws)
+    return ZHA_ERR_INVALID_ARG;
+  const int sms = device_sm_count();
+  if (ws_bytes < attend_ws_bytes(g, kStreamDense, g.B, sms)) return ZHA_ERR_WORKSPACE;
+  AttendArgs a{};
+  a.kind = kStreamDense;
+  a.k = cache->k;
+  a.v = cache->v;
+  a.q = q;
+  a.out = out;
+  a.seq_len = cache->seq_len;
+  a.nq = g.B;
+  return cuda_status(launch_attend(g, a, ws, ws_bytes, sms, (cudaStream_t)stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,90 @@
+// Host-side internal interfaces of libzha (not part of the public C-ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/zha.h"
+
+namespace zha {
+
+constexpr int kMaxLevelsHost = 8;
+
+// Geometry derived once per call from a zha_config.
+struct Geometry {
+  int d, b, L, Hq, Hkv, B, G;
+  int64_t ncap;
+  int dtype;               // zha_dtype
+  int64_t span[kMaxLevelsHost + 1];        // b^l, l = 0..L
+  int64_t level_rows[kMaxLevelsHost];      // rows per unit of level l at index l-1
+  int64_t level_off[kMaxLevelsHost];       // element offset of level l at index l-1
+  int64_t tree_elems;
+  float inv_sqrt_d;
+  float lnsize[kMaxLevelsHost];            // fp32(l ln b) at index l-1
+  int elem_bytes;
+};
+
+zha_status make_geometry(const zha_config* cfg, Geometry* g);
+
+// ---- tree build -----------------------------------------------------------
+// old_len == nullptr builds every complete node; otherwise nodes completed in
+// (old_len, seq_len]. max_new_tokens < 0 means "whole sequence".
+cudaError_t launch_tree(const Geometry& g, const void* k, void* tree, const float* r,
+                        const int32_t* seq_len, const int32_t* old_len, int64_t max_new_tokens,
+                        cudaStream_t stream);
+
+// ---- traversal ------------------------------------------------------------
+struct TraverseOut {
+  // decode mode: per unit, the union of kept level-1 nodes with per-head masks
+  uint32_t* kept;          // [units][max_cand] packed (mask << 24) | node
+  int32_t* n_kept;         // [units]
+  // list mode: per query head, the selected token list
+  int32_t* idx;            // [nq][Hq][idx_cap]
+  int64_t idx_cap;
+  int32_t* n_idx;          // [nq][Hq]
+  int32_t* level_counts;   // [nq][Hq][L] (nullable)
+};
+
+// Workspace bytes the traversal needs for `units` (query token, KV head) units:
+// two candidate lists and the G score arrays per unit.
+size_t traverse_ws_bytes(const Geometry& g, int64_t units);
+
+// Decode mode: query token = sequence s at position seq_len[s]-1, q [B][Hq][d].
+// List mode: query token i at (q_seq[i], q_pos[i]), q [nq][Hq][d].
+cudaError_t launch_traverse(const Geometry& g, const void* tree, const void* q,
+                            const int32_t* seq_len, const int32_t* q_seq, const int32_t* q_pos,
+                            int64_t nq, uint64_t p_q, int list_mode, const TraverseOut& out,
+                            void* ws, size_t ws_bytes, int32_t* status, int num_sms,
+                            cudaStream_t stream);
+
+// ---- attention ------------------------------------------------------------
+enum StreamKind { kStreamTree = 0, kStreamDense = 1, kStreamList = 2 };
+
+struct AttendArgs {
+  int kind;                      // StreamKind
+  const void* k;
+  const void* v;
+  const void* q;                 // tree/dense: [B][Hq][d]; list: [nq][Hq][d]
+  void* out;                     // same shape as q
+  const int32_t* seq_len;        // [B]
+  const int32_t* q_seq;          // list mode / explicit positions: [nq]
+  const int32_t* q_pos;          // tree stream with explicit positions (prefill), else null
+  int64_t nq;                    // query tokens (decode/dense: B)
+  // tree stream
+  const uint32_t* kept;          // [units][kept_stride]
+  const int32_t* n_kept;         // [units]
+  int64_t kept_stride;
+  // list stream
+  const int32_t* idx;
+  int64_t idx_cap;
+  const int32_t* n_idx;
+};
+
+size_t attend_ws_bytes(const Geometry& g, int kind, int64_t nq, int num_sms);
+
+cudaError_t launch_attend(const Geometry& g, const AttendArgs& a, void* ws, size_t ws_bytes,
+                          int num_sms, cudaStream_t stream);
+
+int device_sm_count();
+
+}  // namespace zha
