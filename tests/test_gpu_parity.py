@@ -184,3 +184,16 @@ def test_decode_wide_256k_full_size_sampled():
     wl = W.make("decode-wide-256k-b8", device="cuda")
     wl.K, wl.V, wl.R = wl.K.cpu(), wl.V.cpu(), wl.R.cpu()
     _run_decode_case(wl, units=[3], heads=list(range(16)), check_tree_units=[(3, 0), (3, 1)])
+
+
+def test_zero_query_all_ties():
+    """q = 0: every node of a level has the same score, so each cut is decided
+    purely by the lower-node-index rule (ordered tie ranks)."""
+    wl = W.make("decode-deep-32k", n_tokens=20000)
+    c = wl.cfg
+    gpu = Gpu(wl)
+    ref = Ref(wl, c.n_tokens)
+    _decode_parity.gpu, _decode_parity.ref = gpu, ref
+    q = torch.zeros_like(wl.queries(0))
+    for p in (0.3, 0.95):
+        _decode_parity(wl, q, p, c.n_tokens)

@@ -90,14 +90,13 @@ struct DecodeLayout {
 static DecodeLayout decode_layout(const Geometry& g, int64_t nq, int kind, int sms) {
   DecodeLayout L{};
   L.units = nq * g.Hkv;
-  const int64_t max_cand = g.level_rows[0] + 1;
   size_t off = 0;
   L.trav = off;
-  off = align256(off + traverse_ws_bytes(g, L.units));
+  off = align256(off + traverse_ws_bytes(g, L.units, sms));
   L.kept = off;
-  off = align256(off + sizeof(uint32_t) * (size_t)max_cand * L.units);
+  off = align256(off + traverse_kept_bytes(g, L.units, sms));
   L.n_kept = off;
-  off = align256(off + sizeof(int32_t) * (size_t)L.units);
+  off = align256(off + sizeof(int32_t) * (size_t)L.units * kMaxClusterHost);
   L.part = off;
   off = align256(off + attend_ws_bytes(g, kind, nq, sms));
   L.total = off;
@@ -188,7 +187,7 @@ zha_status zha_workspace_bytes(const zha_config* cfg, int32_t op, int64_t max_qu
   switch (op) {
     case ZHA_OP_SELECT:
       if (max_queries < 1) return ZHA_ERR_INVALID_ARG;
-      *bytes = align256(traverse_ws_bytes(g, max_queries * g.Hkv));
+      *bytes = align256(traverse_ws_bytes(g, max_queries * g.Hkv, sms));
       return ZHA_OK;
     case ZHA_OP_ATTEND:
       if (max_queries < 1) return ZHA_ERR_INVALID_ARG;
@@ -248,15 +247,15 @@ zha_status zha_select(const zha_config* cfg, const zha_cache* cache, const void*
   uint64_t p_q;
   if (!q || !q_seq || !q_pos || nq < 1 || !idx || idx_cap < 1 || !n_idx || !ws || !check_p(p, &p_q))
     return ZHA_ERR_INVALID_ARG;
-  if (ws_bytes < traverse_ws_bytes(g, nq * g.Hkv)) return ZHA_ERR_WORKSPACE;
+  const int sms = device_sm_count();
+  if (ws_bytes < traverse_ws_bytes(g, nq * g.Hkv, sms)) return ZHA_ERR_WORKSPACE;
   TraverseOut out{};
   out.idx = idx;
   out.idx_cap = idx_cap;
   out.n_idx = n_idx;
   out.level_counts = level_counts;
   return cuda_status(launch_traverse(g, cache->tree, q, cache->seq_len, q_seq, q_pos, nq, p_q, 1,
-                                     out, ws, ws_bytes, dev_status, device_sm_count(),
-                                     (cudaStream_t)stream));
+                                     out, ws, ws_bytes, dev_status, sms, (cudaStream_t)stream));
 }
 
 zha_status zha_attend(const zha_config* cfg, const zha_cache* cache, const void* q,
@@ -311,7 +310,8 @@ static zha_status run_tree_decode(const Geometry& g, const zha_cache* cache, con
   a.nq = nq;
   a.kept = to.kept;
   a.n_kept = to.n_kept;
-  a.kept_stride = g.level_rows[0] + 1;
+  a.kept_stride = traverse_kept_stride(g);
+  a.kept_segs = traverse_cluster_size(g, L.units, sms);
   return cuda_status(launch_attend(g, a, ws + L.part, L.total - L.part, sms, s));
 }
 

@@ -49,6 +49,7 @@ struct AttParams {
   const uint32_t* kept;
   const int32_t* n_kept;
   int64_t kept_stride;
+  int kept_segs;
   // list stream
   const int32_t* idx;
   int64_t idx_cap;
@@ -76,7 +77,9 @@ struct Span {
   int64_t t0, t1;       // tail rows (tree) / dense rows / list positions
   int64_t tail_start;
   int64_t rows;
-  const uint32_t* kept;
+  const uint32_t* kept;        // segment 0 of the unit
+  const unsigned int* segbase; // [segs + 1] prefix of segment sizes (shared memory)
+  int64_t stride;
   const int32_t* list;
 };
 
@@ -92,7 +95,10 @@ __device__ __forceinline__ void row_of(const AttParams& p, const Span& s, int64_
     v -= s.tok0;
     const int64_t nrows = (s.n1 - s.n0) * p.b;
     if (v < nrows) {
-      const uint32_t e = s.kept[s.n0 + v / p.b];
+      const int64_t j = s.n0 + v / p.b;
+      int r = 0;
+      while ((int64_t)s.segbase[r + 1] <= j) ++r;
+      const uint32_t e = s.kept[r * s.stride + (j - s.segbase[r])];
       const int64_t node = e & 0x00ffffffu;
       const int off = (int)(v % p.b);
       *row = node * p.b + off;
@@ -119,6 +125,7 @@ __global__ void __launch_bounds__(Cfg<T, D>::kThreads, 1) attend_kernel(AttParam
   constexpr int kPer = Elem<T>::kPerChunk;
   constexpr int kDL = C::kDimsPerLane;
   extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ unsigned int s_segbase[kMaxCluster + 1];
   float* qs = reinterpret_cast<float*>(smem);                       // [D][8]
   unsigned char* wbase = smem + D * kMaxGroup * sizeof(float);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -169,8 +176,19 @@ __global__ void __launch_bounds__(Cfg<T, D>::kThreads, 1) attend_kernel(AttParam
       const int64_t T_top = (t + 1) / p.span_L;
       s.tail_start = p.span_L * T_top;
       const int64_t tail_len = t + 1 - s.tail_start;
-      const int64_t nk = T_top > 0 ? p.n_kept[unit] : 0;
-      s.kept = p.kept + (int64_t)unit * p.kept_stride;
+      if (tid == 0) {
+        unsigned int acc = 0;
+        for (int r = 0; r < p.kept_segs; ++r) {
+          s_segbase[r] = acc;
+          acc += T_top > 0 ? (unsigned int)p.n_kept[(int64_t)unit * p.kept_segs + r] : 0u;
+        }
+        s_segbase[p.kept_segs] = acc;
+      }
+      __syncthreads();
+      const int64_t nk = s_segbase[p.kept_segs];
+      s.kept = p.kept + (int64_t)unit * p.kept_segs * p.kept_stride;
+      s.segbase = s_segbase;
+      s.stride = p.kept_stride;
       s.tok0 = (T_top > 0 && split == 0) ? 1 : 0;
       s.n0 = nk * split / p.S;
       s.n1 = nk * (split + 1) / p.S;
@@ -440,6 +458,7 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads, 1) attend_mma_kernel(AttP
   using C = MmaCfg<D>;
   using T = __nv_bfloat16;
   extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ unsigned int s_segbase[kMaxCluster + 1];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t4 = lane & 3;   // MMA fragment coordinates
   unsigned char* my = smem + warp * C::kWarpBytes;
@@ -471,8 +490,19 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads, 1) attend_mma_kernel(AttP
     const int64_t T_top = (t + 1) / p.span_L;
     s.tail_start = p.span_L * T_top;
     const int64_t tail_len = t + 1 - s.tail_start;
-    const int64_t nk = T_top > 0 ? p.n_kept[unit] : 0;
-    s.kept = p.kept + (int64_t)unit * p.kept_stride;
+    if (tid == 0) {
+      unsigned int acc = 0;
+      for (int r = 0; r < p.kept_segs; ++r) {
+        s_segbase[r] = acc;
+        acc += T_top > 0 ? (unsigned int)p.n_kept[(int64_t)unit * p.kept_segs + r] : 0u;
+      }
+      s_segbase[p.kept_segs] = acc;
+    }
+    __syncthreads();
+    const int64_t nk = s_segbase[p.kept_segs];
+    s.kept = p.kept + (int64_t)unit * p.kept_segs * p.kept_stride;
+    s.segbase = s_segbase;
+    s.stride = p.kept_stride;
     s.tok0 = (T_top > 0 && split == 0) ? 1 : 0;
     s.n0 = nk * split / p.S;
     s.n1 = nk * (split + 1) / p.S;
@@ -507,23 +537,30 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads, 1) attend_mma_kernel(AttP
   auto issue = [&](int64_t blk, int stage) {
     const int64_t v = blk * 32 + lane;
     uint32_t m = 0;
+    int64_t row = 0;
     if (blk < nblk && v < s.rows) {
-      int64_t row;
       row_of(p, s, v, &row, &m, all);
       if (row < 0 || row >= p.ncap) m = 0u;
-      if (m) {
-        unsigned char* kd = my + stage * C::kStageBytes + lane * C::kRowBytes;
-        unsigned char* vd = kd + 32 * C::kRowBytes;
-        const unsigned char* ks = reinterpret_cast<const unsigned char*>(kbase + row * D);
-        const unsigned char* vs = reinterpret_cast<const unsigned char*>(vbase + row * D);
-#pragma unroll
-        for (int c = 0; c < C::kRowBytes / 16; ++c) {
-          cp_async16(kd + swz(c, lane) * 16, ks + c * 16);
-          cp_async16(vd + swz(c, lane) * 16, vs + c * 16);
-        }
-      }
     }
     rmask[stage * 32 + lane] = (uint8_t)m;
+    // every instruction moves whole rows: lanes 16j..16j+15 copy the 16-byte
+    // chunks of one row, so each warp request is a few full 128-byte lines
+    constexpr int kCh = C::kRowBytes / 16;   // chunks per row (8 or 16)
+    constexpr int kRowsPerInstr = 32 / kCh;  // rows per warp instruction
+    const int c = lane % kCh;
+    unsigned char* st = my + stage * C::kStageBytes;
+#pragma unroll
+    for (int i = 0; i < 32 / kRowsPerInstr; ++i) {
+      const int r = i * kRowsPerInstr + lane / kCh;
+      const int64_t rr = __shfl_sync(0xffffffffu, row, r);
+      const uint32_t mm = __shfl_sync(0xffffffffu, m, r);
+      if (mm) {
+        const int64_t off = rr * C::kRowBytes + c * 16;
+        const int dst = r * C::kRowBytes + swz(c, r) * 16;
+        cp_async16(st + dst, reinterpret_cast<const unsigned char*>(kbase) + off);
+        cp_async16(st + 32 * C::kRowBytes + dst, reinterpret_cast<const unsigned char*>(vbase) + off);
+      }
+    }
     cp_async_commit();
   };
 
@@ -727,7 +764,8 @@ int64_t units_of(const Geometry& g, int kind, int64_t nq) {
 
 int splits_of(const Geometry& g, int kind, int64_t nq, int num_sms) {
   const int64_t units = units_of(g, kind, nq);
-  int64_t S = (2 * (int64_t)num_sms + units - 1) / units;
+  // about two CTAs per SM in total, rounded down so the last wave is full
+  int64_t S = (2 * (int64_t)num_sms) / units;
   if (S < 1) S = 1;
   if (S > 256) S = 256;
   return (int)S;
@@ -765,6 +803,7 @@ cudaError_t launch_attend(const Geometry& g, const AttendArgs& a, void* ws, size
   p.kept = a.kept;
   p.n_kept = a.n_kept;
   p.kept_stride = a.kept_stride;
+  p.kept_segs = a.kept_segs;
   p.idx = a.idx;
   p.idx_cap = a.idx_cap;
   p.n_idx = a.n_idx;

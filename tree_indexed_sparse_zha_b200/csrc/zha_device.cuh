@@ -14,6 +14,7 @@ namespace zha {
 constexpr int kNRef = 16;         // reference queries per node summary
 constexpr int kMaxLevels = 8;
 constexpr int kMaxGroup = 8;      // query heads per KV head
+constexpr int kMaxCluster = 16;   // CTAs cooperating on one traversal unit
 
 // ---------------------------------------------------------------------------
 // canonical arithmetic

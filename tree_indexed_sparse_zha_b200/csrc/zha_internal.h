@@ -9,6 +9,7 @@
 namespace zha {
 
 constexpr int kMaxLevelsHost = 8;
+constexpr int kMaxClusterHost = 16;  // upper bound of traverse_cluster_size()
 
 // Geometry derived once per call from a zha_config.
 struct Geometry {
@@ -35,9 +36,10 @@ cudaError_t launch_tree(const Geometry& g, const void* k, void* tree, const floa
 
 // ---- traversal ------------------------------------------------------------
 struct TraverseOut {
-  // decode mode: per unit, the union of kept level-1 nodes with per-head masks
-  uint32_t* kept;          // [units][max_cand] packed (mask << 24) | node
-  int32_t* n_kept;         // [units]
+  // decode mode: per unit, the union of kept level-1 nodes with per-head masks,
+  // as C ordered segments (C = traverse_cluster_size) of traverse_kept_stride
+  uint32_t* kept;          // [units][C][stride] packed (mask << 24) | node
+  int32_t* n_kept;         // [units][C]
   // list mode: per query head, the selected token list
   int32_t* idx;            // [nq][Hq][idx_cap]
   int64_t idx_cap;
@@ -45,12 +47,17 @@ struct TraverseOut {
   int32_t* level_counts;   // [nq][Hq][L] (nullable)
 };
 
-// Workspace bytes the traversal needs for `units` (query token, KV head) units:
-// two candidate lists and the G score arrays per unit.
-size_t traverse_ws_bytes(const Geometry& g, int64_t units);
+// CTAs per traversal cluster for `units` (query token, KV head) units.
+int traverse_cluster_size(const Geometry& g, int64_t units, int num_sms);
+// Scratch bytes of the traversal (candidate segments, scores, keep bits).
+size_t traverse_ws_bytes(const Geometry& g, int64_t units, int num_sms);
+// Bytes of the decode-mode kept list and its per-segment stride (entries).
+size_t traverse_kept_bytes(const Geometry& g, int64_t units, int num_sms);
+int64_t traverse_kept_stride(const Geometry& g);
 
-// Decode mode: query token = sequence s at position seq_len[s]-1, q [B][Hq][d].
-// List mode: query token i at (q_seq[i], q_pos[i]), q [nq][Hq][d].
+// Decode mode (q_pos == nullptr): query token = sequence s at position
+// seq_len[s]-1, q [B][Hq][d]. Otherwise query token i at (q_seq[i], q_pos[i]),
+// q [nq][Hq][d]. list_mode selects the per-head index-list output.
 cudaError_t launch_traverse(const Geometry& g, const void* tree, const void* q,
                             const int32_t* seq_len, const int32_t* q_seq, const int32_t* q_pos,
                             int64_t nq, uint64_t p_q, int list_mode, const TraverseOut& out,
@@ -70,10 +77,11 @@ struct AttendArgs {
   const int32_t* q_seq;          // list mode / explicit positions: [nq]
   const int32_t* q_pos;          // tree stream with explicit positions (prefill), else null
   int64_t nq;                    // query tokens (decode/dense: B)
-  // tree stream
-  const uint32_t* kept;          // [units][kept_stride]
-  const int32_t* n_kept;         // [units]
+  // tree stream: kept level-1 nodes as kept_segs ordered segments per unit
+  const uint32_t* kept;          // [units][kept_segs][kept_stride]
+  const int32_t* n_kept;         // [units][kept_segs]
   int64_t kept_stride;
+  int kept_segs;
   // list stream
   const int32_t* idx;
   int64_t idx_cap;
