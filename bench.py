@@ -1,0 +1,427 @@
+#!/usr/bin/env python
+"""Decode benchmark of the ZHA hot path on B200.
+
+Workload (default): the 256K-context deep-tree decode run -- 8 sequences, 16
+query / 2 KV heads, d = 128, 262,144 cached tokens, tree of blocks of 4 over 6
+levels, p = 0.95. One step appends one token per sequence and runs
+zha_extend_tree + the traversal + sparse attention for all 128 (sequence,
+head) queries. Inputs are synthetic (seeded Gaussian-mixture keys with planted
+needles) and resident in HBM; K+V (2.15 GB) is larger than L2, so no flush is
+needed between steps.
+
+One JSON line on rank 0. Under torchrun every rank runs an independent replica
+(weak scaling, no data-path collective); timing is the max over ranks.
+--impl reference times the CPU oracle on the same metric (a bounded sample).
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+WORKLOAD = "decode-deep-256k-b8"
+METRIC = "ZHA decode queries/s at 256K ctx (B=8, p=0.95); % of HBM roofline"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="zha", choices=["zha", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("traverse.cu", "attend.cu", "zha_device.cuh"):
+        with open(os.path.join(ROOT, "tree_indexed_sparse_zha_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "decode-deep-256k-b8_traffic.txt")
+    try:
+        vals = {}
+        with open(path) as f:
+            for ln in f:
+                if ":" in ln and not ln.startswith("#"):
+                    k, v = ln.split(":", 1)
+                    vals[k.strip()] = v.strip()
+        if vals.get("kernel_source_hash") != kernel_source_hash():
+            return None
+        return vals
+    except OSError:
+        return None
+
+
+# ---------------------------------------------------------------------------
+# oracle CPU baseline (rank 0, bounded sample)
+# ---------------------------------------------------------------------------
+
+def oracle_rate(wl, n_queries: int, budget_s: float = 20.0):
+    """Times the CPU oracle (tree for one (sequence, KV head) built untimed, then
+    select + fp64 attention per query) on decode steps of that unit."""
+    import numpy as np
+
+    import oracle
+
+    c = wl.cfg
+    K = wl.K[0, 0].float().cpu().numpy()
+    V = wl.V[0, 0].float().cpu().numpy()
+    R = wl.R.float().cpu().numpy()
+    tr = oracle.build_tree(K, c.n_tokens, R, c.block, c.levels, True, c.capacity)
+    done = 0
+    t0 = time.perf_counter()
+    step = 1
+    while done < n_queries and time.perf_counter() - t0 < budget_s:
+        q = wl.queries(step)[0].float().cpu().numpy()
+        t = c.n_tokens + step - 1
+        for h in range(c.group):
+            idx, _, _, _ = oracle.select(q[h], tr, t, c.p)
+            oracle.attend(q[h], K, V, idx)
+            done += 1
+            if done >= n_queries:
+                break
+        step += 1
+    el = time.perf_counter() - t0
+    return done / el, done, el
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+
+def run_zha(args, rank, world, dev):
+    import tree_indexed_sparse_zha_b200 as z
+    from tree_indexed_sparse_zha_b200 import workloads as W
+
+    z.lib()  # fail loudly if the extension is missing
+    wl = W.make(args.workload, device=dev)
+    c = wl.cfg
+    n_steps_cap = c.steps
+    cfg = z.make_config(c.head_dim, c.block, c.levels, c.n_q_heads, c.n_kv_heads, c.batch,
+                        c.capacity, c.torch_dtype)
+    B, Hq, Hkv, D, b, L = c.batch, c.n_q_heads, c.n_kv_heads, c.head_dim, c.block, c.levels
+    # per-step lengths and queries are precomputed inputs (resident in HBM)
+    lens = (c.n_tokens + torch.arange(n_steps_cap + 1, device=dev, dtype=torch.int32))
+    lens = lens.view(-1, 1).expand(-1, B).contiguous()           # [step][B]
+    queries = torch.stack([wl.queries(s) for s in range(1, n_steps_cap + 1)])  # [step][B][Hq][D]
+    tree = z.alloc_tree(cfg, dev)
+    cache = z.Cache(wl.K, wl.V, wl.R.float().contiguous(), tree, lens[0])
+    ws = z.alloc_workspace(cfg, z.ZHA_OP_DECODE, device=dev)
+    wsd = z.alloc_workspace(cfg, z.ZHA_OP_DENSE, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    out = torch.empty(B, Hq, D, dtype=c.torch_dtype, device=dev)
+    stream = torch.cuda.current_stream()
+
+    # ---- tree build (rate reported; not part of a decode step) ----
+    z.zha_build_tree(cfg, cache)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+    e0.record()
+    z.zha_build_tree(cfg, cache)
+    e1.record()
+    torch.cuda.synchronize()
+    build_ms = e0.elapsed_time(e1)
+    n_tok = B * Hkv * c.n_tokens
+    sum_rows = sum(B * Hkv * (c.n_tokens // b ** l) for l in range(1, L + 1))
+    build_bytes = (n_tok + sum_rows * 2 - B * Hkv * (c.n_tokens // b ** L)) * D * 2
+    build_flops = 2.0 * 16 * D * (n_tok + sum_rows - B * Hkv * (c.n_tokens // b ** L))
+
+    def step_inputs(i):
+        s = (i % n_steps_cap) + 1  # wrap: rebuilt nodes are identical
+        return s, lens[s - 1], lens[s], queries[s - 1]
+
+    def one_step(i, ev=None):
+        s, old, new, q = step_inputs(i)
+        cache.seq_len = new
+        if ev:
+            ev[0].record(stream)
+        z.zha_extend_tree(cfg, cache, old, 1)
+        if ev:
+            ev[1].record(stream)
+        z.zha_decode_select(cfg, cache, q, c.p, None, ws, st)
+        if ev:
+            ev[2].record(stream)
+        z.zha_decode_attend(cfg, cache, q, out, ws)
+        if ev:
+            ev[3].record(stream)
+
+    # reset the tree to the initial length, then warm up
+    cache.seq_len = lens[0]
+    z.zha_build_tree(cfg, cache)
+    for i in range(args.warmup):
+        one_step(i)
+    torch.cuda.synchronize()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {z.status_string(int(st.item()))}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(True), torch.cuda.Event(True)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    t_start.record(stream)
+    for i in range(args.steps):
+        one_step(args.warmup + i, evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    ms_total = t_start.elapsed_time(t_end)
+    ms_ext = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    ms_sel = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    ms_att = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+    if world > 1:
+        tt = torch.tensor([ms_total], device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / args.steps
+    queries_per_step = B * Hq
+    value = queries_per_step * args.steps * world / (ms_total / 1e3)
+
+    # ---- bytes touched per step (work counters of the last timed step) ----
+    stats = torch.zeros(B * Hkv, L + 1, dtype=torch.int32, device=dev)
+    z.zha_decode_stats(cfg, ws, stats)
+    torch.cuda.synchronize()
+    stats = stats.cpu()
+    s_last, _, new_last, _ = step_inputs(args.warmup + args.steps - 1)
+    n_last = int(new_last[0].item())
+    top = n_last // b ** L
+    tail = n_last - b ** L * top
+    row = D * 2
+    cand_rows = int(stats[:, :L].sum())
+    kept_nodes = int(stats[:, L].sum())
+    kv_rows = kept_nodes * b + B * Hkv * (1 + tail)
+    sel_bytes = cand_rows * row + kept_nodes * 4 + 2 * queries_per_step * row
+    att_bytes = kv_rows * 2 * row + kept_nodes * 4 + 2 * queries_per_step * row
+    ext_bytes = 0
+    step_bytes = sel_bytes + att_bytes + ext_bytes
+    peak, peak_kind = measured_peaks()
+    hbm_frac = step_bytes / (ms_step / 1e3) / 1e9 / peak
+
+    # ---- dense flash-decoding from the same library, same step inputs ----
+    nd = min(20, args.steps)
+    z.zha_dense_decode(cfg, cache, queries[0], out, wsd)
+    torch.cuda.synchronize()
+    e0.record()
+    for i in range(nd):
+        z.zha_dense_decode(cfg, cache, queries[i % n_steps_cap], out, wsd)
+    e1.record()
+    torch.cuda.synchronize()
+    dense_ms = e0.elapsed_time(e1) / nd
+    dense_bytes = B * Hkv * n_last * 2 * row + 2 * queries_per_step * row
+
+    # ---- end to end through the API with host buffers ----
+    ne = min(50, args.steps)
+    kv_host = torch.empty(ne, 2, B, Hkv, D, dtype=c.torch_dtype).pin_memory()
+    q_host = torch.empty(ne, B, Hq, D, dtype=c.torch_dtype).pin_memory()
+    for i in range(ne):
+        s, _, _, q = step_inputs(i)
+        kv_host[i, 0].copy_(wl.K[:, :, c.n_tokens + s - 1])
+        kv_host[i, 1].copy_(wl.V[:, :, c.n_tokens + s - 1])
+        q_host[i].copy_(q)
+    out_host = torch.empty(ne, B, Hq, D, dtype=c.torch_dtype).pin_memory()
+    kv_dev = torch.empty(2, B, Hkv, D, dtype=c.torch_dtype, device=dev)
+    q_dev = torch.empty(B, Hq, D, dtype=c.torch_dtype, device=dev)
+    cache.seq_len = lens[0]
+    z.zha_build_tree(cfg, cache)
+    torch.cuda.synchronize()
+    e0.record()
+    for i in range(ne):
+        s, old, new, _ = step_inputs(i)
+        kv_dev.copy_(kv_host[i], non_blocking=True)
+        q_dev.copy_(q_host[i], non_blocking=True)
+        wl.K[:, :, c.n_tokens + s - 1] = kv_dev[0]
+        wl.V[:, :, c.n_tokens + s - 1] = kv_dev[1]
+        cache.seq_len = new
+        z.zha_extend_tree(cfg, cache, old, 1)
+        z.zha_decode(cfg, cache, q_dev, c.p, out, None, ws, st)
+        out_host[i].copy_(out, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / ne
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    h2d = kv_host[0].numel() * kv_host.element_size() + q_host[0].numel() * q_host.element_size()
+    d2h = out_host[0].numel() * out_host.element_size()
+
+    # ---- roofline of the dominant kernel group ----
+    traffic = recorded_traffic()
+    if ms_att >= ms_sel:
+        roof = {"kernel": "attend_mma_kernel + combine (zha_decode_attend)", "bound": "hbm",
+                "achieved": att_bytes / (ms_att / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                "peak_kind": peak_kind}
+        roof["traffic"] = float(traffic["attend_dram_bytes_per_launch"]) if traffic else None
+    else:
+        roof = {"kernel": "traverse_kernel (zha_decode_select)", "bound": "hbm",
+                "achieved": sel_bytes / (ms_sel / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                "peak_kind": peak_kind}
+        roof["traffic"] = float(traffic["traverse_dram_bytes_per_launch"]) if traffic else None
+    roof["frac"] = roof["achieved"] / roof["peak"]
+
+    res = {
+        "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Gaussian-mixture keys, planted needles; no dataset)",
+        "config": {"workload": args.workload, "batch": B, "context": c.n_tokens,
+                   "heads": f"{Hq}q/{Hkv}kv", "head_dim": D, "tree": f"b={b},L={L}", "p": c.p,
+                   "queries_per_step": queries_per_step,
+                   "l2": "inputs larger than L2 (K+V 2.15 GB), no flush"},
+        "hbm_frac": hbm_frac,
+        "hbm_frac_of_nominal_8tbs": step_bytes / (ms_step / 1e3) / 8e12,
+        "bytes_touched_per_step": step_bytes,
+        "phases_ms": {"extend": ms_ext, "select": ms_sel, "attend": ms_att},
+        "selection": {"summary_rows_scored": cand_rows, "kept_level1_nodes": kept_nodes,
+                      "kv_rows_read": kv_rows,
+                      "kv_fraction_read": kv_rows / (B * Hkv * n_last)},
+        "roofline": roof,
+        "dense": {"ms_per_step": dense_ms, "queries_per_s": queries_per_step * world / (dense_ms / 1e3),
+                  "hbm_gbs": dense_bytes / (dense_ms / 1e3) / 1e9,
+                  "hbm_frac": dense_bytes / (dense_ms / 1e3) / 1e9 / peak},
+        "tree_build": {"ms": build_ms, "gb_per_s": build_bytes / (build_ms / 1e3) / 1e9,
+                       "tflops": build_flops / (build_ms / 1e3) / 1e12,
+                       "tokens": n_tok},
+        "e2e": {"value": queries_per_step * world / (e2e_ms / 1e3), "unit": "queries/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+    }
+    return res, wl
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        from tree_indexed_sparse_zha_b200 import workloads as W
+
+        dev = "cuda" if torch.cuda.is_available() else "cpu"
+        wl = W.make(args.workload, device=dev)
+        n = args.steps + args.warmup
+        oracle_rate(wl, min(args.warmup, 2), budget_s=60.0)  # warm-up
+        rate, done, el = oracle_rate(wl, args.steps, budget_s=600.0)
+        line = {"impl": "reference", "metric": METRIC, "value": rate, "unit": "queries/s",
+                "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": el / done * 1e3, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f32 select / f64 attention",
+                "data": "synthetic", "config": {"workload": args.workload},
+                "cpu_baseline": {"value": rate, "unit": "queries/s", "cores": 1,
+                                 "kind": "oracle",
+                                 "sample": f"{done} queries (one query head per step) of sequence 0 / "
+                                           "KV head 0, tree built untimed"},
+                "e2e": {"value": rate, "unit": "queries/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    res, wl = run_zha(args, rank, world, dev)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            rate, done, el = oracle_rate(wl, 200, budget_s=20.0)
+            res["cpu_baseline"] = {"value": rate, "unit": "queries/s", "cores": 1, "kind": "oracle",
+                                   "sample": f"{done} queries of sequence 0 / KV head 0 over "
+                                             f"{el:.1f} s (tree built untimed)"}
+        else:
+            res["cpu_baseline"] = None
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

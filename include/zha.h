@@ -166,6 +166,25 @@ zha_status zha_decode(const zha_config* cfg, const zha_cache* cache, const void*
                       void* out, int32_t* level_counts, void* ws, size_t ws_bytes,
                       int32_t* dev_status, void* stream);
 
+/* The two halves of zha_decode, for callers that schedule or time them
+ * separately. zha_decode_select runs the traversal for every sequence and
+ * leaves the kept level-1 nodes (union over the query heads of each KV head,
+ * with per-head masks) in ws; zha_decode_attend then attends over them. Both
+ * must get the same cfg, cache, q and ws; nothing may touch ws in between. */
+zha_status zha_decode_select(const zha_config* cfg, const zha_cache* cache, const void* q,
+                             double p, int32_t* level_counts, void* ws, size_t ws_bytes,
+                             int32_t* dev_status, void* stream);
+zha_status zha_decode_attend(const zha_config* cfg, const zha_cache* cache, const void* q,
+                             void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Work counters of the last zha_decode / zha_decode_select on ws, written to
+ * the device int32 array stats[B * Hkv][L + 1]: for each (sequence, KV head),
+ * the number of distinct nodes scored at levels L..1 (union over its query
+ * heads; each costs one summary-row read) followed by the number of distinct
+ * kept level-1 nodes (each costs b K rows and b V rows). Asynchronous. */
+zha_status zha_decode_stats(const zha_config* cfg, const void* ws, size_t ws_bytes,
+                            int32_t* stats, void* stream);
+
 /* Chunked prefill of sequence `seq`: the caller has written the chunk's K and V
  * rows [chunk_start, chunk_start + T) and set seq_len[seq] = chunk_start + T.
  * Extends the tree over the chunk, then for every token i of the chunk

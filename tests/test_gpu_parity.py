@@ -134,6 +134,14 @@ def test_prefill_scaled():
     ws = z.alloc_workspace(gpu.cfg, z.ZHA_OP_PREFILL, c.chunk, device=gpu.dev)
     z.zha_prefill_chunk(gpu.cfg, gpu.cache, q, 0, start, c.p, out, lc, ws, gpu.status)
     gpu.check_status()
+    # repeated calls on the same tree are bitwise identical (the cut is exact)
+    for _ in range(4):
+        out2 = torch.empty_like(q)
+        lc2 = torch.full_like(lc, -1)
+        gpu.cache.seq_len.fill_(start + c.chunk)
+        z.zha_prefill_chunk(gpu.cfg, gpu.cache, q, 0, start, c.p, out2, lc2, ws, gpu.status)
+        gpu.check_status()
+        assert torch.equal(lc2, lc) and torch.equal(out2.view(torch.int16), out.view(torch.int16))
     ref = Ref(wl, start + c.chunk)
     compare_tree(gpu, ref, 0, 0)
     compare_tree(gpu, ref, 0, 1)

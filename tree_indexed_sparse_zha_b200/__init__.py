@@ -40,8 +40,8 @@ ZHA_OP_DENSE = 4
 
 EXPORTS = (
     "zha_status_string", "zha_tree_layout", "zha_workspace_bytes", "zha_build_tree",
-    "zha_extend_tree", "zha_select", "zha_attend", "zha_decode", "zha_prefill_chunk",
-    "zha_dense_decode",
+    "zha_extend_tree", "zha_select", "zha_attend", "zha_decode", "zha_decode_select",
+    "zha_decode_attend", "zha_decode_stats", "zha_prefill_chunk", "zha_dense_decode",
 )
 
 
@@ -99,6 +99,9 @@ def lib() -> ctypes.CDLL:
                            i32),
             "zha_attend": ([c_cfg, c_cache, vp, vp, i64, vp, i64, vp, vp, vp, sz, vp, vp], i32),
             "zha_decode": ([c_cfg, c_cache, vp, d, vp, vp, vp, sz, vp, vp], i32),
+            "zha_decode_select": ([c_cfg, c_cache, vp, d, vp, vp, sz, vp, vp], i32),
+            "zha_decode_attend": ([c_cfg, c_cache, vp, vp, vp, sz, vp], i32),
+            "zha_decode_stats": ([c_cfg, vp, sz, vp, vp], i32),
             "zha_prefill_chunk": ([c_cfg, c_cache, vp, i32, i64, i64, d, vp, vp, vp, sz, vp, vp],
                                   i32),
             "zha_dense_decode": ([c_cfg, c_cache, vp, vp, vp, sz, vp], i32),
@@ -229,6 +232,28 @@ def zha_decode(cfg: zha_config, cache: Cache, q: torch.Tensor, p: float, out: to
     _check("zha_decode", lib().zha_decode(
         ctypes.byref(cfg), ctypes.byref(c), _ptr(q), float(p), _ptr(out), _ptr(level_counts),
         _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream)))
+
+
+def zha_decode_select(cfg: zha_config, cache: Cache, q: torch.Tensor, p: float,
+                      level_counts: Optional[torch.Tensor], ws: torch.Tensor,
+                      dev_status: Optional[torch.Tensor] = None, stream=None):
+    c = cache.c()
+    _check("zha_decode_select", lib().zha_decode_select(
+        ctypes.byref(cfg), ctypes.byref(c), _ptr(q), float(p), _ptr(level_counts), _ptr(ws),
+        ws.numel(), _ptr(dev_status), _stream(stream)))
+
+
+def zha_decode_attend(cfg: zha_config, cache: Cache, q: torch.Tensor, out: torch.Tensor,
+                      ws: torch.Tensor, stream=None):
+    c = cache.c()
+    _check("zha_decode_attend", lib().zha_decode_attend(
+        ctypes.byref(cfg), ctypes.byref(c), _ptr(q), _ptr(out), _ptr(ws), ws.numel(),
+        _stream(stream)))
+
+
+def zha_decode_stats(cfg: zha_config, ws: torch.Tensor, stats: torch.Tensor, stream=None):
+    _check("zha_decode_stats", lib().zha_decode_stats(
+        ctypes.byref(cfg), _ptr(ws), ws.numel(), _ptr(stats), _stream(stream)))
 
 
 def zha_prefill_chunk(cfg: zha_config, cache: Cache, q: torch.Tensor, seq: int, chunk_start: int,

@@ -83,7 +83,7 @@ static zha_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ZHA_OK 
 // ---- workspace layouts ----------------------------------------------------
 
 struct DecodeLayout {
-  size_t trav, kept, n_kept, part, total;
+  size_t trav, kept, n_kept, stats, part, total;
   int64_t units;
 };
 
@@ -97,6 +97,8 @@ static DecodeLayout decode_layout(const Geometry& g, int64_t nq, int kind, int s
   off = align256(off + traverse_kept_bytes(g, L.units, sms));
   L.n_kept = off;
   off = align256(off + sizeof(int32_t) * (size_t)L.units * kMaxClusterHost);
+  L.stats = off;
+  off = align256(off + sizeof(int32_t) * (size_t)L.units * g.L);
   L.part = off;
   off = align256(off + attend_ws_bytes(g, kind, nq, sms));
   L.total = off;
@@ -286,18 +288,24 @@ zha_status zha_attend(const zha_config* cfg, const zha_cache* cache, const void*
   return cuda_status(launch_attend(g, a, ws, ws_bytes, sms, (cudaStream_t)stream));
 }
 
-static zha_status run_tree_decode(const Geometry& g, const zha_cache* cache, const void* q,
+static zha_status run_tree_select(const Geometry& g, const zha_cache* cache, const void* q,
                                   const int32_t* q_seq, const int32_t* q_pos, int64_t nq,
-                                  uint64_t p_q, void* out, int32_t* level_counts,
-                                  unsigned char* ws, const DecodeLayout& L, int32_t* dev_status,
-                                  int sms, cudaStream_t s) {
+                                  uint64_t p_q, int32_t* level_counts, unsigned char* ws,
+                                  const DecodeLayout& L, int32_t* dev_status, int sms,
+                                  cudaStream_t s) {
   TraverseOut to{};
   to.kept = reinterpret_cast<uint32_t*>(ws + L.kept);
   to.n_kept = reinterpret_cast<int32_t*>(ws + L.n_kept);
+  to.stats = reinterpret_cast<int32_t*>(ws + L.stats);
   to.level_counts = level_counts;
-  cudaError_t e = launch_traverse(g, cache->tree, q, cache->seq_len, q_seq, q_pos, nq, p_q, 0, to,
-                                  ws + L.trav, L.kept - L.trav, dev_status, sms, s);
-  if (e != cudaSuccess) return ZHA_ERR_CUDA;
+  return cuda_status(launch_traverse(g, cache->tree, q, cache->seq_len, q_seq, q_pos, nq, p_q, 0,
+                                     to, ws + L.trav, L.kept - L.trav, dev_status, sms, s));
+}
+
+static zha_status run_tree_attend(const Geometry& g, const zha_cache* cache, const void* q,
+                                  const int32_t* q_seq, const int32_t* q_pos, int64_t nq,
+                                  void* out, unsigned char* ws, const DecodeLayout& L, int sms,
+                                  cudaStream_t s) {
   AttendArgs a{};
   a.kind = kStreamTree;
   a.k = cache->k;
@@ -308,11 +316,32 @@ static zha_status run_tree_decode(const Geometry& g, const zha_cache* cache, con
   a.q_seq = q_seq;
   a.q_pos = q_pos;
   a.nq = nq;
-  a.kept = to.kept;
-  a.n_kept = to.n_kept;
+  a.kept = reinterpret_cast<const uint32_t*>(ws + L.kept);
+  a.n_kept = reinterpret_cast<const int32_t*>(ws + L.n_kept);
   a.kept_stride = traverse_kept_stride(g);
   a.kept_segs = traverse_cluster_size(g, L.units, sms);
   return cuda_status(launch_attend(g, a, ws + L.part, L.total - L.part, sms, s));
+}
+
+static zha_status run_tree_decode(const Geometry& g, const zha_cache* cache, const void* q,
+                                  const int32_t* q_seq, const int32_t* q_pos, int64_t nq,
+                                  uint64_t p_q, void* out, int32_t* level_counts,
+                                  unsigned char* ws, const DecodeLayout& L, int32_t* dev_status,
+                                  int sms, cudaStream_t s) {
+  zha_status st = run_tree_select(g, cache, q, q_seq, q_pos, nq, p_q, level_counts, ws, L,
+                                  dev_status, sms, s);
+  if (st != ZHA_OK) return st;
+  return run_tree_attend(g, cache, q, q_seq, q_pos, nq, out, ws, L, sms, s);
+}
+
+__global__ void decode_stats_kernel(const int32_t* stats, const int32_t* n_kept, int units, int L,
+                                    int segs, int32_t* out) {
+  const int u = blockIdx.x * blockDim.x + threadIdx.x;
+  if (u >= units) return;
+  int kept = 0;
+  for (int r = 0; r < segs; ++r) kept += n_kept[(int64_t)u * segs + r];
+  for (int l = 0; l < L; ++l) out[(int64_t)u * (L + 1) + l] = stats[(int64_t)u * L + l];
+  out[(int64_t)u * (L + 1) + L] = kept;
 }
 
 zha_status zha_decode(const zha_config* cfg, const zha_cache* cache, const void* q, double p,
@@ -330,6 +359,54 @@ zha_status zha_decode(const zha_config* cfg, const zha_cache* cache, const void*
   return run_tree_decode(g, cache, q, nullptr, nullptr, g.B, p_q, out, level_counts,
                          static_cast<unsigned char*>(ws), L, dev_status, sms,
                          (cudaStream_t)stream);
+}
+
+zha_status zha_decode_select(const zha_config* cfg, const zha_cache* cache, const void* q,
+                             double p, int32_t* level_counts, void* ws, size_t ws_bytes,
+                             int32_t* dev_status, void* stream) {
+  Geometry g;
+  zha_status st = make_geometry(cfg, &g);
+  if (st != ZHA_OK) return st;
+  if ((st = check_cache(cache, false)) != ZHA_OK) return st;
+  uint64_t p_q;
+  if (!q || !ws || !check_p(p, &p_q)) return ZHA_ERR_INVALID_ARG;
+  const int sms = device_sm_count();
+  const DecodeLayout L = decode_layout(g, g.B, kStreamTree, sms);
+  if (ws_bytes < L.total) return ZHA_ERR_WORKSPACE;
+  return run_tree_select(g, cache, q, nullptr, nullptr, g.B, p_q, level_counts,
+                         static_cast<unsigned char*>(ws), L, dev_status, sms,
+                         (cudaStream_t)stream);
+}
+
+zha_status zha_decode_attend(const zha_config* cfg, const zha_cache* cache, const void* q,
+                             void* out, void* ws, size_t ws_bytes, void* stream) {
+  Geometry g;
+  zha_status st = make_geometry(cfg, &g);
+  if (st != ZHA_OK) return st;
+  if ((st = check_cache(cache, true)) != ZHA_OK) return st;
+  if (!q || !out || !ws) return ZHA_ERR_INVALID_ARG;
+  const int sms = device_sm_count();
+  const DecodeLayout L = decode_layout(g, g.B, kStreamTree, sms);
+  if (ws_bytes < L.total) return ZHA_ERR_WORKSPACE;
+  return run_tree_attend(g, cache, q, nullptr, nullptr, g.B, out,
+                         static_cast<unsigned char*>(ws), L, sms, (cudaStream_t)stream);
+}
+
+zha_status zha_decode_stats(const zha_config* cfg, const void* ws, size_t ws_bytes,
+                            int32_t* stats, void* stream) {
+  Geometry g;
+  zha_status st = make_geometry(cfg, &g);
+  if (st != ZHA_OK) return st;
+  if (!ws || !stats) return ZHA_ERR_INVALID_ARG;
+  const int sms = device_sm_count();
+  const DecodeLayout L = decode_layout(g, g.B, kStreamTree, sms);
+  if (ws_bytes < L.total) return ZHA_ERR_WORKSPACE;
+  const unsigned char* w = static_cast<const unsigned char*>(ws);
+  const int units = (int)L.units;
+  decode_stats_kernel<<<(units + 127) / 128, 128, 0, (cudaStream_t)stream>>>(
+      reinterpret_cast<const int32_t*>(w + L.stats), reinterpret_cast<const int32_t*>(w + L.n_kept),
+      units, g.L, traverse_cluster_size(g, L.units, sms), stats);
+  return cuda_status(cudaGetLastError());
 }
 
 zha_status zha_prefill_chunk(const zha_config* cfg, const zha_cache* cache, const void* q,

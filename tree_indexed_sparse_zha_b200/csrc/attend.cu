@@ -78,6 +78,7 @@ struct Span {
   int64_t tail_start;
   int64_t rows;
   const uint32_t* kept;        // segment 0 of the unit
+  const uint32_t* kept_local;  // this CTA's node range [n0, n1) in shared memory, or null
   const unsigned int* segbase; // [segs + 1] prefix of segment sizes (shared memory)
   int64_t stride;
   const int32_t* list;
@@ -96,9 +97,14 @@ __device__ __forceinline__ void row_of(const AttParams& p, const Span& s, int64_
     const int64_t nrows = (s.n1 - s.n0) * p.b;
     if (v < nrows) {
       const int64_t j = s.n0 + v / p.b;
-      int r = 0;
-      while ((int64_t)s.segbase[r + 1] <= j) ++r;
-      const uint32_t e = s.kept[r * s.stride + (j - s.segbase[r])];
+      uint32_t e;
+      if (s.kept_local) {
+        e = s.kept_local[j - s.n0];
+      } else {
+        int r = 0;
+        while ((int64_t)s.segbase[r + 1] <= j) ++r;
+        e = s.kept[r * s.stride + (j - s.segbase[r])];
+      }
       const int64_t node = e & 0x00ffffffu;
       const int off = (int)(v % p.b);
       *row = node * p.b + off;
@@ -419,6 +425,7 @@ struct MmaCfg {
   static constexpr int kStageBytes = 32 * kRowBytes * 2;             // K and V of 32 rows
   static constexpr int kWarpBytes = kStages * kStageBytes + kStages * 32;  // + row masks
   static constexpr int kWarps = 4;
+  static constexpr int kKeptCap = 5120;   // kept-list entries staged in shared memory
   static constexpr int kThreads = 32 * kWarps;
   static constexpr int kKSteps = D / 16;   // QK k-steps
   static constexpr int kNTiles = D / 8;    // PV n-tiles
@@ -509,6 +516,16 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads, 1) attend_mma_kernel(AttP
     s.t0 = tail_len * split / p.S;
     s.t1 = tail_len * (split + 1) / p.S;
     s.rows = s.tok0 + (s.n1 - s.n0) * p.b + (s.t1 - s.t0);
+    if (s.n1 - s.n0 <= C::kKeptCap) {  // stage this CTA's kept entries in smem once
+      uint32_t* kl = reinterpret_cast<uint32_t*>(smem + C::kWarps * C::kWarpBytes);
+      for (int64_t j = s.n0 + tid; j < s.n1; j += C::kThreads) {
+        int r = 0;
+        while ((int64_t)s_segbase[r + 1] <= j) ++r;
+        kl[j - s.n0] = s.kept[r * s.stride + (j - s_segbase[r])];
+      }
+      s.kept_local = kl;
+      __syncthreads();
+    }
   }
 
   // Q fragments (rows g < G; exact bf16 inputs), kept in registers
@@ -534,15 +551,23 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads, 1) attend_mma_kernel(AttP
   const int nw = C::kWarps;
   const int64_t nblk = (s.rows + 31) / 32;
 
-  auto issue = [&](int64_t blk, int stage) {
-    const int64_t v = blk * 32 + lane;
-    uint32_t m = 0;
-    int64_t row = 0;
-    if (blk < nblk && v < s.rows) {
-      row_of(p, s, v, &row, &m, all);
-      if (row < 0 || row >= p.ncap) m = 0u;
+  // Row metadata of the next block to issue is computed one block ahead, so the
+  // kept-list load it needs completes while the current block is computed.
+  int64_t nxt_blk = warp;
+  int64_t pr_row = 0;
+  uint32_t pr_m = 0;
+  auto fetch_row = [&]() {
+    const int64_t v = nxt_blk * 32 + lane;
+    pr_m = 0;
+    pr_row = 0;
+    if (nxt_blk < nblk && v < s.rows) {
+      row_of(p, s, v, &pr_row, &pr_m, all);
+      if (pr_row < 0 || pr_row >= p.ncap) pr_m = 0u;
     }
-    rmask[stage * 32 + lane] = (uint8_t)m;
+  };
+  fetch_row();
+  auto issue = [&](int stage) {
+    rmask[stage * 32 + lane] = (uint8_t)pr_m;
     // every instruction moves whole rows: lanes 16j..16j+15 copy the 16-byte
     // chunks of one row, so each warp request is a few full 128-byte lines
     constexpr int kCh = C::kRowBytes / 16;   // chunks per row (8 or 16)
@@ -552,8 +577,8 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads, 1) attend_mma_kernel(AttP
 #pragma unroll
     for (int i = 0; i < 32 / kRowsPerInstr; ++i) {
       const int r = i * kRowsPerInstr + lane / kCh;
-      const int64_t rr = __shfl_sync(0xffffffffu, row, r);
-      const uint32_t mm = __shfl_sync(0xffffffffu, m, r);
+      const int64_t rr = __shfl_sync(0xffffffffu, pr_row, r);
+      const uint32_t mm = __shfl_sync(0xffffffffu, pr_m, r);
       if (mm) {
         const int64_t off = rr * C::kRowBytes + c * 16;
         const int dst = r * C::kRowBytes + swz(c, r) * 16;
@@ -562,6 +587,8 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads, 1) attend_mma_kernel(AttP
       }
     }
     cp_async_commit();
+    nxt_blk += nw;
+    fetch_row();
   };
 
   float o[C::kNTiles][4];
@@ -572,10 +599,10 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads, 1) attend_mma_kernel(AttP
   // prologue: stages 0 .. kStages-2
   int64_t blk = warp;
 #pragma unroll
-  for (int st = 0; st < C::kStages - 1; ++st) issue(blk + (int64_t)st * nw, st);
+  for (int st = 0; st < C::kStages - 1; ++st) issue(st);
   int stage = 0;
   for (; blk < nblk; blk += nw) {
-    issue(blk + (int64_t)(C::kStages - 1) * nw, (stage + C::kStages - 1) % C::kStages);
+    issue((stage + C::kStages - 1) % C::kStages);
     cp_async_wait<C::kStages - 1>();
     __syncwarp();
     const unsigned char* kst = my + stage * C::kStageBytes;
@@ -724,7 +751,7 @@ cudaError_t launch_t(const AttParams& p, int64_t units, void* out, cudaStream_t 
   if constexpr (sizeof(T) == 2 && G >= 2) {
     if (p.kind != kStreamList) {
       using M = MmaCfg<D>;
-      const size_t smem = (size_t)M::kWarps * M::kWarpBytes;
+      const size_t smem = (size_t)M::kWarps * M::kWarpBytes + sizeof(uint32_t) * M::kKeptCap;
       auto kern = attend_mma_kernel<D, G>;
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;

@@ -47,9 +47,10 @@ constexpr int kBuckets = 2048;
 constexpr int kDigit = 11;
 constexpr int kCandPerThread = 4;
 constexpr uint32_t kNodeMask = 0x00ffffffu;
-constexpr int kChunk = 2048;          // candidates per streamed chunk (8 per thread)
+constexpr int kChunk = 8 * kThreads;  // candidates per streamed chunk (8 per thread)
 constexpr int kStages = 3;            // cp.async ring depth of the cut passes
 constexpr int kListCap = 2048;        // crossing-bucket members finished in shared memory
+constexpr int kRankCap = 256;         // per-head frontiers this small are cut by explicit ranks
 
 struct TravParams {
   const void* tree;
@@ -77,6 +78,7 @@ struct TravParams {
   int64_t idx_cap;
   int32_t* n_idx;
   int32_t* level_counts;
+  int32_t* stats;        // [units][L]: union candidates scored per level (nullable)
   int32_t* status;
 };
 
@@ -100,6 +102,9 @@ struct Smem {
   unsigned int list_n;
   unsigned int seg_n[kMaxCluster];
   unsigned int chunk_start[kMaxCluster + 1];
+  unsigned int res_base[kMaxCluster];   // resident copy: segment r at ring[res_base[r]]
+  float g_zmax[kMaxCluster][kMaxGroup];  // every rank's segment extremes, gathered once
+  float g_zmin[kMaxCluster][kMaxGroup];
   float red_f[kWarps][kMaxGroup][2];
   unsigned long long red_u64[kWarps];
   unsigned int red_u32[kWarps];
@@ -145,6 +150,25 @@ __device__ __forceinline__ unsigned long long block_sum_u64(unsigned long long v
   return t;
 }
 
+// Exclusive scan of a u64 over the CTA in thread order.
+__device__ __forceinline__ unsigned long long block_excl_scan_u64(unsigned long long v, Smem& S) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned long long x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const unsigned long long y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) S.red_u64[warp] = x;
+  __syncthreads();
+  unsigned long long wbase = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w)
+    if (w < warp) wbase += S.red_u64[w];
+  __syncthreads();
+  return wbase + x - v;
+}
+
 // Exact 64-bit accumulation into a (lo, hi) pair of 32-bit shared counters.
 __device__ __forceinline__ void hist_add(Smem& S, int b, unsigned long long m, unsigned int n) {
   const unsigned int lo = (unsigned int)m;
@@ -167,9 +191,46 @@ __device__ __forceinline__ unsigned long long ceil_mul_shift32(unsigned long lon
 // Streams head h's (score, candidate) pairs of every segment, in ascending node
 // order, through a cp.async ring; f(z[8], c[8], nvalid, pos0) sees the 8
 // consecutive candidates of this thread (pos0 = (segment << 24) | first index).
+constexpr int kResidentCap = kStages * kChunk;  // candidates kept resident per head
+
+// Copies head h's scores and candidate entries of every segment into the ring
+// (segment r at res_base[r], 32-aligned); returns false if they do not fit.
+__device__ __forceinline__ bool load_resident(Smem& S, int C, const uint32_t* cbase,
+                                              const float* zbase, int64_t seg) {
+  float* rz = &S.ring_z[0][0];
+  uint32_t* rc = &S.ring_c[0][0];
+  unsigned int acc = 0;
+  for (int r = 0; r < C; ++r) acc += (S.seg_n[r] + 31u) & ~31u;
+  if (acc > (unsigned)kResidentCap) return false;
+  if (threadIdx.x == 0) {
+    unsigned int b = 0;
+    for (int r = 0; r < C; ++r) {
+      S.res_base[r] = b;
+      b += (S.seg_n[r] + 31u) & ~31u;
+    }
+  }
+  __syncthreads();
+  for (int r = 0; r < C; ++r) {
+    const int pieces = (int)((S.seg_n[r] + 3u) >> 2);
+    for (int e = threadIdx.x; e < pieces; e += kThreads) {
+      cp_async16(rz + S.res_base[r] + e * 4, zbase + r * seg + e * 4);
+      cp_async16(rc + S.res_base[r] + e * 4, cbase + r * seg + e * 4);
+    }
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+  return true;
+}
+
+// Visits head h's (score, candidate) pairs of every segment, in ascending node
+// order; f(z[8], c[8], nvalid, pos0, idx0, r) sees 8 consecutive candidates of
+// segment r starting at index idx0 (pos0 = (r << 24) | idx0). Chunks come from
+// the resident copy, or are streamed through the cp.async ring.
 template <typename F>
 __device__ __forceinline__ void stream_head(Smem& S, int C, const uint32_t* cbase,
-                                            const float* zbase, int64_t seg, F&& f) {
+                                            const float* zbase, int64_t seg, bool resident,
+                                            F&& f) {
   const int tid = threadIdx.x;
   const int nchunks = (int)S.chunk_start[C];
   auto locate = [&](int k, int& r, int64_t& off) {
@@ -192,34 +253,52 @@ __device__ __forceinline__ void stream_head(Smem& S, int C, const uint32_t* cbas
     }
     cp_async_commit();
   };
+  if (!resident) {
 #pragma unroll
-  for (int st = 0; st < kStages - 1; ++st) issue(st, st);
+    for (int st = 0; st < kStages - 1; ++st) issue(st, st);
+  }
   for (int k = 0; k < nchunks; ++k) {
-    issue(k + kStages - 1, (k + kStages - 1) % kStages);
-    cp_async_wait<kStages - 1>();
-    __syncthreads();
-    const int st = k % kStages;
+    const float* zsrc;
+    const uint32_t* csrc;
     int r;
     int64_t off;
     locate(k, r, off);
+    if (!resident) {
+      issue(k + kStages - 1, (k + kStages - 1) % kStages);
+      cp_async_wait<kStages - 1>();
+      __syncthreads();
+      zsrc = &S.ring_z[k % kStages][0];
+      csrc = &S.ring_c[k % kStages][0];
+    } else {
+      zsrc = &S.ring_z[0][0] + S.res_base[r] + off;
+      csrc = &S.ring_c[0][0] + S.res_base[r] + off;
+    }
     const int64_t n = S.seg_n[r];
     const int len = (int)((n - off) < kChunk ? (n - off) : kChunk);
     const int first = tid * 8;
     const int nvalid = len - first < 0 ? 0 : (len - first > 8 ? 8 : len - first);
     float z[8];
     uint32_t c[8];
-    const float4 z0 = *reinterpret_cast<const float4*>(&S.ring_z[st][first]);
-    const float4 z1 = *reinterpret_cast<const float4*>(&S.ring_z[st][first + 4]);
-    const uint4 c0 = *reinterpret_cast<const uint4*>(&S.ring_c[st][first]);
-    const uint4 c1 = *reinterpret_cast<const uint4*>(&S.ring_c[st][first + 4]);
-    z[0] = z0.x; z[1] = z0.y; z[2] = z0.z; z[3] = z0.w;
-    z[4] = z1.x; z[5] = z1.y; z[6] = z1.z; z[7] = z1.w;
-    c[0] = c0.x; c[1] = c0.y; c[2] = c0.z; c[3] = c0.w;
-    c[4] = c1.x; c[5] = c1.y; c[6] = c1.z; c[7] = c1.w;
+    if (nvalid > 0) {
+      const float4 z0 = *reinterpret_cast<const float4*>(zsrc + first);
+      const float4 z1 = *reinterpret_cast<const float4*>(zsrc + first + 4);
+      const uint4 c0 = *reinterpret_cast<const uint4*>(csrc + first);
+      const uint4 c1 = *reinterpret_cast<const uint4*>(csrc + first + 4);
+      z[0] = z0.x; z[1] = z0.y; z[2] = z0.z; z[3] = z0.w;
+      z[4] = z1.x; z[5] = z1.y; z[6] = z1.z; z[7] = z1.w;
+      c[0] = c0.x; c[1] = c0.y; c[2] = c0.z; c[3] = c0.w;
+      c[4] = c1.x; c[5] = c1.y; c[6] = c1.z; c[7] = c1.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        z[j] = 0.0f;
+        c[j] = 0u;
+      }
+    }
     f(z, c, nvalid, ((uint32_t)r << 24) | (uint32_t)(off + first), off + first, r);
-    __syncthreads();
+    if (!resident) __syncthreads();
   }
-  cp_async_wait<0>();
+  if (!resident) cp_async_wait<0>();
 }
 
 // Adds (mass m, count n) to bucket d, aggregating across the warp when every
@@ -247,7 +326,7 @@ __device__ __forceinline__ void hist_add_warp(Smem& S, bool valid, uint32_t d,
 
 // Crossing digit of the current histogram: above + mass(digits > d) < need <=
 // above + mass(digits >= d). Returns false if none exists (never for exact sums).
-__device__ __forceinline__ bool find_crossing(Smem& S, unsigned long long above,
+__device__ __forceinline__ bool find_crossing(Smem& S, int nb, unsigned long long above,
                                               unsigned long long need, uint32_t* beta,
                                               unsigned long long* above_out,
                                               unsigned long long* bmass, unsigned int* bcnt) {
@@ -257,8 +336,8 @@ __device__ __forceinline__ bool find_crossing(Smem& S, unsigned long long above,
   unsigned long long tsum = 0;
 #pragma unroll
   for (int j = 0; j < kPerT; ++j) {
-    const int d = tid * kPerT + j;
-    mloc[j] = ((unsigned long long)S.hhi[d] << 32) | S.hlo[d];
+    const int d = tid * kPerT + j;  // buckets >= nb were not cleared this pass
+    mloc[j] = d < nb ? ((unsigned long long)S.hhi[d] << 32) | S.hlo[d] : 0ull;
     tsum += mloc[j];
   }
   unsigned long long x = tsum;  // suffix over lanes (higher lanes = higher digits)
@@ -295,8 +374,8 @@ __device__ __forceinline__ bool find_crossing(Smem& S, unsigned long long above,
   return ok;
 }
 
-__device__ __forceinline__ void clear_hist(Smem& S) {
-  for (int e = threadIdx.x; e < kBuckets; e += kThreads) {
+__device__ __forceinline__ void clear_hist(Smem& S, int nb) {
+  for (int e = threadIdx.x; e < nb; e += kThreads) {
     S.hlo[e] = 0u;
     S.hhi[e] = 0u;
     S.hcnt[e] = 0u;
@@ -441,6 +520,7 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
     const T* qrow = static_cast<const T*>(p.q) + ((int64_t)qi * p.Hq + (int64_t)kvh * G + h) * D;
     S.q[e] = (h < G) ? Elem<T>::to_f(qrow[i]) : 0.0f;
   }
+  if (p.stats && rank == 0 && tid < p.L) p.stats[(int64_t)unit * p.L + tid] = 0;
   __syncthreads();
 
   uint32_t* cand_u = p.cand + (int64_t)unit * 2 * C * seg;
@@ -523,11 +603,18 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
     if (tid == 0) S.xch.count = (unsigned int)my_n;
     __syncthreads();
     cluster.sync();  // S1: every segment scored
+    if (p.stats && tid == 0) atomicAdd(&p.stats[(int64_t)unit * p.L + (p.L - level)], (int)my_n);
 
     // ------------------------------------------------------------------
     // 2. exact cut for the heads this CTA owns
     // ------------------------------------------------------------------
-    if (tid < C) S.seg_n[tid] = cluster.map_shared_rank(&S.xch, tid)->count;
+    for (int e = tid; e < C * (2 * G + 1); e += kThreads) {  // one parallel DSMEM gather
+      const int r = e / (2 * G + 1), k = e % (2 * G + 1);
+      const Xch* rx = cluster.map_shared_rank(&S.xch, r);
+      if (k == 0) S.seg_n[r] = rx->count;
+      else if (k <= G) S.g_zmax[r][k - 1] = rx->zmax[k - 1];
+      else S.g_zmin[r][k - 1 - G] = rx->zmin[k - 1 - G];
+    }
     __syncthreads();
     if (tid == 0) {
       unsigned int acc = 0;
@@ -544,9 +631,8 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
       if (tid == 0) {
         float mx = -INFINITY, mn = INFINITY;
         for (int r = 0; r < C; ++r) {
-          const Xch* rx = cluster.map_shared_rank(&S.xch, r);
-          mx = fmaxf(mx, rx->zmax[h]);
-          mn = fminf(mn, rx->zmin[h]);
+          mx = fmaxf(mx, S.g_zmax[r][h]);
+          mn = fminf(mn, S.g_zmin[r][h]);
         }
         S.bc_u32[0] = __float_as_uint(mx);
         S.bc_u32[1] = __float_as_uint(mn);
@@ -554,6 +640,89 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
       }
       __syncthreads();
       const float zmax = __uint_as_float(S.bc_u32[0]);
+      // small frontiers: one copy into shared memory serves every pass
+      const bool resident = load_resident(S, C, cseg, zseg, seg);
+      if (resident) {
+        // gather head h's candidates (score, position); tiny frontiers are cut by
+        // explicit ranks instead of digit passes
+        if (tid == 0) S.list_n = 0u;
+        __syncthreads();
+        stream_head(S, C, cseg, zseg, seg, true,
+                    [&](const float* z, const uint32_t* c, int nvalid, uint32_t pos0, int64_t,
+                        int) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (j < nvalid && ((c[j] >> (24 + h)) & 1u)) {
+              const unsigned slot = atomicAdd(&S.list_n, 1u);
+              if (slot < (unsigned)kListCap) {
+                S.list_z[slot] = z[j];
+                S.list_pos[slot] = pos0 + (uint32_t)j;
+              }
+            }
+        });
+        __syncthreads();
+      }
+      const int n_h = resident ? (int)S.list_n : kRankCap + 1;
+      __syncthreads();  // every warp has read list_n before the radix path resets it
+      if (n_h <= kRankCap) {
+        // rank_i = #{j : z_j > z_i, or z_j == z_i and pos_j < pos_i}; mass M_i is
+        // scattered to its rank; the cut is the shortest rank prefix reaching need
+        unsigned long long tloc = 0;
+        for (int i = tid; i < n_h; i += kThreads) {
+          const float zi = S.list_z[i];
+          const uint32_t pi = S.list_pos[i];
+          unsigned int rk = 0;
+          for (int j = 0; j < n_h; ++j) {
+            const float zj = S.list_z[j];
+            rk += (zj > zi || (zj == zi && S.list_pos[j] < pi)) ? 1u : 0u;
+          }
+          const unsigned long long m = mass_fixed(zi, zmax);
+          tloc += m;
+          S.hcnt[i] = rk;
+          S.hlo[rk] = (unsigned int)m;
+          S.hhi[rk] = (unsigned int)(m >> 32);
+        }
+        const unsigned long long Tm = block_sum_u64(tloc, S);
+        const unsigned long long need_r = ceil_mul_shift32(Tm, p.p_q);
+        // thread t owns ranks [4t, 4t + 4)
+        unsigned long long part[4];
+        unsigned long long tsum = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int rk = tid * 4 + j;
+          part[j] = rk < n_h ? (((unsigned long long)S.hhi[rk] << 32) | S.hlo[rk]) : 0ull;
+          tsum += part[j];
+        }
+        unsigned long long run = block_excl_scan_u64(tsum, S);
+        if (tid == 0) S.bc_u32[5] = (unsigned)n_h;
+        __syncthreads();
+        if (!p.keep_all) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int rk = tid * 4 + j;
+            if (rk < n_h && run < need_r && run + part[j] >= need_r) S.bc_u32[5] = (unsigned)rk + 1u;
+            run += part[j];
+          }
+        }
+        __syncthreads();
+        const unsigned int k = S.bc_u32[5];
+        // keep bits: clear head h's words, then set the kept ranks
+        for (int r = 0; r < C; ++r) {
+          uint32_t* kb = kptr(h, r);
+          for (int wd = tid; wd < (int)((S.seg_n[r] + 31u) >> 5); wd += kThreads) kb[wd] = 0u;
+        }
+        __syncthreads();
+        for (int i = tid; i < n_h; i += kThreads)
+          if (S.hcnt[i] < k) {
+            const uint32_t pi = S.list_pos[i];
+            atomicOr(&kptr(h, (int)(pi >> 24))[(pi & kNodeMask) >> 5], 1u << (pi & 31u));
+          }
+        if (lc_base && tid == 0) lc_base[(int64_t)h * p.L + (p.L - level)] = (int32_t)k;
+        __syncthreads();
+      }
+      if (n_h > kRankCap) {  // radix-select cut
+      if (tid == 0) S.list_n = 0u;
+      __syncthreads();
       const uint32_t kmax = order_key(zmax), kmin = order_key(__uint_as_float(S.bc_u32[1]));
       const uint32_t diff = kmax ^ kmin;
       int shift = diff ? 32 - __clz(diff) : 0;
@@ -566,35 +735,42 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
       for (int pass = 0; !done && pass < 4; ++pass) {  // <= ceil(32/11) digit passes
         const int w = shift < kDigit ? shift : kDigit;
         const int sh = shift - w;
-        clear_hist(S);
+        clear_hist(S, 1 << w);
         unsigned long long tloc = 0;
         if (!listed) {
           // full streaming pass over every candidate of head h
-          stream_head(S, C, cseg, zseg, seg,
+          stream_head(S, C, cseg, zseg, seg, resident,
                       [&](const float* z, const uint32_t* c, int nvalid, uint32_t, int64_t, int) {
-            // per-thread run-length aggregation over its 8 consecutive candidates
+            // the 8 masses first (independent chains), then per-thread run-length
+            // aggregation of equal digits
+            bool ok[8];
+            uint32_t dg[8];
+            unsigned long long ms[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const uint32_t key = order_key(z[j]);
+              ok[j] = j < nvalid && ((c[j] >> (24 + h)) & 1u) &&
+                      (uint32_t)((uint64_t)key >> shift) == prefix;
+              dg[j] = (key >> sh) & ((1u << w) - 1u);
+              ms[j] = ok[j] ? mass_fixed(z[j], zmax) : 0ull;
+            }
             bool have = false;
             uint32_t rd = 0;
             unsigned long long rm = 0;
             unsigned int rc = 0;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-              if (j < nvalid && ((c[j] >> (24 + h)) & 1u)) {
-                const uint32_t key = order_key(z[j]);
-                if ((uint32_t)((uint64_t)key >> shift) == prefix) {
-                  const uint32_t d = (key >> sh) & ((1u << w) - 1u);
-                  const unsigned long long m = mass_fixed(z[j], zmax);
-                  tloc += m;
-                  if (have && d != rd) {
-                    hist_add(S, (int)rd, rm, rc);
-                    rm = 0;
-                    rc = 0;
-                  }
-                  have = true;
-                  rd = d;
-                  rm += m;
-                  rc += 1;
+              if (ok[j]) {
+                tloc += ms[j];
+                if (have && dg[j] != rd) {
+                  hist_add(S, (int)rd, rm, rc);
+                  rm = 0;
+                  rc = 0;
                 }
+                have = true;
+                rd = dg[j];
+                rm += ms[j];
+                rc += 1;
               }
             }
             hist_add_warp(S, have, rd, rm, rc);
@@ -624,7 +800,7 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
         }
         __syncthreads();
         uint32_t beta;
-        if (!find_crossing(S, above, need, &beta, &above, &bmass, &bcnt)) {
+        if (!find_crossing(S, 1 << w, above, need, &beta, &above, &bmass, &bcnt)) {
           if (tid == 0) raise_status(p.status, ZHA_ERR_INTERNAL);  // never loop forever
           done = true;
           break;
@@ -634,7 +810,7 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
         done = (bcnt == 1u) || (shift == 0);
         if (!done && !listed && bcnt <= (unsigned)kListCap) {
           // gather the crossing bucket's members once; later digits run in smem
-          stream_head(S, C, cseg, zseg, seg,
+          stream_head(S, C, cseg, zseg, seg, resident,
                       [&](const float* z, const uint32_t* c, int nvalid, uint32_t pos0, int64_t,
                           int) {
 #pragma unroll
@@ -681,7 +857,7 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
         pos_thr = S.bc_u32[4];
       }
       unsigned int kept_loc = 0, tie_run = 0;
-      stream_head(S, C, cseg, zseg, seg,
+      stream_head(S, C, cseg, zseg, seg, resident,
                   [&](const float* z, const uint32_t* c, int nvalid, uint32_t pos0,
                       int64_t idx0, int r) {
         uint32_t bits = 0, ties = 0;
@@ -722,6 +898,7 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
       unsigned int ktot;
       block_excl_scan(kept_loc, &ktot, S);
       if (lc_base && tid == 0) lc_base[(int64_t)h * p.L + (p.L - level)] = (int32_t)ktot;
+      }  // radix-select cut
 
       if (level == 1 && p.list_mode) {
         // ascending token list of head h: {0} (unless node 0 is kept) +
@@ -984,6 +1161,7 @@ cudaError_t launch_traverse(const Geometry& g, const void* tree, const void* q,
   p.idx_cap = out.idx_cap;
   p.n_idx = out.n_idx;
   p.level_counts = out.level_counts;
+  p.stats = out.stats;
   p.status = status;
   if (g.dtype == ZHA_BF16) {
     if (g.d == 128) return launch_g<__nv_bfloat16, 128>(g.G, p, units, C, stream);

@@ -45,6 +45,7 @@ struct TraverseOut {
   int64_t idx_cap;
   int32_t* n_idx;          // [nq][Hq]
   int32_t* level_counts;   // [nq][Hq][L] (nullable)
+  int32_t* stats;          // [units][L] union candidates per level (nullable)
 };
 
 // CTAs per traversal cluster for `units` (query token, KV head) units.
