@@ -30,7 +30,8 @@
  *   - All tensor pointers are DEVICE pointers owned by the caller (for example
  *     PyTorch tensors), contiguous, 16-byte aligned. The library never
  *     allocates, never synchronises the device and keeps no state between
- *     calls; it is re-entrant.
+ *     calls; it is re-entrant (zha_decode_noalloc, which works in a static
+ *     device array instead of a caller workspace, is the one exception).
  *   - `stream` is a cudaStream_t passed as void*; every call is asynchronous on
  *     it.
  *   - Argument errors return synchronously before any launch
@@ -201,6 +202,30 @@ zha_status zha_prefill_chunk(const zha_config* cfg, const zha_cache* cache, cons
  * ws: ZHA_OP_DENSE workspace. */
 zha_status zha_dense_decode(const zha_config* cfg, const zha_cache* cache, const void* q,
                             void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* zha_decode without a caller workspace. The pages describe no counterpart of
+ * this call; it exists for callers that cannot hand the library a workspace --
+ * plugins loaded by a host that owns the device allocator and exposes none of
+ * it, and hot paths where an allocation is not allowed (cudaMalloc and
+ * cudaFree synchronise the device). It computes exactly what zha_decode
+ * computes, using as its workspace a 64 MiB array in the library's static
+ * device memory instead of ws; nothing is allocated by the call.
+ *   - Limit: geometries whose ZHA_OP_DECODE workspace (zha_workspace_bytes)
+ *     exceeds 64 MiB are rejected with ZHA_ERR_WORKSPACE before any launch
+ *     (for example B = 1, Hkv = 2, G = 8, b = 4 fits up to about 180K tokens).
+ *   - Set-up: the first call on each device looks up the array's device
+ *     address (this loads its module on that device); make that first call
+ *     with the device current and outside any stream capture.
+ *   - The scratch needs no clearing: every word is written before it is read.
+ *   - Unlike the other entry points this one is NOT re-entrant: every call on
+ *     a device shares the one array, so two calls whose executions overlap
+ *     (different streams, or different host threads, without ordering between
+ *     them) race and corrupt each other's results. Order them on one stream or
+ *     with events.
+ * Arguments, layouts, dev_status and errors are those of zha_decode. */
+zha_status zha_decode_noalloc(const zha_config* cfg, const zha_cache* cache, const void* q,
+                              double p, void* out, int32_t* level_counts, int32_t* dev_status,
+                              void* stream);
 
 #ifdef __cplusplus
 }

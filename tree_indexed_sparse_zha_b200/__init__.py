@@ -42,6 +42,7 @@ EXPORTS = (
     "zha_status_string", "zha_tree_layout", "zha_workspace_bytes", "zha_build_tree",
     "zha_extend_tree", "zha_select", "zha_attend", "zha_decode", "zha_decode_select",
     "zha_decode_attend", "zha_decode_stats", "zha_prefill_chunk", "zha_dense_decode",
+    "zha_decode_noalloc",
 )
 
 
@@ -105,6 +106,7 @@ def lib() -> ctypes.CDLL:
             "zha_prefill_chunk": ([c_cfg, c_cache, vp, i32, i64, i64, d, vp, vp, vp, sz, vp, vp],
                                   i32),
             "zha_dense_decode": ([c_cfg, c_cache, vp, vp, vp, sz, vp], i32),
+            "zha_decode_noalloc": ([c_cfg, c_cache, vp, d, vp, vp, vp, vp], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -271,6 +273,18 @@ def zha_dense_decode(cfg: zha_config, cache: Cache, q: torch.Tensor, out: torch.
     _check("zha_dense_decode", lib().zha_dense_decode(
         ctypes.byref(cfg), ctypes.byref(c), _ptr(q), _ptr(out), _ptr(ws), ws.numel(),
         _stream(stream)))
+
+
+def zha_decode_noalloc(cfg: zha_config, cache: Cache, q: torch.Tensor, p: float,
+                       out: torch.Tensor, level_counts: Optional[torch.Tensor],
+                       dev_status: Optional[torch.Tensor] = None, stream=None):
+    """zha_decode with the library's static 64 MiB device scratch as workspace
+    (no allocation). Calls whose executions overlap share that scratch and race;
+    order them on one stream."""
+    c = cache.c()
+    _check("zha_decode_noalloc", lib().zha_decode_noalloc(
+        ctypes.byref(cfg), ctypes.byref(c), _ptr(q), float(p), _ptr(out), _ptr(level_counts),
+        _ptr(dev_status), _stream(stream)))
 
 
 __all__ = [n for n in globals() if n.startswith("zha_")] + [
