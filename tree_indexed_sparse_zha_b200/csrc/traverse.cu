@@ -15,16 +15,27 @@
 // A thread-block cluster of C CTAs cooperates on a unit. CTA r owns an ordered
 // SEGMENT of the frontier: the top nodes are split into C contiguous ranges and
 // each CTA keeps the children of its own kept nodes, so the concatenation of
-// the segments in rank order is always sorted by node index and no global
-// compaction is needed. Per level:
-//   1. score   -- each CTA scores its segment for all heads (canonical fp32
-//                 chains; 4 candidates x G heads per thread).      cluster sync
-//   2. cut     -- the CTA owning head h (h mod C) runs the exact cut for h over
-//                 every segment: radix select on the order-preserving bits of z
-//                 with fixed-point mass sums per bucket (11-bit digits), then
-//                 writes h's keep bits.                            cluster sync
-//   3. expand  -- each CTA turns its segment's keep bits into the next level's
-//                 candidates (children of nodes kept by any head).
+// the segments in rank order is always sorted by node index. Per level:
+//   1. score  -- each CTA scores its segment for all heads (canonical fp32
+//                chains, 4 candidates x G heads per thread); the segment's
+//                score extremes go to distributed shared memory.  cluster sync
+//   2. cut    -- a distributed select per head. Every CTA histograms its own
+//                segment for all heads at once into 256 buckets holding the
+//                exact fixed-point mass and the count of their members; the
+//                CTA owning head h sums the C histograms of h
+//                through DSMEM, finds the bucket where the mass taken in
+//                descending score order reaches the target, and publishes the
+//                narrowed group.                      two cluster syncs a pass
+//                The first pass buckets z linearly over the head's score
+//                range, so the crossing group is small; later passes resolve
+//                the group's order-preserving key 8 bits at a time. The
+//                result is a rule per head: keep iff key > kthr, or key ==
+//                kthr and the candidate is among the first quota[r] such
+//                candidates of segment r (exact ties, node order).
+//   3. expand -- each CTA applies the rules to its own segment and writes the
+//                children of the nodes kept by any head, or, at level 1, the
+//                kept list.
+// No candidate, score or keep bit crosses CTAs through global memory.
 // Canonical arithmetic (identical to the CPU oracle):
 //   z = (dot(q, s) * inv_sqrt_d) + fp32(l ln b),  M = trunc(exp(z - zmax) 2^40),
 //   need = ceil(T p_q / 2^32); keep the shortest prefix of (z desc, node asc)
@@ -43,14 +54,19 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kBuckets = 2048;
-constexpr int kDigit = 11;
+constexpr int kDigit = 8;                 // key bits resolved per radix pass
+constexpr int kBuckets = 1 << kDigit;     // == kThreads: one bucket per thread
 constexpr int kCandPerThread = 4;
 constexpr uint32_t kNodeMask = 0x00ffffffu;
-constexpr int kChunk = 8 * kThreads;  // candidates per streamed chunk (8 per thread)
-constexpr int kStages = 3;            // cp.async ring depth of the cut passes
-constexpr int kListCap = 2048;        // crossing-bucket members finished in shared memory
-constexpr int kRankCap = 256;         // per-head frontiers this small are cut by explicit ranks
+static_assert(kBuckets == kThreads, "one histogram bucket per thread");
+
+enum HeadMode : int {
+  kModeRadix = 0,  // group being narrowed by key digits
+  kModeAll = 1,    // keep every candidate of the head
+  kModeThr = 2,    // keep iff key >= kthr
+  kModeTie = 3,    // keep iff key > kthr, or key == kthr within the segment's quota
+  kModeQuant = 4,  // first pass pending: buckets are a linear map of z
+};
 
 struct TravParams {
   const void* tree;
@@ -70,8 +86,7 @@ struct TravParams {
   int list_mode;
   int64_t seg;           // capacity of one segment (candidates), multiple of 32
   uint32_t* cand;        // [units][2][C][seg]   (head mask << 24) | node
-  float* zbuf;           // [units][G][C][seg]
-  uint32_t* kbits;       // [units][G][C][seg/32]
+  float* zbuf;           // [units][C][seg][G]   scores, candidate-major
   uint32_t* kept;        // [units][C][seg]     decode mode: union-kept level-1 nodes
   int32_t* n_kept;       // [units][C]
   int32_t* idx;          // [nq][Hq][idx_cap]   list mode
@@ -82,40 +97,64 @@ struct TravParams {
   int32_t* status;
 };
 
-// Per-CTA values read by the other CTAs of the cluster through DSMEM.
+// Cut state of one head. After every publish step it is identical on all CTAs
+// of the cluster (each copies it from the head's owner).
+struct HeadState {
+  unsigned long long above;  // mass of the candidates ranked above the current group
+  unsigned long long need;   // coverage target
+  unsigned long long bmass;  // mass of the current group
+  unsigned int prefix;       // kModeRadix: key prefix shared by the current group
+  int shift;                 // kModeRadix: key bits below the prefix
+  unsigned int kgmin, kgmax; // key range of the group (its members are exactly the
+                             // head's candidates with a key in this range)
+  float zlo, zscale;         // kModeQuant: bucket = clamp(floor((z - zlo) zscale))
+  unsigned int cabove;       // candidates ranked above the current group
+  unsigned int bcnt;         // candidates in the current group
+  int mode;                  // HeadMode
+  unsigned int kthr;         // threshold key of the final rule
+  unsigned int count;        // kept candidates (the level count)
+  unsigned int quota[kMaxCluster];  // kModeTie: kept members of each segment
+};
+
+// Per-CTA values read by the other CTAs through DSMEM after the score sync;
+// double-buffered by level parity so a fast CTA never overwrites a value a
+// slow one is still reading.
 struct Xch {
-  unsigned int count;            // candidates in my segment at this level
+  unsigned int count;             // candidates in my segment
+  unsigned int hcount[kMaxGroup]; // ... of which in head h's frontier
   float zmax[kMaxGroup];
   float zmin[kMaxGroup];
 };
 
-// Every member read or written with 8/16-byte vector accesses is 16-aligned.
 struct Smem {
-  alignas(16) unsigned int hlo[kBuckets];
-  alignas(16) unsigned int hhi[kBuckets];
-  alignas(16) unsigned int hcnt[kBuckets];
-  alignas(16) float ring_z[kStages][kChunk];
-  alignas(16) uint32_t ring_c[kStages][kChunk];
-  alignas(16) float list_z[kListCap];
-  alignas(16) uint32_t list_pos[kListCap];   // (segment << 24) | index: ascending = node order
-  alignas(16) float q[kMaxGroup * 128];      // [i][8] fp32, i < D (float4 reads)
-  unsigned int list_n;
-  unsigned int seg_n[kMaxCluster];
-  unsigned int chunk_start[kMaxCluster + 1];
-  unsigned int res_base[kMaxCluster];   // resident copy: segment r at ring[res_base[r]]
-  float g_zmax[kMaxCluster][kMaxGroup];  // every rank's segment extremes, gathered once
-  float g_zmin[kMaxCluster][kMaxGroup];
+  alignas(16) unsigned int hist_lo[kMaxGroup][kBuckets];       // bucket masses, low and
+  alignas(16) unsigned int hist_hi[kMaxGroup][kBuckets];       // high 32 bits
+  alignas(16) unsigned int hist_c[kMaxGroup][kBuckets];        // bucket counts
+  alignas(16) float q[kMaxGroup * 128];                        // [i][8] fp32, i < D
+  HeadState pub[kMaxGroup];   // owner's result of the last pass
+  HeadState st[kMaxGroup];    // this CTA's copy of every head's state
+  Xch xch[2];
+  unsigned int seg_n[kMaxCluster];     // every rank's segment size at this level
+  float zmax[kMaxGroup];               // cluster-wide score maximum per head
+  unsigned long long red_u64[kWarps][2];
+  unsigned int red_u32[kWarps][2];
+  unsigned int found[6];
+  unsigned long long found_u64[2];
+  unsigned int kc[kMaxGroup];          // kept candidates of my segment per head
+  unsigned int node0;                  // list mode: heads keeping node 0 (bit mask)
+  unsigned int tie_run[kMaxGroup];     // kModeTie: members seen so far (expand)
   float red_f[kWarps][kMaxGroup][2];
-  unsigned long long red_u64[kWarps];
-  unsigned int red_u32[kWarps];
-  unsigned long long bc_u64[4];
-  unsigned int bc_u32[8];
-  Xch xch;
+  float g_zmax[kMaxCluster][kMaxGroup];          // gathered per-rank extremes and counts
+  float g_zmin[kMaxCluster][kMaxGroup];
+  unsigned int g_hcnt[kMaxCluster][kMaxGroup];
+  unsigned int nh[kMaxGroup];                    // candidates of head h at this level
+  unsigned int tie_cnt[kMaxCluster];             // crossing-bucket members per rank
+  unsigned int my_hcnt[kMaxGroup];               // my segment's candidates in head h's frontier
 };
 
 // Exclusive scan of v over the CTA in thread order; *total receives the sum.
 __device__ __forceinline__ unsigned int block_excl_scan(unsigned int v, unsigned int* total,
-                                                        Smem& S) {
+                                                        Smem& S, int slot = 0) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   unsigned int x = v;
 #pragma unroll
@@ -123,12 +162,12 @@ __device__ __forceinline__ unsigned int block_excl_scan(unsigned int v, unsigned
     const unsigned int y = __shfl_up_sync(0xffffffffu, x, off);
     if (lane >= off) x += y;
   }
-  if (lane == 31) S.red_u32[warp] = x;
+  if (lane == 31) S.red_u32[warp][slot] = x;
   __syncthreads();
   unsigned int wbase = 0, tot = 0;
 #pragma unroll
   for (int w = 0; w < kWarps; ++w) {
-    const unsigned int s = S.red_u32[w];
+    const unsigned int s = S.red_u32[w][slot];
     if (w < warp) wbase += s;
     tot += s;
   }
@@ -137,47 +176,7 @@ __device__ __forceinline__ unsigned int block_excl_scan(unsigned int v, unsigned
   return wbase + x - v;
 }
 
-__device__ __forceinline__ unsigned long long block_sum_u64(unsigned long long v, Smem& S) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-  if (lane == 0) S.red_u64[warp] = v;
-  __syncthreads();
-  unsigned long long t = 0;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w) t += S.red_u64[w];
-  __syncthreads();
-  return t;
-}
-
-// Exclusive scan of a u64 over the CTA in thread order.
-__device__ __forceinline__ unsigned long long block_excl_scan_u64(unsigned long long v, Smem& S) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  unsigned long long x = v;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const unsigned long long y = __shfl_up_sync(0xffffffffu, x, off);
-    if (lane >= off) x += y;
-  }
-  if (lane == 31) S.red_u64[warp] = x;
-  __syncthreads();
-  unsigned long long wbase = 0;
-#pragma unroll
-  for (int w = 0; w < kWarps; ++w)
-    if (w < warp) wbase += S.red_u64[w];
-  __syncthreads();
-  return wbase + x - v;
-}
-
-// Exact 64-bit accumulation into a (lo, hi) pair of 32-bit shared counters.
-__device__ __forceinline__ void hist_add(Smem& S, int b, unsigned long long m, unsigned int n) {
-  const unsigned int lo = (unsigned int)m;
-  const unsigned int old = atomicAdd(&S.hlo[b], lo);
-  const unsigned int hi = (unsigned int)(m >> 32) + ((old + lo < old) ? 1u : 0u);
-  if (hi) atomicAdd(&S.hhi[b], hi);
-  atomicAdd(&S.hcnt[b], n);
-}
-
+// ceil(T * pq / 2^32) without overflow.
 __device__ __forceinline__ unsigned long long ceil_mul_shift32(unsigned long long T,
                                                                unsigned long long pq) {
   const unsigned long long lo = T * pq;
@@ -187,213 +186,74 @@ __device__ __forceinline__ unsigned long long ceil_mul_shift32(unsigned long lon
   return r;
 }
 
-
-// Streams head h's (score, candidate) pairs of every segment, in ascending node
-// order, through a cp.async ring; f(z[8], c[8], nvalid, pos0) sees the 8
-// consecutive candidates of this thread (pos0 = (segment << 24) | first index).
-constexpr int kResidentCap = kStages * kChunk;  // candidates kept resident per head
-
-// Copies head h's scores and candidate entries of every segment into the ring
-// (segment r at res_base[r], 32-aligned); returns false if they do not fit.
-__device__ __forceinline__ bool load_resident(Smem& S, int C, const uint32_t* cbase,
-                                              const float* zbase, int64_t seg) {
-  float* rz = &S.ring_z[0][0];
-  uint32_t* rc = &S.ring_c[0][0];
-  unsigned int acc = 0;
-  for (int r = 0; r < C; ++r) acc += (S.seg_n[r] + 31u) & ~31u;
-  if (acc > (unsigned)kResidentCap) return false;
-  if (threadIdx.x == 0) {
-    unsigned int b = 0;
-    for (int r = 0; r < C; ++r) {
-      S.res_base[r] = b;
-      b += (S.seg_n[r] + 31u) & ~31u;
-    }
-  }
-  __syncthreads();
-  for (int r = 0; r < C; ++r) {
-    const int pieces = (int)((S.seg_n[r] + 3u) >> 2);
-    for (int e = threadIdx.x; e < pieces; e += kThreads) {
-      cp_async16(rz + S.res_base[r] + e * 4, zbase + r * seg + e * 4);
-      cp_async16(rc + S.res_base[r] + e * 4, cbase + r * seg + e * 4);
-    }
-  }
-  cp_async_commit();
-  cp_async_wait<0>();
-  __syncthreads();
-  return true;
+// L2 eviction policies: summary rows stream through L2 once (evict first);
+// the per-candidate scores are re-read by every pass of the cut (evict last).
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t pol;
+  asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t pol;
+  asm("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint4 ld_policy(const uint4* ptr, uint64_t pol) {
+  uint4 v;
+  asm("ld.global.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+      : "l"(ptr), "l"(pol));
+  return v;
+}
+__device__ __forceinline__ void st_policy(float4* ptr, float4 v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(ptr), "f"(v.x),
+               "f"(v.y), "f"(v.z), "f"(v.w), "l"(pol)
+               : "memory");
 }
 
-// Visits head h's (score, candidate) pairs of every segment, in ascending node
-// order; f(z[8], c[8], nvalid, pos0, idx0, r) sees 8 consecutive candidates of
-// segment r starting at index idx0 (pos0 = (r << 24) | idx0). Chunks come from
-// the resident copy, or are streamed through the cp.async ring.
-template <typename F>
-__device__ __forceinline__ void stream_head(Smem& S, int C, const uint32_t* cbase,
-                                            const float* zbase, int64_t seg, bool resident,
-                                            F&& f) {
-  const int tid = threadIdx.x;
-  const int nchunks = (int)S.chunk_start[C];
-  auto locate = [&](int k, int& r, int64_t& off) {
-    r = 0;
-    while ((int)S.chunk_start[r + 1] <= k) ++r;
-    off = (int64_t)(k - (int)S.chunk_start[r]) * kChunk;
-  };
-  auto issue = [&](int k, int st) {
-    if (k < nchunks) {
-      int r;
-      int64_t off;
-      locate(k, r, off);
-      const int64_t n = S.seg_n[r];
-      const int len = (int)((n - off) < kChunk ? (n - off) : kChunk);
-      const int pieces = (len + 3) >> 2;  // 16-byte pieces (segments are 128-byte aligned)
-      for (int e = tid; e < pieces; e += kThreads) {
-        cp_async16(&S.ring_z[st][e * 4], zbase + r * seg + off + e * 4);
-        cp_async16(&S.ring_c[st][e * 4], cbase + r * seg + off + e * 4);
-      }
-    }
-    cp_async_commit();
-  };
-  if (!resident) {
+// The G scores of candidate i (candidate-major rows of G floats).
+template <int G>
+__device__ __forceinline__ void load_scores(const float* zown, int64_t i, float* z) {
+  if constexpr (G >= 4) {
 #pragma unroll
-    for (int st = 0; st < kStages - 1; ++st) issue(st, st);
-  }
-  for (int k = 0; k < nchunks; ++k) {
-    const float* zsrc;
-    const uint32_t* csrc;
-    int r;
-    int64_t off;
-    locate(k, r, off);
-    if (!resident) {
-      issue(k + kStages - 1, (k + kStages - 1) % kStages);
-      cp_async_wait<kStages - 1>();
-      __syncthreads();
-      zsrc = &S.ring_z[k % kStages][0];
-      csrc = &S.ring_c[k % kStages][0];
-    } else {
-      zsrc = &S.ring_z[0][0] + S.res_base[r] + off;
-      csrc = &S.ring_c[0][0] + S.res_base[r] + off;
+    for (int j = 0; j < G / 4; ++j) {
+      const float4 v = *reinterpret_cast<const float4*>(zown + i * G + 4 * j);
+      z[4 * j] = v.x;
+      z[4 * j + 1] = v.y;
+      z[4 * j + 2] = v.z;
+      z[4 * j + 3] = v.w;
     }
-    const int64_t n = S.seg_n[r];
-    const int len = (int)((n - off) < kChunk ? (n - off) : kChunk);
-    const int first = tid * 8;
-    const int nvalid = len - first < 0 ? 0 : (len - first > 8 ? 8 : len - first);
-    float z[8];
-    uint32_t c[8];
-    if (nvalid > 0) {
-      const float4 z0 = *reinterpret_cast<const float4*>(zsrc + first);
-      const float4 z1 = *reinterpret_cast<const float4*>(zsrc + first + 4);
-      const uint4 c0 = *reinterpret_cast<const uint4*>(csrc + first);
-      const uint4 c1 = *reinterpret_cast<const uint4*>(csrc + first + 4);
-      z[0] = z0.x; z[1] = z0.y; z[2] = z0.z; z[3] = z0.w;
-      z[4] = z1.x; z[5] = z1.y; z[6] = z1.z; z[7] = z1.w;
-      c[0] = c0.x; c[1] = c0.y; c[2] = c0.z; c[3] = c0.w;
-      c[4] = c1.x; c[5] = c1.y; c[6] = c1.z; c[7] = c1.w;
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        z[j] = 0.0f;
-        c[j] = 0u;
-      }
-    }
-    f(z, c, nvalid, ((uint32_t)r << 24) | (uint32_t)(off + first), off + first, r);
-    if (!resident) __syncthreads();
-  }
-  if (!resident) cp_async_wait<0>();
-}
-
-// Adds (mass m, count n) to bucket d, aggregating across the warp when every
-// participating lane hits the same bucket.
-__device__ __forceinline__ void hist_add_warp(Smem& S, bool valid, uint32_t d,
-                                              unsigned long long m, unsigned int n) {
-  const int lane = threadIdx.x & 31;
-  const unsigned vmask = __ballot_sync(0xffffffffu, valid);
-  if (vmask == 0u) return;
-  const int leader = __ffs(vmask) - 1;
-  const uint32_t d0 = __shfl_sync(0xffffffffu, d, leader);
-  if (__all_sync(0xffffffffu, !valid || d == d0)) {
-    unsigned long long s = valid ? m : 0ull;
-    unsigned int c = valid ? n : 0u;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      s += __shfl_xor_sync(0xffffffffu, s, off);
-      c += __shfl_xor_sync(0xffffffffu, c, off);
-    }
-    if (lane == leader) hist_add(S, (int)d0, s, c);
-  } else if (valid) {
-    hist_add(S, (int)d, m, n);
+  } else if constexpr (G == 2) {
+    const float2 v = *reinterpret_cast<const float2*>(zown + i * 2);
+    z[0] = v.x;
+    z[1] = v.y;
+  } else {
+    z[0] = zown[i];
   }
 }
 
-// Crossing digit of the current histogram: above + mass(digits > d) < need <=
-// above + mass(digits >= d). Returns false if none exists (never for exact sums).
-__device__ __forceinline__ bool find_crossing(Smem& S, int nb, unsigned long long above,
-                                              unsigned long long need, uint32_t* beta,
-                                              unsigned long long* above_out,
-                                              unsigned long long* bmass, unsigned int* bcnt) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int kPerT = kBuckets / kThreads;
-  unsigned long long mloc[kPerT];
-  unsigned long long tsum = 0;
-#pragma unroll
-  for (int j = 0; j < kPerT; ++j) {
-    const int d = tid * kPerT + j;  // buckets >= nb were not cleared this pass
-    mloc[j] = d < nb ? ((unsigned long long)S.hhi[d] << 32) | S.hlo[d] : 0ull;
-    tsum += mloc[j];
-  }
-  unsigned long long x = tsum;  // suffix over lanes (higher lanes = higher digits)
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const unsigned long long y = __shfl_down_sync(0xffffffffu, x, off);
-    if (lane + off < 32) x += y;
-  }
-  if (lane == 0) S.red_u64[warp] = x;
-  if (tid == 0) S.bc_u32[2] = 0xffffffffu;
-  __syncthreads();
-  unsigned long long run = above + (x - tsum);
-#pragma unroll
-  for (int w2 = 0; w2 < kWarps; ++w2)
-    if (w2 > warp) run += S.red_u64[w2];
-#pragma unroll
-  for (int j = kPerT - 1; j >= 0; --j) {
-    const int d = tid * kPerT + j;
-    if (run < need && run + mloc[j] >= need) {
-      S.bc_u32[2] = (unsigned)d;
-      S.bc_u64[0] = run;
-      S.bc_u64[1] = mloc[j];
-      S.bc_u32[3] = S.hcnt[d];
-    }
-    run += mloc[j];
-  }
-  __syncthreads();
-  const bool ok = S.bc_u32[2] != 0xffffffffu;
-  *beta = S.bc_u32[2];
-  *above_out = S.bc_u64[0];
-  *bmass = S.bc_u64[1];
-  *bcnt = S.bc_u32[3];
-  __syncthreads();
-  return ok;
-}
-
-__device__ __forceinline__ void clear_hist(Smem& S, int nb) {
-  for (int e = threadIdx.x; e < nb; e += kThreads) {
-    S.hlo[e] = 0u;
-    S.hhi[e] = 0u;
-    S.hcnt[e] = 0u;
-  }
-  __syncthreads();
+// First-pass bucket of score z: a linear map of [zlo, zlo + 256 / zscale)
+// onto 0..255, clamped. Non-decreasing in z, and evaluated with the same
+// operations on every CTA.
+__device__ __forceinline__ uint32_t quant_bucket(float z, float zlo, float zscale) {
+  const float f = __fmul_rn(__fsub_rn(z, zlo), zscale);
+  if (!(f > 0.0f)) return 0u;
+  return f >= 255.0f ? 255u : (uint32_t)f;
 }
 
 // Score candidates [0, n) of a segment against G queries; 4 candidates per
-// thread so that each broadcast of q[i][0..G) feeds 4*G chains. zseg points at
-// head 0's array; head h's array is zstride further.
+// thread so that each broadcast of q[i][0..G) feeds 4*G chains. The G scores
+// of candidate i go to zseg[i*G .. i*G+G). lmax/lmin accumulate the extremes
+// over the candidates in each head's frontier.
 template <typename T, int D, int G>
 __device__ __forceinline__ void score_segment(const TravParams& p, Smem& S, const T* lvl,
-                                              const uint32_t* cand, float* zseg, int64_t zstride,
-                                              int64_t n, float lns, float* lmax, float* lmin,
-                                              bool top, int64_t top_base) {
+                                              const uint32_t* cand, float* zseg, int64_t n,
+                                              float lns, float* lmax, float* lmin, bool top,
+                                              int64_t top_base) {
   constexpr int kPer = Elem<T>::kPerChunk;
   constexpr int kNch = D * (int)sizeof(T) / 16;
   const int tid = threadIdx.x;
+  const uint64_t pol_rows = policy_evict_first(), pol_z = policy_evict_last();
   for (int64_t base = 0; base < n; base += kThreads * kCandPerThread) {
     const uint4* rows[kCandPerThread];
     uint32_t pm[kCandPerThread];
@@ -419,7 +279,7 @@ __device__ __forceinline__ void score_segment(const TravParams& p, Smem& S, cons
     uint4 cur[kCandPerThread], nxt[kCandPerThread];
 #pragma unroll
     for (int k = 0; k < kCandPerThread; ++k) {
-      cur[k] = ok[k] ? rows[k][0] : make_uint4(0, 0, 0, 0);
+      cur[k] = ok[k] ? ld_policy(rows[k], pol_rows) : make_uint4(0, 0, 0, 0);
       nxt[k] = cur[k];
     }
 #pragma unroll 1
@@ -427,7 +287,7 @@ __device__ __forceinline__ void score_segment(const TravParams& p, Smem& S, cons
       if (ch + 1 < kNch) {
 #pragma unroll
         for (int k = 0; k < kCandPerThread; ++k)
-          nxt[k] = ok[k] ? rows[k][ch + 1] : make_uint4(0, 0, 0, 0);
+          nxt[k] = ok[k] ? ld_policy(rows[k] + ch + 1, pol_rows) : make_uint4(0, 0, 0, 0);
       }
       float x[kCandPerThread][kPer];
 #pragma unroll
@@ -465,18 +325,242 @@ __device__ __forceinline__ void score_segment(const TravParams& p, Smem& S, cons
     for (int k = 0; k < kCandPerThread; ++k) {
       if (!ok[k]) continue;
       const int64_t i = base + k * kThreads + tid;
+      float z[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const float raw = (G == 1) ? acc1[k] : ((h & 1) ? acc[k][h / 2].y : acc[k][h / 2].x);
-        const float z = __fadd_rn(__fmul_rn(raw, p.inv_sqrt_d), lns);
-        zseg[(int64_t)h * zstride + i] = z;
+        z[h] = __fadd_rn(__fmul_rn(raw, p.inv_sqrt_d), lns);
         if ((pm[k] >> h) & 1u) {
-          lmax[h] = fmaxf(lmax[h], z);
-          lmin[h] = fminf(lmin[h], z);
+          lmax[h] = fmaxf(lmax[h], z[h]);
+          lmin[h] = fminf(lmin[h], z[h]);
         }
+      }
+      if constexpr (G >= 4) {
+#pragma unroll
+        for (int j = 0; j < G / 4; ++j)
+          st_policy(reinterpret_cast<float4*>(zseg + i * G + 4 * j),
+                    make_float4(z[4 * j], z[4 * j + 1], z[4 * j + 2], z[4 * j + 3]), pol_z);
+      } else if constexpr (G == 2) {
+        *reinterpret_cast<float2*>(zseg + i * 2) = make_float2(z[0], z[1]);
+      } else {
+        zseg[i] = z[0];
       }
     }
   }
+}
+
+// Adds (mass m, count 1) to bucket d of head h. The 64-bit mass goes into two
+// 32-bit counters with an explicit carry (a 64-bit shared-memory add is far
+// slower under contention).
+__device__ __forceinline__ void hist_add(Smem& S, int h, uint32_t d, unsigned long long m) {
+  const unsigned lo = (unsigned)m;
+  const unsigned old = atomicAdd(&S.hist_lo[h][d], lo);
+  const unsigned hi = (unsigned)(m >> 32) + ((old + lo < old) ? 1u : 0u);
+  if (hi) atomicAdd(&S.hist_hi[h][d], hi);
+  atomicAdd(&S.hist_c[h][d], 1u);
+}
+
+// Inverse of order_key.
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Smallest key in [lo, hi] whose first-pass bucket is >= beta; the bucket of
+// key_float(hi) must be >= beta. Binary search over the key order.
+__device__ __forceinline__ uint32_t quant_first_key(float zlo, float zscale, uint32_t beta,
+                                                    uint32_t lo, uint32_t hi) {
+  while (lo < hi) {
+    const uint32_t mid = lo + (hi - lo) / 2;
+    if (quant_bucket(key_float(mid), zlo, zscale) >= beta) hi = mid;
+    else lo = mid + 1;
+  }
+  return lo;
+}
+
+// First key of bucket beta (beta >= 1): the search starts in a window of 512
+// keys around the estimate zlo + beta / zscale and widens to the whole key
+// range of the finite scores when the window does not bracket the boundary.
+__device__ __forceinline__ uint32_t quant_boundary(float zlo, float zscale, uint32_t beta) {
+  const uint32_t kneg = order_key(-INFINITY), kpos = order_key(INFINITY);
+  const uint32_t ke = order_key(__fadd_rn(zlo, __fdiv_rn((float)beta, zscale)));
+  uint32_t lo = ke > kneg + 256u ? ke - 256u : kneg;
+  uint32_t hi = ke < kpos - 256u ? ke + 256u : kpos;
+  if (lo < kneg || hi > kpos || lo > hi || quant_bucket(key_float(lo), zlo, zscale) >= beta ||
+      quant_bucket(key_float(hi), zlo, zscale) < beta) {
+    lo = kneg;
+    hi = kpos;
+  }
+  return quant_first_key(zlo, zscale, beta, lo, hi);
+}
+
+// Key interval [*klo, *khi] of the finite scores whose first-pass bucket is
+// beta (an interval, as the bucket map is non-decreasing in the score).
+__device__ __forceinline__ void quant_interval(float zlo, float zscale, uint32_t beta,
+                                               uint32_t* klo, uint32_t* khi) {
+  *klo = beta == 0u ? order_key(-INFINITY) : quant_boundary(zlo, zscale, beta);
+  *khi = beta >= (uint32_t)kBuckets - 1u || zscale == 0.0f
+             ? order_key(INFINITY)
+             : quant_boundary(zlo, zscale, beta + 1u) - 1u;
+}
+
+// Digit width and position of a kModeRadix pass over the group [kgmin, kgmax]
+// (kgmin < kgmax): the bits below the range's common prefix, 8 at a time.
+__device__ __forceinline__ void radix_digit(unsigned kgmin, unsigned kgmax, int* sh, int* w) {
+  const int shift = 32 - __clz(kgmin ^ kgmax);
+  *w = shift < kDigit ? shift : kDigit;
+  *sh = shift - *w;
+}
+
+// Owner step of one pass for head h (every thread of the owner CTA calls it):
+// sums the C per-rank histograms of h through DSMEM, finds the bucket where
+// the mass in descending score order reaches the target, narrows the head's
+// state to that bucket's group and leaves it in S.pub[h].
+template <int G>
+__device__ __noinline__ void owner_pass(const TravParams& p, Smem& S, cg::cluster_group& cluster,
+                                        int C, int h) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const HeadState s0 = S.st[h];
+  const bool quant = s0.mode == kModeQuant;
+  int nb = kBuckets;
+  if (!quant) {
+    int sh, w;
+    radix_digit(s0.kgmin, s0.kgmax, &sh, &w);
+    nb = 1 << w;
+  }
+  unsigned long long m = 0;
+  unsigned int c = 0;
+  if (tid < nb) {
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r) {
+      if (r < C) {
+        const Smem* R = cluster.map_shared_rank(&S, r);
+        m += ((unsigned long long)R->hist_hi[h][tid] << 32) | R->hist_lo[h][tid];
+        c += R->hist_c[h][tid];
+      }
+    }
+  }
+  // suffix sums over buckets (thread t = bucket t; higher buckets rank first)
+  unsigned long long xs = m;
+  unsigned int xc = c;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const unsigned long long ym = __shfl_down_sync(0xffffffffu, xs, off);
+    const unsigned int yc = __shfl_down_sync(0xffffffffu, xc, off);
+    if (lane + off < 32) {
+      xs += ym;
+      xc += yc;
+    }
+  }
+  if (lane == 0) {
+    S.red_u64[warp][0] = xs;
+    S.red_u32[warp][0] = xc;
+  }
+  if (tid == 0) S.found[0] = 0xffffffffu;
+  __syncthreads();
+  unsigned long long hm = 0, total = 0;
+  unsigned int hc = 0;
+#pragma unroll
+  for (int w2 = 0; w2 < kWarps; ++w2) {
+    total += S.red_u64[w2][0];
+    if (w2 > warp) {
+      hm += S.red_u64[w2][0];
+      hc += S.red_u32[w2][0];
+    }
+  }
+  // the first pass sees every candidate of the head: its total fixes the target
+  const unsigned long long need = quant ? ceil_mul_shift32(total, p.p_q) : s0.need;
+  const unsigned long long above = s0.above + hm + (xs - m);  // mass of buckets > tid
+  if (tid < nb && above < need && above + m >= need) {
+    S.found[0] = (unsigned)tid;
+    S.found[1] = s0.cabove + hc + (xc - c);
+    S.found[2] = c;
+    S.found_u64[0] = above;
+    S.found_u64[1] = m;
+  }
+  __syncthreads();
+  const unsigned beta = S.found[0];
+  const bool ok = beta != 0xffffffffu;
+  const unsigned bcnt = ok ? S.found[2] : 0u;
+  // the group's key interval: the bucket's interval on the first pass, the
+  // digit's sub-interval of the previous group on later passes
+  uint32_t gmin = 0, gmax = 0;
+  if (ok) {
+    if (quant) {
+      if (tid == 0) quant_interval(s0.zlo, s0.zscale, beta, &S.found[3], &S.found[4]);
+      __syncthreads();
+      gmin = S.found[3];
+      gmax = S.found[4];
+    } else {
+      int sh, w;
+      radix_digit(s0.kgmin, s0.kgmax, &sh, &w);
+      const uint32_t top = (uint32_t)(((unsigned long long)s0.kgmin >> (sh + w)) << (sh + w));
+      const uint32_t dlo = top | (beta << sh);
+      const uint32_t dhi = dlo | (uint32_t)((1ull << sh) - 1ull);
+      gmin = dlo > s0.kgmin ? dlo : s0.kgmin;
+      gmax = dhi < s0.kgmax ? dhi : s0.kgmax;
+    }
+  }
+  const bool tie = ok && bcnt > 1u && gmin == gmax;
+  if (tie && tid < C) {  // members of the tie group in each segment
+    const Smem* R = cluster.map_shared_rank(&S, tid);
+    S.tie_cnt[tid] = R->hist_c[h][beta];
+  }
+  if (tie) __syncthreads();
+  if (tid == 0) {
+    HeadState ns = s0;
+    ns.need = need;
+    if (!ok) {  // cannot happen with exact sums; keep everything rather than loop
+      raise_status(p.status, ZHA_ERR_INTERNAL);
+      ns.mode = kModeAll;
+      ns.count = S.nh[h];
+    } else {
+      ns.above = S.found_u64[0];
+      ns.cabove = S.found[1];
+      ns.bmass = S.found_u64[1];
+      ns.bcnt = bcnt;
+      ns.kgmin = gmin;
+      ns.kgmax = gmax;
+      ns.mode = kModeRadix;
+      if (bcnt == 1u) {
+        ns.mode = kModeThr;  // the group's only member is the last kept candidate;
+        ns.kthr = ns.kgmin;  // no other candidate has a key in the group's interval
+        ns.count = ns.cabove + 1u;
+      } else if (ns.kgmin == ns.kgmax) {
+        // bcnt members share one key, hence one z and one mass: keep the first
+        // tie_need of them in node order
+        const unsigned long long mt = ns.bmass / bcnt;
+        const unsigned long long rem = need - ns.above;
+        const unsigned long long tn = mt ? (rem + mt - 1) / mt : bcnt;
+        ns.kthr = ns.kgmin;
+        if (tn >= bcnt) {
+          ns.mode = kModeThr;
+          ns.count = ns.cabove + bcnt;
+        } else {
+          ns.mode = kModeTie;
+          ns.count = ns.cabove + (unsigned)tn;
+          unsigned long long run = 0;
+          for (int r = 0; r < C; ++r) {
+            const unsigned long long cr = S.tie_cnt[r];
+            ns.quota[r] = (unsigned)(run >= tn ? 0ull : (tn - run < cr ? tn - run : cr));
+            run += cr;
+          }
+        }
+      }
+    }
+    S.pub[h] = ns;
+  }
+  __syncthreads();
+}
+
+// Final keep rule of one head for a candidate with order key `key`; *member
+// reports a kModeTie candidate whose keep depends on its rank among the ties.
+__device__ __forceinline__ bool keep_rule(int mode, unsigned kthr, uint32_t key, bool* member) {
+  *member = false;
+  if (mode == kModeAll) return true;
+  if (mode == kModeThr) return key >= kthr;
+  if (key > kthr) return true;
+  *member = key == kthr;
+  return false;
 }
 
 template <typename T, int D, int G>
@@ -524,11 +608,8 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
   __syncthreads();
 
   uint32_t* cand_u = p.cand + (int64_t)unit * 2 * C * seg;
-  float* z_u = p.zbuf + (int64_t)unit * G * C * seg;
-  uint32_t* kb_u = p.kbits + (int64_t)unit * G * C * (seg / 32);
-  auto cptr = [&](int buf, int r) { return cand_u + ((int64_t)buf * C + r) * seg; };
-  auto zptr = [&](int h, int r) { return z_u + ((int64_t)h * C + r) * seg; };
-  auto kptr = [&](int h, int r) { return kb_u + ((int64_t)h * C + r) * (seg / 32); };
+  float* zown = p.zbuf + ((int64_t)unit * C + rank) * seg * G;  // [seg][G]
+  auto cptr = [&](int buf) { return cand_u + ((int64_t)buf * C + rank) * seg; };
   int32_t* lc_base = p.level_counts ? p.level_counts + ((int64_t)qi * p.Hq + (int64_t)kvh * G) * p.L
                                     : nullptr;
 
@@ -550,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
     if (lc_base)
       for (int h = rank; h < G; h += C)
         for (int e = tid; e < p.L; e += kThreads) lc_base[(int64_t)h * p.L + e] = 0;
-    return;  // uniform across the cluster: no barrier is pending
+    return;  // uniform across the cluster and before any DSMEM access
   }
 
   // my segment at the top level: a contiguous range of the complete top nodes
@@ -561,432 +642,326 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
     const bool top = level == p.L;
     const T* lvl = static_cast<const T*>(p.tree) + p.level_off[level - 1] +
                    (int64_t)tree_unit * p.level_rows[level - 1] * D;
+    uint32_t* cc = cptr(cur);
     // ------------------------------------------------------------------
     // 1. score my segment
     // ------------------------------------------------------------------
-    float lmax[G], lmin[G];
+    {
+      float lmax[G], lmin[G];
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      lmax[h] = -INFINITY;
-      lmin[h] = INFINITY;
-    }
-    score_segment<T, D, G>(p, S, lvl, cptr(cur, rank), zptr(0, rank), (int64_t)C * seg, my_n,
-                           p.lnsize[level - 1], lmax, lmin, top, top_lo);
-    if (top) {  // materialise the top candidates (all heads)
-      uint32_t* cc = cptr(cur, rank);
-      for (int64_t i = tid; i < my_n; i += kThreads)
-        cc[i] = (((1u << G) - 1u) << 24) | (uint32_t)(top_lo + i);
-    }
+      for (int h = 0; h < G; ++h) {
+        lmax[h] = -INFINITY;
+        lmin[h] = INFINITY;
+      }
+      score_segment<T, D, G>(p, S, lvl, cc, zown, my_n, p.lnsize[level - 1], lmax, lmin, top,
+                             top_lo);
+      if (top)  // materialise the top candidates (all heads)
+        for (int64_t i = tid; i < my_n; i += kThreads)
+          cc[i] = (((1u << G) - 1u) << 24) | (uint32_t)(top_lo + i);
 #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      float mx = lmax[h], mn = lmin[h];
+      for (int h = 0; h < G; ++h) {
+        float mx = lmax[h], mn = lmin[h];
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+        for (int off = 16; off > 0; off >>= 1) {
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+          mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+        }
+        if (lane == 0) {
+          S.red_f[warp][h][0] = mx;
+          S.red_f[warp][h][1] = mn;
+        }
       }
-      if (lane == 0) {
-        S.red_f[warp][h][0] = mx;
-        S.red_f[warp][h][1] = mn;
+      __syncthreads();
+      Xch& X = S.xch[level & 1];
+      if (tid < G) {
+        float mx = -INFINITY, mn = INFINITY;
+        for (int w = 0; w < kWarps; ++w) {
+          mx = fmaxf(mx, S.red_f[w][tid][0]);
+          mn = fminf(mn, S.red_f[w][tid][1]);
+        }
+        X.zmax[tid] = mx;
+        X.zmin[tid] = mn;
+        X.hcount[tid] = top ? (unsigned int)my_n : S.my_hcnt[tid];
       }
+      if (tid == 0) X.count = (unsigned int)my_n;
     }
-    __syncthreads();
-    if (tid < G) {
-      float mx = -INFINITY, mn = INFINITY;
-      for (int w = 0; w < kWarps; ++w) {
-        mx = fmaxf(mx, S.red_f[w][tid][0]);
-        mn = fminf(mn, S.red_f[w][tid][1]);
-      }
-      S.xch.zmax[tid] = mx;
-      S.xch.zmin[tid] = mn;
-    }
-    if (tid == 0) S.xch.count = (unsigned int)my_n;
-    __syncthreads();
     cluster.sync();  // S1: every segment scored
     if (p.stats && tid == 0) atomicAdd(&p.stats[(int64_t)unit * p.L + (p.L - level)], (int)my_n);
 
     // ------------------------------------------------------------------
-    // 2. exact cut for the heads this CTA owns
+    // 2. distributed cut
     // ------------------------------------------------------------------
-    for (int e = tid; e < C * (2 * G + 1); e += kThreads) {  // one parallel DSMEM gather
-      const int r = e / (2 * G + 1), k = e % (2 * G + 1);
-      const Xch* rx = cluster.map_shared_rank(&S.xch, r);
+    for (int e = tid; e < C * (3 * G + 1); e += kThreads) {  // one parallel DSMEM gather
+      const int r = e / (3 * G + 1), k = e % (3 * G + 1);
+      const Xch* rx = &cluster.map_shared_rank(&S, r)->xch[level & 1];
       if (k == 0) S.seg_n[r] = rx->count;
       else if (k <= G) S.g_zmax[r][k - 1] = rx->zmax[k - 1];
-      else S.g_zmin[r][k - 1 - G] = rx->zmin[k - 1 - G];
+      else if (k <= 2 * G) S.g_zmin[r][k - 1 - G] = rx->zmin[k - 1 - G];
+      else S.g_hcnt[r][k - 1 - 2 * G] = rx->hcount[k - 1 - 2 * G];
     }
     __syncthreads();
-    if (tid == 0) {
-      unsigned int acc = 0;
+    if (tid < G) {
+      float mx = -INFINITY, mn = INFINITY;
+      unsigned int n = 0;
       for (int r = 0; r < C; ++r) {
-        S.chunk_start[r] = acc;
-        acc += (S.seg_n[r] + kChunk - 1) / kChunk;
+        mx = fmaxf(mx, S.g_zmax[r][tid]);
+        mn = fminf(mn, S.g_zmin[r][tid]);
+        n += S.g_hcnt[r][tid];
       }
-      S.chunk_start[C] = acc;
+      S.zmax[tid] = mx;
+      S.nh[tid] = n;
+      HeadState s{};
+      s.count = n;
+      if (p.keep_all || n == 0u) {
+        s.mode = kModeAll;
+      } else {
+        // the first pass spreads the head's scores over 256 linear buckets;
+        // scores more than 32 below the maximum carry zero mass and share
+        // bucket 0
+        s.mode = kModeQuant;
+        const float lo = fmaxf(mn, __fsub_rn(mx, 32.0f));
+        s.zlo = lo;
+        s.zscale = mx > lo ? __fdiv_rn(256.0f, __fsub_rn(mx, lo)) : 0.0f;
+      }
+      S.st[tid] = s;
     }
     __syncthreads();
-    for (int h = rank; h < G; h += C) {
-      const uint32_t* cseg = cptr(cur, 0);  // segment r at cseg + r * seg
-      const float* zseg = zptr(h, 0);
-      if (tid == 0) {
-        float mx = -INFINITY, mn = INFINITY;
-        for (int r = 0; r < C; ++r) {
-          mx = fmaxf(mx, S.g_zmax[r][h]);
-          mn = fminf(mn, S.g_zmin[r][h]);
-        }
-        S.bc_u32[0] = __float_as_uint(mx);
-        S.bc_u32[1] = __float_as_uint(mn);
-        S.list_n = 0u;
+    for (int pass = 0; pass < 40; ++pass) {  // every pass strictly narrows each group
+      unsigned cut_heads = 0;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const int m = S.st[h].mode;
+        cut_heads |= (m == kModeRadix || m == kModeQuant ? 1u : 0u) << h;
+      }
+      if (!cut_heads) break;  // uniform: every CTA holds the same states
+      for (int e = tid; e < G * kBuckets; e += kThreads) {
+        (&S.hist_lo[0][0])[e] = 0u;
+        (&S.hist_hi[0][0])[e] = 0u;
+        (&S.hist_c[0][0])[e] = 0u;
       }
       __syncthreads();
-      const float zmax = __uint_as_float(S.bc_u32[0]);
-      // small frontiers: one copy into shared memory serves every pass
-      const bool resident = load_resident(S, C, cseg, zseg, seg);
-      if (resident) {
-        // gather head h's candidates (score, position); tiny frontiers are cut by
-        // explicit ranks instead of digit passes
-        if (tid == 0) S.list_n = 0u;
-        __syncthreads();
-        stream_head(S, C, cseg, zseg, seg, true,
-                    [&](const float* z, const uint32_t* c, int nvalid, uint32_t pos0, int64_t,
-                        int) {
+      // local histograms of my segment for every head still being cut; kHU
+      // consecutive candidates per thread, loaded up front
+      constexpr int kHU = G >= 8 ? 2 : 4;
+      for (int64_t base = 0; base < my_n; base += kHU * kThreads) {
+        const int64_t i0 = base + kHU * tid;
+        uint32_t hm[kHU];
+        float z[kHU][G];
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (j < nvalid && ((c[j] >> (24 + h)) & 1u)) {
-              const unsigned slot = atomicAdd(&S.list_n, 1u);
-              if (slot < (unsigned)kListCap) {
-                S.list_z[slot] = z[j];
-                S.list_pos[slot] = pos0 + (uint32_t)j;
-              }
+        for (int u = 0; u < kHU; ++u) hm[u] = i0 + u < my_n ? (cc[i0 + u] >> 24) & cut_heads : 0u;
+#pragma unroll
+        for (int u = 0; u < kHU; ++u)
+          if (i0 + u < my_n) load_scores<G>(zown, i0 + u, z[u]);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          if (!((cut_heads >> h) & 1u)) continue;
+          const HeadState& s = S.st[h];
+          const bool quant = s.mode == kModeQuant;
+          int sh = 0, w = 0;
+          if (!quant) radix_digit(s.kgmin, s.kgmax, &sh, &w);
+#pragma unroll
+          for (int u = 0; u < kHU; ++u) {
+            if (!((hm[u] >> h) & 1u)) continue;
+            const uint32_t key = order_key(z[u][h]);
+            uint32_t d;
+            if (quant) {
+              d = quant_bucket(z[u][h], s.zlo, s.zscale);
+            } else {
+              if (key < s.kgmin || key > s.kgmax) continue;
+              d = (key >> sh) & ((1u << w) - 1u);
             }
-        });
-        __syncthreads();
-      }
-      const int n_h = resident ? (int)S.list_n : kRankCap + 1;
-      __syncthreads();  // every warp has read list_n before the radix path resets it
-      if (n_h <= kRankCap) {
-        // rank_i = #{j : z_j > z_i, or z_j == z_i and pos_j < pos_i}; mass M_i is
-        // scattered to its rank; the cut is the shortest rank prefix reaching need
-        unsigned long long tloc = 0;
-        for (int i = tid; i < n_h; i += kThreads) {
-          const float zi = S.list_z[i];
-          const uint32_t pi = S.list_pos[i];
-          unsigned int rk = 0;
-          for (int j = 0; j < n_h; ++j) {
-            const float zj = S.list_z[j];
-            rk += (zj > zi || (zj == zi && S.list_pos[j] < pi)) ? 1u : 0u;
+            hist_add(S, h, d, mass_fixed(z[u][h], S.zmax[h]));
           }
-          const unsigned long long m = mass_fixed(zi, zmax);
-          tloc += m;
-          S.hcnt[i] = rk;
-          S.hlo[rk] = (unsigned int)m;
-          S.hhi[rk] = (unsigned int)(m >> 32);
-        }
-        const unsigned long long Tm = block_sum_u64(tloc, S);
-        const unsigned long long need_r = ceil_mul_shift32(Tm, p.p_q);
-        // thread t owns ranks [4t, 4t + 4)
-        unsigned long long part[4];
-        unsigned long long tsum = 0;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int rk = tid * 4 + j;
-          part[j] = rk < n_h ? (((unsigned long long)S.hhi[rk] << 32) | S.hlo[rk]) : 0ull;
-          tsum += part[j];
-        }
-        unsigned long long run = block_excl_scan_u64(tsum, S);
-        if (tid == 0) S.bc_u32[5] = (unsigned)n_h;
-        __syncthreads();
-        if (!p.keep_all) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int rk = tid * 4 + j;
-            if (rk < n_h && run < need_r && run + part[j] >= need_r) S.bc_u32[5] = (unsigned)rk + 1u;
-            run += part[j];
-          }
-        }
-        __syncthreads();
-        const unsigned int k = S.bc_u32[5];
-        // keep bits: clear head h's words, then set the kept ranks
-        for (int r = 0; r < C; ++r) {
-          uint32_t* kb = kptr(h, r);
-          for (int wd = tid; wd < (int)((S.seg_n[r] + 31u) >> 5); wd += kThreads) kb[wd] = 0u;
-        }
-        __syncthreads();
-        for (int i = tid; i < n_h; i += kThreads)
-          if (S.hcnt[i] < k) {
-            const uint32_t pi = S.list_pos[i];
-            atomicOr(&kptr(h, (int)(pi >> 24))[(pi & kNodeMask) >> 5], 1u << (pi & 31u));
-          }
-        if (lc_base && tid == 0) lc_base[(int64_t)h * p.L + (p.L - level)] = (int32_t)k;
-        __syncthreads();
-      }
-      if (n_h > kRankCap) {  // radix-select cut
-      if (tid == 0) S.list_n = 0u;
-      __syncthreads();
-      const uint32_t kmax = order_key(zmax), kmin = order_key(__uint_as_float(S.bc_u32[1]));
-      const uint32_t diff = kmax ^ kmin;
-      int shift = diff ? 32 - __clz(diff) : 0;
-      uint32_t prefix = (uint32_t)((uint64_t)kmax >> shift);
-      unsigned long long above = 0, need = 0, bmass = 1;
-      unsigned int bcnt = 1;
-      bool done = p.keep_all != 0;
-      bool listed = false;    // the current group lives in S.list_*
-      bool first = true;
-      for (int pass = 0; !done && pass < 4; ++pass) {  // <= ceil(32/11) digit passes
-        const int w = shift < kDigit ? shift : kDigit;
-        const int sh = shift - w;
-        clear_hist(S, 1 << w);
-        unsigned long long tloc = 0;
-        if (!listed) {
-          // full streaming pass over every candidate of head h
-          stream_head(S, C, cseg, zseg, seg, resident,
-                      [&](const float* z, const uint32_t* c, int nvalid, uint32_t, int64_t, int) {
-            // the 8 masses first (independent chains), then per-thread run-length
-            // aggregation of equal digits
-            bool ok[8];
-            uint32_t dg[8];
-            unsigned long long ms[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const uint32_t key = order_key(z[j]);
-              ok[j] = j < nvalid && ((c[j] >> (24 + h)) & 1u) &&
-                      (uint32_t)((uint64_t)key >> shift) == prefix;
-              dg[j] = (key >> sh) & ((1u << w) - 1u);
-              ms[j] = ok[j] ? mass_fixed(z[j], zmax) : 0ull;
-            }
-            bool have = false;
-            uint32_t rd = 0;
-            unsigned long long rm = 0;
-            unsigned int rc = 0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              if (ok[j]) {
-                tloc += ms[j];
-                if (have && dg[j] != rd) {
-                  hist_add(S, (int)rd, rm, rc);
-                  rm = 0;
-                  rc = 0;
-                }
-                have = true;
-                rd = dg[j];
-                rm += ms[j];
-                rc += 1;
-              }
-            }
-            hist_add_warp(S, have, rd, rm, rc);
-          });
-        } else {
-          const int nl = (int)S.list_n;
-          for (int base = 0; base < nl; base += kThreads) {
-            const int i = base + tid;
-            bool valid = false;
-            uint32_t d = 0;
-            unsigned long long m = 0;
-            if (i < nl) {
-              const uint32_t key = order_key(S.list_z[i]);
-              if ((uint32_t)((uint64_t)key >> shift) == prefix) {
-                valid = true;
-                d = (key >> sh) & ((1u << w) - 1u);
-                m = mass_fixed(S.list_z[i], zmax);
-              }
-            }
-            hist_add_warp(S, valid, d, m, 1u);
-          }
-        }
-        if (first) {
-          const unsigned long long Tm = block_sum_u64(tloc, S);
-          need = ceil_mul_shift32(Tm, p.p_q);
-          first = false;
-        }
-        __syncthreads();
-        uint32_t beta;
-        if (!find_crossing(S, 1 << w, above, need, &beta, &above, &bmass, &bcnt)) {
-          if (tid == 0) raise_status(p.status, ZHA_ERR_INTERNAL);  // never loop forever
-          done = true;
-          break;
-        }
-        prefix = (prefix << w) | beta;
-        shift = sh;
-        done = (bcnt == 1u) || (shift == 0);
-        if (!done && !listed && bcnt <= (unsigned)kListCap) {
-          // gather the crossing bucket's members once; later digits run in smem
-          stream_head(S, C, cseg, zseg, seg, resident,
-                      [&](const float* z, const uint32_t* c, int nvalid, uint32_t pos0, int64_t,
-                          int) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              if (j < nvalid && ((c[j] >> (24 + h)) & 1u) &&
-                  (uint32_t)((uint64_t)order_key(z[j]) >> shift) == prefix) {
-                const unsigned slot = atomicAdd(&S.list_n, 1u);
-                if (slot < (unsigned)kListCap) {
-                  S.list_z[slot] = z[j];
-                  S.list_pos[slot] = pos0 + (uint32_t)j;
-                }
-              }
-            }
-          });
-          listed = true;
         }
       }
-      // keep = (key >> shift) > prefix, plus the first tie_need members of the
-      // boundary group (key >> shift) == prefix in ascending node order
-      unsigned long long tie_need = 0;
-      if (!p.keep_all) {
-        const unsigned long long mt = bmass / bcnt;
-        tie_need = (need - above + mt - 1) / mt;
-      }
-      const bool rank_ties = !p.keep_all && tie_need < bcnt;
-      // with the boundary group listed, the kept ties are those whose position is
-      // at most the tie_need-th smallest position of the group
-      uint32_t pos_thr = 0xffffffffu;
-      const bool thr_mode = rank_ties && listed;
-      if (thr_mode) {
-        if (tid == 0) S.bc_u32[4] = 0u;
-        __syncthreads();
-        const int nl = (int)S.list_n;
-        for (int i = tid; i < nl; i += kThreads) {
-          if ((uint32_t)((uint64_t)order_key(S.list_z[i]) >> shift) != prefix) continue;
-          unsigned int rk = 0;  // members of the group with a smaller position
-          for (int j = 0; j < nl; ++j)
-            if ((uint32_t)((uint64_t)order_key(S.list_z[j]) >> shift) == prefix &&
-                S.list_pos[j] < S.list_pos[i])
-              ++rk;
-          if (rk + 1 == tie_need) S.bc_u32[4] = S.list_pos[i];
-        }
-        __syncthreads();
-        pos_thr = S.bc_u32[4];
-      }
-      unsigned int kept_loc = 0, tie_run = 0;
-      stream_head(S, C, cseg, zseg, seg, resident,
-                  [&](const float* z, const uint32_t* c, int nvalid, uint32_t pos0,
-                      int64_t idx0, int r) {
-        uint32_t bits = 0, ties = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (j < nvalid && ((c[j] >> (24 + h)) & 1u)) {
-            bool keep = true, tie = false;
-            if (!p.keep_all) {
-              const uint32_t pre = (uint32_t)((uint64_t)order_key(z[j]) >> shift);
-              keep = pre > prefix;
-              tie = pre == prefix;
-            }
-            if (tie) {
-              if (!rank_ties || (thr_mode && pos0 + (uint32_t)j <= pos_thr)) keep = true;
-              else if (!thr_mode) ties |= 1u << j;
-            }
-            if (keep) bits |= 1u << j;
-          }
-        }
-        if (rank_ties && !thr_mode) {  // ordered ranks of unlisted ties (rare)
-          unsigned int tot;
-          unsigned int rk = block_excl_scan(__popc(ties), &tot, S);
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if ((ties >> j) & 1u) {
-              if (tie_run + rk < tie_need) bits |= 1u << j;
-              ++rk;
-            }
-          tie_run += tot;
-        }
-        kept_loc += __popc(bits);
-        // 4 consecutive threads own the 32 candidates of one keep word
-        uint32_t word = bits << (8 * (threadIdx.x & 3));
-        word |= __shfl_xor_sync(0xffffffffu, word, 1);
-        word |= __shfl_xor_sync(0xffffffffu, word, 2);
-        if ((threadIdx.x & 3) == 0 && nvalid > 0) kptr(h, r)[(idx0 >> 5)] = word;
-      });
-      unsigned int ktot;
-      block_excl_scan(kept_loc, &ktot, S);
-      if (lc_base && tid == 0) lc_base[(int64_t)h * p.L + (p.L - level)] = (int32_t)ktot;
-      }  // radix-select cut
-
-      if (level == 1 && p.list_mode) {
-        // ascending token list of head h: {0} (unless node 0 is kept) +
-        // tokens of the kept level-1 nodes + causal tail
-        __syncthreads();
-        const int64_t qh = (int64_t)qi * p.Hq + (int64_t)kvh * G + h;
-        int32_t* out = p.idx + qh * p.idx_cap;
-        int r0 = 0;
-        while (r0 < C && S.seg_n[r0] == 0) ++r0;
-        const bool node0 =
-            r0 < C && (cptr(cur, r0)[0] & kNodeMask) == 0u && (kptr(h, r0)[0] & 1u);
-        const int64_t off0 = node0 ? 0 : 1;
-        if (!node0 && tid == 0 && p.idx_cap > 0) out[0] = 0;
-        unsigned int pos_run = 0;
-        for (int r = 0; r < C; ++r) {
-          const uint32_t* cc = cptr(cur, r);
-          const uint32_t* kb = kptr(h, r);
-          const int64_t n = S.seg_n[r];
-          for (int64_t base = 0; base < n; base += kThreads) {
-            const int64_t i = base + tid;
-            const bool kh = i < n && ((kb[i >> 5] >> (i & 31)) & 1u);
-            unsigned int tot;
-            const unsigned int rk = block_excl_scan(kh ? 1u : 0u, &tot, S);
-            if (kh) {
-              const int64_t pos = off0 + (int64_t)b * (pos_run + rk);
-              const int64_t node = cc[i] & kNodeMask;
-              for (int c = 0; c < b; ++c)
-                if (pos + c < p.idx_cap) out[pos + c] = (int32_t)(node * b + c);
-            }
-            pos_run += tot;
-          }
-        }
-        const int64_t tail_start = p.span[p.L] * T_top;
-        const int64_t tail_len = n_vis - tail_start;
-        const int64_t tail_pos = off0 + (int64_t)b * pos_run;
-        for (int64_t j = tid; j < tail_len; j += kThreads)
-          if (tail_pos + j < p.idx_cap) out[tail_pos + j] = (int32_t)(tail_start + j);
-        if (tid == 0) {
-          const int64_t n = tail_pos + tail_len;
-          p.n_idx[qh] = (int32_t)n;
-          if (n > p.idx_cap) raise_status(p.status, ZHA_ERR_CAPACITY);
+      cluster.sync();  // every rank's histograms complete
+      for (int h = rank; h < G; h += C)
+        if ((cut_heads >> h) & 1u) owner_pass<G>(p, S, cluster, C, h);
+      cluster.sync();  // every owner published
+      {  // copy the narrowed states of the heads being cut from their owners
+        constexpr int kWords = (int)(sizeof(HeadState) / 4);
+        for (int e = tid; e < G * kWords; e += kThreads) {
+          const int h = e / kWords, k = e % kWords;
+          if (!((cut_heads >> h) & 1u)) continue;
+          const Smem* R = cluster.map_shared_rank(&S, h % C);
+          reinterpret_cast<unsigned int*>(&S.st[h])[k] =
+              reinterpret_cast<const unsigned int*>(&R->pub[h])[k];
         }
       }
       __syncthreads();
     }
-    cluster.sync();  // S2: keep bits of every head written
+    if (tid < G) {
+      const int m = S.st[tid].mode;
+      if (m == kModeRadix || m == kModeQuant) {  // unreachable: passes always finish
+        if (rank == 0) raise_status(p.status, ZHA_ERR_INTERNAL);
+        S.st[tid].mode = kModeAll;
+        S.st[tid].count = S.nh[tid];
+      }
+    }
+    if (lc_base && rank == 0 && tid < G)
+      lc_base[(int64_t)tid * p.L + (p.L - level)] = (int32_t)S.st[tid].count;
 
     // ------------------------------------------------------------------
-    // 3. expand my segment into the next level's candidates
+    // 3. expand my segment with the final rules
     // ------------------------------------------------------------------
-    {
-      const uint32_t* cc = cptr(cur, rank);
-      uint32_t* cn = cptr(cur ^ 1, rank);
-      unsigned int run = 0;
-      for (int64_t base = 0; base < my_n; base += kThreads) {
-        const int64_t i = base + tid;
-        uint32_t km = 0u, cv = 0u;
-        if (i < my_n) {
-          cv = cc[i];
+    if (tid < G) {
+      S.kc[tid] = 0u;
+      S.tie_run[tid] = 0u;
+    }
+    __syncthreads();
+    bool any_tie = false;
 #pragma unroll
-          for (int h = 0; h < G; ++h) km |= ((kptr(h, rank)[i >> 5] >> (i & 31)) & 1u) << h;
+    for (int h = 0; h < G; ++h) any_tie |= S.st[h].mode == kModeTie;
+    {
+      uint32_t* cn = cptr(cur ^ 1);  // next level's candidates, or (list mode) keep masks
+      unsigned int run = 0;
+      constexpr int kEU = G >= 8 ? 1 : 2;  // consecutive candidates per thread
+      for (int64_t base = 0; base < my_n; base += kEU * kThreads) {
+        const int64_t i0 = base + kEU * tid;
+        uint32_t km[kEU], cv[kEU], ties[kEU];
+        float z[kEU][G];
+#pragma unroll
+        for (int u = 0; u < kEU; ++u) {
+          km[u] = ties[u] = 0u;
+          cv[u] = i0 + u < my_n ? cc[i0 + u] : 0u;
+          if (i0 + u < my_n) load_scores<G>(zown, i0 + u, z[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < kEU; ++u) {
+          const uint32_t hm = cv[u] >> 24;
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            if (!((hm >> h) & 1u)) continue;
+            bool member;
+            if (keep_rule(S.st[h].mode, S.st[h].kthr, order_key(z[u][h]), &member))
+              km[u] |= 1u << h;
+            if (member) ties[u] |= 1u << h;
+          }
+        }
+        if (any_tie) {  // exact ties: the segment keeps its first quota members in node order
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            if (S.st[h].mode != kModeTie) continue;
+            unsigned f = 0;
+#pragma unroll
+            for (int u = 0; u < kEU; ++u) f += (ties[u] >> h) & 1u;
+            unsigned int tot;
+            const unsigned int run_h = S.tie_run[h];
+            unsigned int rk = run_h + block_excl_scan(f, &tot, S);  // syncs: run_h read by all
+            const unsigned int quota = S.st[h].quota[rank];
+#pragma unroll
+            for (int u = 0; u < kEU; ++u)
+              if ((ties[u] >> h) & 1u) {
+                if (rk < quota) km[u] |= 1u << h;
+                ++rk;
+              }
+            if (tid == 0) S.tie_run[h] = run_h + tot;
+          }
+        }
+        unsigned int nk = 0;
+#pragma unroll
+        for (int u = 0; u < kEU; ++u) nk += km[u] ? 1u : 0u;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          unsigned int f = 0;
+#pragma unroll
+          for (int u = 0; u < kEU; ++u) f += (km[u] >> h) & 1u;
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) f += __shfl_xor_sync(0xffffffffu, f, off);
+          if (lane == 0 && f) atomicAdd(&S.kc[h], f);
         }
         unsigned int tot;
-        const unsigned int rk = block_excl_scan(km ? 1u : 0u, &tot, S);
-        if (km) {
-          const int64_t pos = (int64_t)run + rk;
-          const uint32_t node = cv & kNodeMask;
-          if (level > 1) {
-            for (int c = 0; c < b; ++c)
-              cn[pos * b + c] = (km << 24) | (node * (uint32_t)b + (uint32_t)c);
-          } else if (!p.list_mode) {
-            p.kept[((int64_t)unit * C + rank) * seg + pos] = (km << 24) | node;
+        int64_t pos = (int64_t)run + block_excl_scan(nk, &tot, S);
+#pragma unroll
+        for (int u = 0; u < kEU; ++u) {
+          if (km[u]) {
+            const uint32_t node = cv[u] & kNodeMask;
+            if (level > 1) {
+              for (int c = 0; c < b; ++c)
+                cn[pos * b + c] = (km[u] << 24) | (node * (uint32_t)b + (uint32_t)c);
+            } else if (!p.list_mode) {
+              p.kept[((int64_t)unit * C + rank) * seg + pos] = (km[u] << 24) | node;
+            }
+            ++pos;
           }
+          if (level == 1 && p.list_mode && i0 + u < my_n) cn[i0 + u] = km[u];  // for the emission
         }
         run += tot;
       }
       if (level == 1 && !p.list_mode && tid == 0)
         p.n_kept[(int64_t)unit * C + rank] = (int32_t)run;
+      // per-head kept counts of my segment (S.kc): the next level's head
+      // frontiers hold b children of each
+      __syncthreads();
+      if (tid < G) S.my_hcnt[tid] = S.kc[tid] * (unsigned int)b;
       my_n = (int64_t)run * b;
       if (level > 1 && my_n > seg) {  // cannot happen: a segment holds every level-1 node
-        raise_status(p.status, ZHA_ERR_WORKSPACE);
+        if (tid == 0) raise_status(p.status, ZHA_ERR_WORKSPACE);
         my_n = seg;
+      }
+    }
+
+    if (level == 1 && p.list_mode) {
+      // per-head ascending token lists: {0} (unless node 0 is kept) + tokens of
+      // the kept level-1 nodes in node order + causal tail
+      const uint32_t* km_seg = cptr(cur ^ 1);
+      const int64_t n1 = S.seg_n[rank];  // candidates of my segment at level 1
+      if (tid == 0)
+        S.node0 = (n1 > 0 && (cc[0] & kNodeMask) == 0u) ? km_seg[0] : 0u;
+      cluster.sync();  // every rank's kept counts published
+      unsigned int base[G], total[G];
+      uint32_t node0 = 0;
+#pragma unroll
+      for (int h = 0; h < G; ++h) base[h] = total[h] = 0u;
+      for (int r = 0; r < C; ++r) {
+        const Smem* R = cluster.map_shared_rank(&S, r);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const unsigned int v = R->kc[h];
+          if (r < rank) base[h] += v;
+          total[h] += v;
+        }
+        node0 |= R->node0;
+      }
+      const int64_t tail_start = p.span[p.L] * T_top;
+      const int64_t tail_len = n_vis - tail_start;
+#pragma unroll 1
+      for (int h = 0; h < G; ++h) {
+        const int64_t qh = (int64_t)qi * p.Hq + (int64_t)kvh * G + h;
+        int32_t* out = p.idx + qh * p.idx_cap;
+        const int64_t off0 = ((node0 >> h) & 1u) ? 0 : 1;
+        unsigned int prun = base[h];
+        for (int64_t b0 = 0; b0 < n1; b0 += kThreads) {
+          const int64_t i = b0 + tid;
+          const unsigned f = i < n1 ? (km_seg[i] >> h) & 1u : 0u;
+          unsigned int tot;
+          const unsigned int rk = block_excl_scan(f, &tot, S);
+          if (f) {
+            const int64_t pos = off0 + (int64_t)b * (prun + rk);
+            const int64_t node = cc[i] & kNodeMask;
+            for (int c = 0; c < b; ++c)
+              if (pos + c < p.idx_cap) out[pos + c] = (int32_t)(node * b + c);
+          }
+          prun += tot;
+        }
+        if (rank == 0 && tid == 0 && off0 == 1 && p.idx_cap > 0) out[0] = 0;
+        if (rank == C - 1) {
+          const int64_t tail_pos = off0 + (int64_t)b * total[h];
+          for (int64_t j = tid; j < tail_len; j += kThreads)
+            if (tail_pos + j < p.idx_cap) out[tail_pos + j] = (int32_t)(tail_start + j);
+          if (tid == 0) {
+            const int64_t n = tail_pos + tail_len;
+            p.n_idx[qh] = (int32_t)n;
+            if (n > p.idx_cap) raise_status(p.status, ZHA_ERR_CAPACITY);
+          }
+        }
       }
     }
     cur ^= 1;
     __syncthreads();
   }
-  // no DSMEM access follows the last cluster barrier, so CTAs may exit freely
+  // no CTA may leave while another can still read its shared memory
+  cluster.sync();
 }
 
 template <typename T, int D, int G>
@@ -1068,11 +1043,10 @@ int max_clusters_g(int G, int C) {
 }
 
 int max_clusters(const Geometry& g, int C) {
-  static int cache[2][2][4][5];  // dtype, d, G, log2 C (0 = not queried)
+  static int cache[2][2][4][kMaxCluster + 1];  // dtype, d, G, C (0 = not queried)
   const int i0 = g.dtype == ZHA_BF16, i1 = g.d == 128;
   const int i2 = g.G == 1 ? 0 : g.G == 2 ? 1 : g.G == 4 ? 2 : 3;
-  const int i3 = C == 1 ? 0 : C == 2 ? 1 : C == 4 ? 2 : C == 8 ? 3 : 4;
-  int& v = cache[i0][i1][i2][i3];
+  int& v = cache[i0][i1][i2][C];
   if (v == 0) {
     int n;
     if (g.dtype == ZHA_BF16)
@@ -1087,23 +1061,21 @@ int max_clusters(const Geometry& g, int C) {
 
 }  // namespace
 
-// The largest power-of-two cluster (<= 16 CTAs) that keeps every unit resident
-// in one wave and at most two CTAs per SM.
+// The largest cluster (<= 16 CTAs) that keeps every unit resident in one wave
+// with at most two CTAs per SM.
 int traverse_cluster_size(const Geometry& g, int64_t units, int num_sms) {
-  int best = 1;
-  for (int C = 2; C <= kMaxCluster; C *= 2) {
-    if (units * C > 2 * (int64_t)num_sms) break;
+  for (int C = kMaxCluster; C >= 2; --C) {
+    if (units * C > 2 * (int64_t)num_sms) continue;
     const int n = max_clusters(g, C);
-    if (n > 0 && n >= units) best = C;
+    if (n > 0 && n >= units) return C;
   }
-  return best;
+  return 1;
 }
 
 size_t traverse_ws_bytes(const Geometry& g, int64_t units, int num_sms) {
   const int C = traverse_cluster_size(g, units, num_sms);
   const size_t seg = (size_t)seg_capacity(g);
-  const size_t per = (size_t)C * seg * (2 * sizeof(uint32_t) + (size_t)g.G * sizeof(float)) +
-                     (size_t)g.G * C * (seg / 32) * sizeof(uint32_t);
+  const size_t per = (size_t)C * seg * (2 * sizeof(uint32_t) + (size_t)g.G * sizeof(float));
   return per * (size_t)units + 256;
 }
 
@@ -1150,8 +1122,6 @@ cudaError_t launch_traverse(const Geometry& g, const void* tree, const void* q,
   p.cand = reinterpret_cast<uint32_t*>(w);
   w += sizeof(uint32_t) * (size_t)units * 2 * C * p.seg;
   p.zbuf = reinterpret_cast<float*>(w);
-  w += sizeof(float) * (size_t)units * g.G * C * p.seg;
-  p.kbits = reinterpret_cast<uint32_t*>(w);
   if (!list_mode) {
     if (!out.kept || !out.n_kept) return cudaErrorInvalidValue;
     p.kept = out.kept;
