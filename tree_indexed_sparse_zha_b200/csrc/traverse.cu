@@ -58,14 +58,17 @@ constexpr int kDigit = 8;                 // key bits resolved per radix pass
 constexpr int kBuckets = 1 << kDigit;     // == kThreads: one bucket per thread
 constexpr int kCandPerThread = 4;
 constexpr uint32_t kNodeMask = 0x00ffffffu;
+constexpr int kGather = 512;  // groups this small are finished by the head's owner alone
 static_assert(kBuckets == kThreads, "one histogram bucket per thread");
 
 enum HeadMode : int {
-  kModeRadix = 0,  // group being narrowed by key digits
-  kModeAll = 1,    // keep every candidate of the head
-  kModeThr = 2,    // keep iff key >= kthr
-  kModeTie = 3,    // keep iff key > kthr, or key == kthr within the segment's quota
-  kModeQuant = 4,  // first pass pending: buckets are a linear map of z
+  kModeRadix = 0,     // group being narrowed by key digits
+  kModeAll = 1,       // keep every candidate of the head
+  kModeThr = 2,       // keep iff key >= kthr
+  kModeTie = 3,       // keep iff key > kthr, or key == kthr within the segment's quota
+  kModeQuant = 4,     // first pass pending: buckets are a linear map of z
+  kModeGathered = 5,  // keep iff first-pass bucket > qbeta, or == qbeta and the
+                      // owner marked the candidate kept
 };
 
 struct TravParams {
@@ -87,6 +90,8 @@ struct TravParams {
   int64_t seg;           // capacity of one segment (candidates), multiple of 32
   uint32_t* cand;        // [units][2][C][seg]   (head mask << 24) | node
   float* zbuf;           // [units][C][seg][G]   scores, candidate-major
+  uint8_t* qbuf;         // [units][C][seg][G]   first-pass bucket of each score
+  uint8_t* mkbuf;        // [units][C][seg][G]   kModeGathered: owner's keep mark
   uint32_t* kept;        // [units][C][seg]     decode mode: union-kept level-1 nodes
   int32_t* n_kept;       // [units][C]
   int32_t* idx;          // [nq][Hq][idx_cap]   list mode
@@ -113,6 +118,9 @@ struct HeadState {
   int mode;                  // HeadMode
   unsigned int kthr;         // threshold key of the final rule
   unsigned int count;        // kept candidates (the level count)
+  unsigned int qbeta;        // first-pass bucket of the group (0xffffffff: none)
+  int zfree;                 // kModeThr / kModeTie decided on the first pass: every
+                             // candidate's fate follows from its bucket alone
   unsigned int quota[kMaxCluster];  // kModeTie: kept members of each segment
 };
 
@@ -150,6 +158,13 @@ struct Smem {
   unsigned int nh[kMaxGroup];                    // candidates of head h at this level
   unsigned int tie_cnt[kMaxCluster];             // crossing-bucket members per rank
   unsigned int my_hcnt[kMaxGroup];               // my segment's candidates in head h's frontier
+  // groups of at most kGather members are shipped to the head's owner: one
+  // list per owned head (slot h / C), filled by every rank through DSMEM
+  alignas(16) float mz[kMaxGroup * kGather];
+  alignas(16) uint32_t mpos[kMaxGroup * kGather];  // (rank << 24) | segment index
+  unsigned int mlist_n[kMaxGroup];
+  alignas(16) unsigned long long mrank_m[kGather];   // member sort keys
+  unsigned long long red_scan[kWarps];
 };
 
 // Exclusive scan of v over the CTA in thread order; *total receives the sum.
@@ -230,6 +245,41 @@ __device__ __forceinline__ void load_scores(const float* zown, int64_t i, float*
   } else {
     z[0] = zown[i];
   }
+}
+
+// The G first-pass bucket bytes of candidate i, packed (byte h = head h).
+template <int G>
+__device__ __forceinline__ uint64_t load_qrow(const uint8_t* q, int64_t i) {
+  if constexpr (G == 8) return __ldcg(reinterpret_cast<const unsigned long long*>(q) + i);
+  else if constexpr (G == 4) return __ldcg(reinterpret_cast<const unsigned int*>(q) + i);
+  else if constexpr (G == 2) return __ldcg(reinterpret_cast<const unsigned short*>(q) + i);
+  else return __ldcg(q + i);
+}
+template <int G>
+__device__ __forceinline__ void store_qrow(uint8_t* q, int64_t i, uint64_t v) {
+  if constexpr (G == 8) reinterpret_cast<unsigned long long*>(q)[i] = v;
+  else if constexpr (G == 4) reinterpret_cast<unsigned int*>(q)[i] = (unsigned int)v;
+  else if constexpr (G == 2) reinterpret_cast<unsigned short*>(q)[i] = (unsigned short)v;
+  else q[i] = (uint8_t)v;
+}
+
+// Bit h set where byte h of a is greater than / equal to byte h of b, or
+// where byte h of a is nonzero (SIMD byte compares, then the top bit of each
+// 0x00/0xff byte gathered into one byte by a multiply).
+__device__ __forceinline__ uint32_t gather_bits(uint64_t m) {
+  return (uint32_t)(((m & 0x8080808080808080ull) * 0x0002040810204081ull) >> 56);
+}
+__device__ __forceinline__ uint32_t bytes_gt(uint64_t a, uint64_t b) {
+  return gather_bits(((uint64_t)__vcmpgtu4((unsigned)(a >> 32), (unsigned)(b >> 32)) << 32) |
+                     __vcmpgtu4((unsigned)a, (unsigned)b));
+}
+__device__ __forceinline__ uint32_t bytes_eq(uint64_t a, uint64_t b) {
+  return gather_bits(((uint64_t)__vcmpeq4((unsigned)(a >> 32), (unsigned)(b >> 32)) << 32) |
+                     __vcmpeq4((unsigned)a, (unsigned)b));
+}
+__device__ __forceinline__ uint32_t bytes_nz(uint64_t a) {
+  return gather_bits(((uint64_t)__vcmpne4((unsigned)(a >> 32), 0u) << 32) |
+                     __vcmpne4((unsigned)a, 0u));
 }
 
 // First-pass bucket of score z: a linear map of [zlo, zlo + 256 / zscale)
@@ -485,7 +535,9 @@ __device__ __noinline__ void owner_pass(const TravParams& p, Smem& S, cg::cluste
   // digit's sub-interval of the previous group on later passes
   uint32_t gmin = 0, gmax = 0;
   if (ok) {
-    if (quant) {
+    if (quant && s0.zscale == 0.0f) {  // every score equals zlo
+      gmin = gmax = order_key(s0.zlo);
+    } else if (quant) {
       if (tid == 0) quant_interval(s0.zlo, s0.zscale, beta, &S.found[3], &S.found[4]);
       __syncthreads();
       gmin = S.found[3];
@@ -520,6 +572,8 @@ __device__ __noinline__ void owner_pass(const TravParams& p, Smem& S, cg::cluste
       ns.bcnt = bcnt;
       ns.kgmin = gmin;
       ns.kgmax = gmax;
+      if (quant) ns.qbeta = beta;
+      ns.zfree = quant ? 1 : 0;  // a final rule set now needs no scores in the expand
       ns.mode = kModeRadix;
       if (bcnt == 1u) {
         ns.mode = kModeThr;  // the group's only member is the last kept candidate;
@@ -547,6 +601,86 @@ __device__ __noinline__ void owner_pass(const TravParams& p, Smem& S, cg::cluste
         }
       }
     }
+    S.pub[h] = ns;
+  }
+  __syncthreads();
+}
+
+// Owner step for a head whose group (at most kGather members) has been
+// shipped to this CTA's list S.mz/S.mpos[slot]: sorts the members by
+// (z desc, position asc) (bitonic network on (key << 32 | ~position)), finds
+// the shortest prefix whose mass reaches what the group must still cover,
+// marks every member's fate in mkbuf (the keep byte of (segment, index, head))
+// and publishes kModeGathered in S.pub[h].
+template <int G>
+__device__ __noinline__ void owner_finish(const TravParams& p, Smem& S, int h, int slot,
+                                          uint8_t* mk_u, int64_t seg) {
+  static_assert(kGather == 2 * kThreads, "two sort slots per thread");
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const HeadState s0 = S.st[h];
+  const int n = (int)(S.mlist_n[slot] < (unsigned)kGather ? S.mlist_n[slot] : kGather);
+  int np2 = 2;
+  while (np2 < n) np2 <<= 1;
+  unsigned long long* key = S.mrank_m;  // sort keys, descending
+  for (int i = tid; i < np2; i += kThreads)
+    key[i] = i < n ? ((unsigned long long)order_key(S.mz[slot * kGather + i]) << 32) |
+                         (0xffffffffu - S.mpos[slot * kGather + i])
+                   : 0ull;
+  __syncthreads();
+  for (int k = 2; k <= np2; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = tid; i < np2; i += kThreads) {
+        const int l = i ^ j;
+        if (l > i) {
+          const unsigned long long a = key[i], b = key[l];
+          const bool desc = (i & k) == 0;
+          if (desc ? a < b : a > b) {
+            key[i] = b;
+            key[l] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // masses in rank order; thread t owns ranks 2t and 2t + 1
+  const float zmax = S.zmax[h];
+  const int r0 = 2 * tid;
+  const unsigned long long m0 =
+      r0 < n ? mass_fixed(key_float((uint32_t)(key[r0] >> 32)), zmax) : 0ull;
+  const unsigned long long m1 =
+      r0 + 1 < n ? mass_fixed(key_float((uint32_t)(key[r0 + 1] >> 32)), zmax) : 0ull;
+  unsigned long long x = m0 + m1;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const unsigned long long y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) S.red_scan[warp] = x;
+  if (tid == 0) S.found[5] = 0xffffffffu;
+  __syncthreads();
+  unsigned long long run = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w)
+    if (w < warp) run += S.red_scan[w];
+  run += x - (m0 + m1);  // mass of ranks < r0
+  const unsigned long long rem = s0.need - s0.above;  // > 0: the group holds the crossing
+  if (r0 < n && run < rem && run + m0 >= rem) S.found[5] = (unsigned)r0;
+  if (r0 + 1 < n && run + m0 < rem && run + m0 + m1 >= rem) S.found[5] = (unsigned)r0 + 1u;
+  __syncthreads();
+  unsigned int k = S.found[5];
+  const bool ok = k != 0xffffffffu && n == (int)s0.bcnt;
+  if (!ok) k = (unsigned)n - 1u;  // cannot happen with exact sums: keep the whole group
+  for (int r = tid; r < n; r += kThreads) {
+    const uint32_t pi = 0xffffffffu - (uint32_t)key[r];
+    const int64_t rr = pi >> 24, idx = pi & kNodeMask;
+    mk_u[(rr * seg + idx) * G + h] = (unsigned)r <= k ? 1 : 0;
+  }
+  if (tid == 0) {
+    if (!ok) raise_status(p.status, ZHA_ERR_INTERNAL);
+    HeadState ns = s0;
+    ns.mode = kModeGathered;
+    ns.count = s0.cabove + k + 1u;
     S.pub[h] = ns;
   }
   __syncthreads();
@@ -609,6 +743,9 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
 
   uint32_t* cand_u = p.cand + (int64_t)unit * 2 * C * seg;
   float* zown = p.zbuf + ((int64_t)unit * C + rank) * seg * G;  // [seg][G]
+  uint8_t* qown = p.qbuf + ((int64_t)unit * C + rank) * seg * G;  // [seg][G]
+  uint8_t* mk_u = p.mkbuf + (int64_t)unit * C * seg * G;           // [C][seg][G]
+  const uint8_t* mkown = mk_u + (int64_t)rank * seg * G;
   auto cptr = [&](int buf) { return cand_u + ((int64_t)buf * C + rank) * seg; };
   int32_t* lc_base = p.level_counts ? p.level_counts + ((int64_t)qi * p.Hq + (int64_t)kvh * G) * p.L
                                     : nullptr;
@@ -723,66 +860,137 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
         s.zlo = lo;
         s.zscale = mx > lo ? __fdiv_rn(256.0f, __fsub_rn(mx, lo)) : 0.0f;
       }
+      s.qbeta = 0xffffffffu;
       S.st[tid] = s;
+      S.mlist_n[tid] = 0u;  // my gather lists (slots of the heads I own)
     }
     __syncthreads();
     for (int pass = 0; pass < 40; ++pass) {  // every pass strictly narrows each group
-      unsigned cut_heads = 0;
+      // heads whose group is still open: histogram pass, or (small group)
+      // shipped to the owner who finishes the cut alone
+      unsigned hist_heads = 0, gather_heads = 0;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const int m = S.st[h].mode;
-        cut_heads |= (m == kModeRadix || m == kModeQuant ? 1u : 0u) << h;
+        if (m == kModeQuant) hist_heads |= 1u << h;
+        else if (m == kModeRadix)
+          (S.st[h].bcnt <= (unsigned)kGather ? gather_heads : hist_heads) |= 1u << h;
       }
-      if (!cut_heads) break;  // uniform: every CTA holds the same states
-      for (int e = tid; e < G * kBuckets; e += kThreads) {
-        (&S.hist_lo[0][0])[e] = 0u;
-        (&S.hist_hi[0][0])[e] = 0u;
-        (&S.hist_c[0][0])[e] = 0u;
-      }
+      const unsigned open_heads = hist_heads | gather_heads;
+      if (!open_heads) break;  // uniform: every CTA holds the same states
+      const bool first = pass == 0;  // every open head is in kModeQuant
+      if (hist_heads)
+        for (int e = tid; e < G * kBuckets; e += kThreads) {
+          (&S.hist_lo[0][0])[e] = 0u;
+          (&S.hist_hi[0][0])[e] = 0u;
+          (&S.hist_c[0][0])[e] = 0u;
+        }
       __syncthreads();
-      // local histograms of my segment for every head still being cut; kHU
-      // consecutive candidates per thread, loaded up front
-      constexpr int kHU = G >= 8 ? 2 : 4;
-      for (int64_t base = 0; base < my_n; base += kHU * kThreads) {
-        const int64_t i0 = base + kHU * tid;
-        uint32_t hm[kHU];
-        float z[kHU][G];
-#pragma unroll
-        for (int u = 0; u < kHU; ++u) hm[u] = i0 + u < my_n ? (cc[i0 + u] >> 24) & cut_heads : 0u;
-#pragma unroll
-        for (int u = 0; u < kHU; ++u)
-          if (i0 + u < my_n) load_scores<G>(zown, i0 + u, z[u]);
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          if (!((cut_heads >> h) & 1u)) continue;
-          const HeadState& s = S.st[h];
-          const bool quant = s.mode == kModeQuant;
-          int sh = 0, w = 0;
-          if (!quant) radix_digit(s.kgmin, s.kgmax, &sh, &w);
+      // consecutive candidates per thread, loaded up front (fewer with 8 heads
+      // to stay within the register budget)
+      if (first) {
+        constexpr int kHU = G >= 8 ? 1 : 4;
+        // every open head is in kModeQuant: bucket every score, histogram it,
+        // and keep the bucket bytes for the later passes and the expand
+        for (int64_t base = 0; base < my_n; base += kHU * kThreads) {
+          const int64_t i0 = base + kHU * tid;
+          uint32_t hm[kHU];
+          uint64_t qrow[kHU];
+          float z[kHU][G];
 #pragma unroll
           for (int u = 0; u < kHU; ++u) {
-            if (!((hm[u] >> h) & 1u)) continue;
-            const uint32_t key = order_key(z[u][h]);
-            uint32_t d;
-            if (quant) {
-              d = quant_bucket(z[u][h], s.zlo, s.zscale);
-            } else {
-              if (key < s.kgmin || key > s.kgmax) continue;
-              d = (key >> sh) & ((1u << w) - 1u);
+            const bool in = i0 + u < my_n;
+            hm[u] = in ? (cc[i0 + u] >> 24) & open_heads : 0u;
+            qrow[u] = 0;
+            if (in) load_scores<G>(zown, i0 + u, z[u]);
+          }
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            if (!((open_heads >> h) & 1u)) continue;
+            const float zlo = S.st[h].zlo, zscale = S.st[h].zscale, zmx = S.zmax[h];
+#pragma unroll
+            for (int u = 0; u < kHU; ++u) {
+              if (!((hm[u] >> h) & 1u)) continue;
+              const uint32_t d = quant_bucket(z[u][h], zlo, zscale);
+              qrow[u] |= (uint64_t)d << (8 * h);
+              hist_add(S, h, d, mass_fixed(z[u][h], zmx));
             }
-            hist_add(S, h, d, mass_fixed(z[u][h], S.zmax[h]));
+          }
+#pragma unroll
+          for (int u = 0; u < kHU; ++u)
+            if (i0 + u < my_n) store_qrow<G>(qown, i0 + u, qrow[u]);
+        }
+      } else {
+        // later passes touch only the members of the open groups: candidates
+        // whose first-pass bucket is the group's, and whose key lies in the
+        // group's interval
+        constexpr int kHU = G >= 8 ? 2 : 4;
+        uint64_t qb_pack = 0;
+#pragma unroll
+        for (int h = 0; h < G; ++h) qb_pack |= (uint64_t)(S.st[h].qbeta & 0xffu) << (8 * h);
+        for (int64_t base = 0; base < my_n; base += kHU * kThreads) {
+          const int64_t i0 = base + kHU * tid;
+          uint32_t mem[kHU];
+          float z[kHU][G];
+#pragma unroll
+          for (int u = 0; u < kHU; ++u) {
+            const bool in = i0 + u < my_n;
+            const uint32_t hm = in ? (cc[i0 + u] >> 24) & open_heads : 0u;
+            mem[u] = hm ? hm & bytes_eq(load_qrow<G>(qown, i0 + u), qb_pack) : 0u;
+            if (mem[u]) load_scores<G>(zown, i0 + u, z[u]);
+          }
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            if (!((open_heads >> h) & 1u)) continue;
+            const HeadState& st = S.st[h];
+            const bool gather = (gather_heads >> h) & 1u;
+            int sh = 0, w = 0;
+            radix_digit(st.kgmin, st.kgmax, &sh, &w);
+#pragma unroll
+            for (int u = 0; u < kHU; ++u) {
+              bool v = (mem[u] >> h) & 1u;
+              uint32_t key = 0;
+              if (v) {
+                key = order_key(z[u][h]);
+                v = key >= st.kgmin && key <= st.kgmax;
+              }
+              if (gather) {  // one slot reservation per warp and head
+                const unsigned mb = __ballot_sync(0xffffffffu, v);
+                if (mb) {
+                  const int slot = h / C;
+                  const int leader = __ffs(mb) - 1;
+                  unsigned first_slot = 0;
+                  if (lane == leader)
+                    first_slot = atomicAdd(&cluster.map_shared_rank(&S, h % C)->mlist_n[slot],
+                                           (unsigned)__popc(mb));
+                  first_slot = __shfl_sync(0xffffffffu, first_slot, leader);
+                  if (v) {
+                    const unsigned k = first_slot + __popc(mb & ((1u << lane) - 1u));
+                    if (k < (unsigned)kGather) {
+                      Smem* O = cluster.map_shared_rank(&S, h % C);
+                      O->mz[slot * kGather + k] = z[u][h];
+                      O->mpos[slot * kGather + k] = ((uint32_t)rank << 24) | (uint32_t)(i0 + u);
+                    }
+                  }
+                }
+              } else if (v) {
+                hist_add(S, h, (key >> sh) & ((1u << w) - 1u), mass_fixed(z[u][h], S.zmax[h]));
+              }
+            }
           }
         }
       }
-      cluster.sync();  // every rank's histograms complete
-      for (int h = rank; h < G; h += C)
-        if ((cut_heads >> h) & 1u) owner_pass<G>(p, S, cluster, C, h);
+      cluster.sync();  // every rank's histograms and shipped members complete
+      for (int h = rank; h < G; h += C) {
+        if ((hist_heads >> h) & 1u) owner_pass<G>(p, S, cluster, C, h);
+        else if ((gather_heads >> h) & 1u) owner_finish<G>(p, S, h, h / C, mk_u, seg);
+      }
       cluster.sync();  // every owner published
-      {  // copy the narrowed states of the heads being cut from their owners
+      {  // copy the new states of the open heads from their owners
         constexpr int kWords = (int)(sizeof(HeadState) / 4);
         for (int e = tid; e < G * kWords; e += kThreads) {
           const int h = e / kWords, k = e % kWords;
-          if (!((cut_heads >> h) & 1u)) continue;
+          if (!((open_heads >> h) & 1u)) continue;
           const Smem* R = cluster.map_shared_rank(&S, h % C);
           reinterpret_cast<unsigned int*>(&S.st[h])[k] =
               reinterpret_cast<const unsigned int*>(&R->pub[h])[k];
@@ -809,33 +1017,65 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
       S.tie_run[tid] = 0u;
     }
     __syncthreads();
+    // the rules as byte-parallel masks (bit h = head h)
+    uint32_t allm = 0, gathm = 0, thrz = 0, tiez = 0, needz = 0;
+    uint64_t qb_pack = 0;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const HeadState& st = S.st[h];
+      const uint32_t bit = 1u << h;
+      if (st.mode == kModeAll) allm |= bit;
+      else if (st.mode == kModeGathered) gathm |= bit;
+      else if (st.mode == kModeThr) (st.zfree ? thrz : needz) |= bit;
+      else if (st.mode == kModeTie) (st.zfree ? tiez : needz) |= bit;
+      qb_pack |= (uint64_t)(st.qbeta & 0xffu) << (8 * h);
+    }
     bool any_tie = false;
 #pragma unroll
     for (int h = 0; h < G; ++h) any_tie |= S.st[h].mode == kModeTie;
     {
       uint32_t* cn = cptr(cur ^ 1);  // next level's candidates, or (list mode) keep masks
       unsigned int run = 0;
-      constexpr int kEU = G >= 8 ? 1 : 2;  // consecutive candidates per thread
+      constexpr int kEU = 4;  // consecutive candidates per thread
       for (int64_t base = 0; base < my_n; base += kEU * kThreads) {
         const int64_t i0 = base + kEU * tid;
         uint32_t km[kEU], cv[kEU], ties[kEU];
-        float z[kEU][G];
+        uint64_t qrow[kEU], mrow[kEU];
 #pragma unroll
         for (int u = 0; u < kEU; ++u) {
           km[u] = ties[u] = 0u;
-          cv[u] = i0 + u < my_n ? cc[i0 + u] : 0u;
-          if (i0 + u < my_n) load_scores<G>(zown, i0 + u, z[u]);
+          const bool in = i0 + u < my_n;
+          cv[u] = in ? cc[i0 + u] : 0u;
+          qrow[u] = in ? load_qrow<G>(qown, i0 + u) : 0ull;
+          mrow[u] = in ? load_qrow<G>(mkown, i0 + u) : 0ull;
         }
+        // the fate of a candidate follows from its first-pass bucket: above the
+        // group's bucket it is kept, below it dropped; members of the bucket
+        // carry the owner's mark (kModeGathered), are all kept (kModeThr set on
+        // the first pass) or are exact ties ranked in node order (kModeTie)
 #pragma unroll
         for (int u = 0; u < kEU; ++u) {
           const uint32_t hm = cv[u] >> 24;
+          const uint32_t gt = bytes_gt(qrow[u], qb_pack), eq = bytes_eq(qrow[u], qb_pack);
+          km[u] = hm & (allm | (gt & ~allm) | (eq & gathm & bytes_nz(mrow[u])) | (eq & thrz));
+          ties[u] = hm & eq & tiez;
+        }
+        if (needz) {  // rules narrowed below the first-pass bucket: compare scores
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
-            if (!((hm >> h) & 1u)) continue;
-            bool member;
-            if (keep_rule(S.st[h].mode, S.st[h].kthr, order_key(z[u][h]), &member))
-              km[u] |= 1u << h;
-            if (member) ties[u] |= 1u << h;
+          for (int u = 0; u < kEU; ++u) {
+            if (i0 + u >= my_n) continue;
+            float z[G];
+            load_scores<G>(zown, i0 + u, z);
+            const uint32_t hm = cv[u] >> 24;
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              const HeadState& st = S.st[h];
+              if (!(((hm & needz) >> h) & 1u)) continue;
+              if ((uint32_t)((qrow[u] >> (8 * h)) & 0xffu) != st.qbeta) continue;
+              bool member;
+              if (keep_rule(st.mode, st.kthr, order_key(z[h]), &member)) km[u] |= 1u << h;
+              if (member) ties[u] |= 1u << h;
+            }
           }
         }
         if (any_tie) {  // exact ties: the segment keeps its first quota members in node order
@@ -1075,7 +1315,8 @@ int traverse_cluster_size(const Geometry& g, int64_t units, int num_sms) {
 size_t traverse_ws_bytes(const Geometry& g, int64_t units, int num_sms) {
   const int C = traverse_cluster_size(g, units, num_sms);
   const size_t seg = (size_t)seg_capacity(g);
-  const size_t per = (size_t)C * seg * (2 * sizeof(uint32_t) + (size_t)g.G * sizeof(float));
+  // candidates (two buffers), scores, first-pass buckets and owner marks
+  const size_t per = (size_t)C * seg * (2 * sizeof(uint32_t) + (size_t)g.G * (sizeof(float) + 2));
   return per * (size_t)units + 256;
 }
 
@@ -1122,6 +1363,10 @@ cudaError_t launch_traverse(const Geometry& g, const void* tree, const void* q,
   p.cand = reinterpret_cast<uint32_t*>(w);
   w += sizeof(uint32_t) * (size_t)units * 2 * C * p.seg;
   p.zbuf = reinterpret_cast<float*>(w);
+  w += sizeof(float) * (size_t)units * C * p.seg * g.G;
+  p.qbuf = reinterpret_cast<uint8_t*>(w);
+  w += (size_t)units * C * p.seg * g.G;
+  p.mkbuf = reinterpret_cast<uint8_t*>(w);
   if (!list_mode) {
     if (!out.kept || !out.n_kept) return cudaErrorInvalidValue;
     p.kept = out.kept;
