@@ -158,14 +158,26 @@ struct Smem {
   unsigned int nh[kMaxGroup];                    // candidates of head h at this level
   unsigned int tie_cnt[kMaxCluster];             // crossing-bucket members per rank
   unsigned int my_hcnt[kMaxGroup];               // my segment's candidates in head h's frontier
+  // score_segment: each thread's next summary-row chunks in flight (cp.async)
+  alignas(16) uint4 ring[3][kCandPerThread][kThreads];
   // groups of at most kGather members are shipped to the head's owner: one
-  // list per owned head (slot h / C), filled by every rank through DSMEM
-  alignas(16) float mz[kMaxGroup * kGather];
-  alignas(16) uint32_t mpos[kMaxGroup * kGather];  // (rank << 24) | segment index
+  // list per owned head (slot h / C), filled by every rank through DSMEM;
+  // the lists follow the struct in dynamic shared memory (list_z, list_pos)
   unsigned int mlist_n[kMaxGroup];
   alignas(16) unsigned long long mrank_m[kGather];   // member sort keys
   unsigned long long red_scan[kWarps];
 };
+
+// Shipped-member lists after the struct: z[slots][kGather], then
+// position[slots][kGather] with position = (rank << 24) | segment index.
+__device__ __forceinline__ float* list_z(Smem& S) {
+  return reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(&S) + sizeof(Smem));
+}
+__device__ __forceinline__ uint32_t* list_pos(Smem& S, int slots) {
+  return reinterpret_cast<uint32_t*>(list_z(S) + slots * kGather);
+}
+// owned heads per CTA (lists needed)
+__host__ __device__ __forceinline__ int list_slots(int G, int C) { return (G + C - 1) / C; }
 
 // Exclusive scan of v over the CTA in thread order; *total receives the sum.
 __device__ __forceinline__ unsigned int block_excl_scan(unsigned int v, unsigned int* total,
@@ -201,24 +213,12 @@ __device__ __forceinline__ unsigned long long ceil_mul_shift32(unsigned long lon
   return r;
 }
 
-// L2 eviction policies: summary rows stream through L2 once (evict first);
-// the per-candidate scores are re-read by every pass of the cut (evict last).
-__device__ __forceinline__ uint64_t policy_evict_first() {
-  uint64_t pol;
-  asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-  return pol;
-}
+// L2 eviction policy of the per-candidate scores, which every pass of the cut
+// re-reads (evict last).
 __device__ __forceinline__ uint64_t policy_evict_last() {
   uint64_t pol;
   asm("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
   return pol;
-}
-__device__ __forceinline__ uint4 ld_policy(const uint4* ptr, uint64_t pol) {
-  uint4 v;
-  asm("ld.global.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
-      : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-      : "l"(ptr), "l"(pol));
-  return v;
 }
 __device__ __forceinline__ void st_policy(float4* ptr, float4 v, uint64_t pol) {
   asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(ptr), "f"(v.x),
@@ -303,7 +303,7 @@ __device__ __forceinline__ void score_segment(const TravParams& p, Smem& S, cons
   constexpr int kPer = Elem<T>::kPerChunk;
   constexpr int kNch = D * (int)sizeof(T) / 16;
   const int tid = threadIdx.x;
-  const uint64_t pol_rows = policy_evict_first(), pol_z = policy_evict_last();
+  const uint64_t pol_z = policy_evict_last();
   for (int64_t base = 0; base < n; base += kThreads * kCandPerThread) {
     const uint4* rows[kCandPerThread];
     uint32_t pm[kCandPerThread];
@@ -326,19 +326,28 @@ __device__ __forceinline__ void score_segment(const TravParams& p, Smem& S, cons
 #pragma unroll
       for (int j = 0; j < (G + 1) / 2; ++j) acc[k][j] = make_float2(0.0f, 0.0f);
     }
-    uint4 cur[kCandPerThread], nxt[kCandPerThread];
+    // each thread streams its rows' 16-byte chunks through its own slots of a
+    // 3-stage shared-memory ring: two chunks in flight while one is used
+    uint4 cur[kCandPerThread];
 #pragma unroll
-    for (int k = 0; k < kCandPerThread; ++k) {
-      cur[k] = ok[k] ? ld_policy(rows[k], pol_rows) : make_uint4(0, 0, 0, 0);
-      nxt[k] = cur[k];
+    for (int st = 0; st < 2; ++st) {
+#pragma unroll
+      for (int k = 0; k < kCandPerThread; ++k)
+        if (ok[k] && st < kNch) cp_async16(&S.ring[st][k][tid], rows[k] + st);
+      cp_async_commit();
     }
 #pragma unroll 1
     for (int ch = 0; ch < kNch; ++ch) {
-      if (ch + 1 < kNch) {
+      if (ch + 2 < kNch) {
 #pragma unroll
         for (int k = 0; k < kCandPerThread; ++k)
-          nxt[k] = ok[k] ? ld_policy(rows[k] + ch + 1, pol_rows) : make_uint4(0, 0, 0, 0);
+          if (ok[k]) cp_async16(&S.ring[(ch + 2) % 3][k][tid], rows[k] + ch + 2);
       }
+      cp_async_commit();
+      cp_async_wait<2>();  // this thread's copies of chunk ch have landed
+#pragma unroll
+      for (int k = 0; k < kCandPerThread; ++k)
+        cur[k] = ok[k] ? S.ring[ch % 3][k][tid] : make_uint4(0, 0, 0, 0);
       float x[kCandPerThread][kPer];
 #pragma unroll
       for (int k = 0; k < kCandPerThread; ++k) Elem<T>::unpack(cur[k], x[k]);
@@ -368,8 +377,6 @@ __device__ __forceinline__ void score_segment(const TravParams& p, Smem& S, cons
           }
         }
       }
-#pragma unroll
-      for (int k = 0; k < kCandPerThread; ++k) cur[k] = nxt[k];
     }
 #pragma unroll
     for (int k = 0; k < kCandPerThread; ++k) {
@@ -408,6 +415,25 @@ __device__ __forceinline__ void hist_add(Smem& S, int h, uint32_t d, unsigned lo
   const unsigned hi = (unsigned)(m >> 32) + ((old + lo < old) ? 1u : 0u);
   if (hi) atomicAdd(&S.hist_hi[h][d], hi);
   atomicAdd(&S.hist_c[h][d], 1u);
+}
+
+// hist_add for all G heads of one candidate at once, without branches: head
+// h adds (m[h], c[h]) to bucket d[h] (c[h] = 0 and m[h] = 0 for a head that
+// does not count this candidate). The G low-word atomics are issued back to
+// back before any carry is resolved.
+template <int G>
+__device__ __forceinline__ void hist_add_heads(Smem& S, const uint32_t* d,
+                                               const unsigned long long* m, const uint32_t* c) {
+  unsigned old[G];
+#pragma unroll
+  for (int h = 0; h < G; ++h) old[h] = atomicAdd(&S.hist_lo[h][d[h]], (unsigned)m[h]);
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    const unsigned lo = (unsigned)m[h];
+    const unsigned hi = (unsigned)(m[h] >> 32) + ((old[h] + lo < old[h]) ? 1u : 0u);
+    if (hi) atomicAdd(&S.hist_hi[h][d[h]], hi);
+    if (c[h]) atomicAdd(&S.hist_c[h][d[h]], c[h]);
+  }
 }
 
 // Inverse of order_key.
@@ -614,7 +640,7 @@ __device__ __noinline__ void owner_pass(const TravParams& p, Smem& S, cg::cluste
 // and publishes kModeGathered in S.pub[h].
 template <int G>
 __device__ __noinline__ void owner_finish(const TravParams& p, Smem& S, int h, int slot,
-                                          uint8_t* mk_u, int64_t seg) {
+                                          int slots, uint8_t* mk_u, int64_t seg) {
   static_assert(kGather == 2 * kThreads, "two sort slots per thread");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const HeadState s0 = S.st[h];
@@ -623,8 +649,8 @@ __device__ __noinline__ void owner_finish(const TravParams& p, Smem& S, int h, i
   while (np2 < n) np2 <<= 1;
   unsigned long long* key = S.mrank_m;  // sort keys, descending
   for (int i = tid; i < np2; i += kThreads)
-    key[i] = i < n ? ((unsigned long long)order_key(S.mz[slot * kGather + i]) << 32) |
-                         (0xffffffffu - S.mpos[slot * kGather + i])
+    key[i] = i < n ? ((unsigned long long)order_key(list_z(S)[slot * kGather + i]) << 32) |
+                         (0xffffffffu - list_pos(S, slots)[slot * kGather + i])
                    : 0ull;
   __syncthreads();
   for (int k = 2; k <= np2; k <<= 1) {
@@ -892,29 +918,47 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
         constexpr int kHU = G >= 8 ? 1 : 4;
         // every open head is in kModeQuant: bucket every score, histogram it,
         // and keep the bucket bytes for the later passes and the expand
-        for (int64_t base = 0; base < my_n; base += kHU * kThreads) {
-          const int64_t i0 = base + kHU * tid;
-          uint32_t hm[kHU];
-          uint64_t qrow[kHU];
-          float z[kHU][G];
+        // software-pipelined: the next candidates' scores are in flight while
+        // the current ones are bucketed
+        uint32_t hm[kHU];
+        float z[kHU][G];
+        auto fetch = [&](int64_t i0, uint32_t* hmo, float (*zo)[G]) {
 #pragma unroll
           for (int u = 0; u < kHU; ++u) {
             const bool in = i0 + u < my_n;
-            hm[u] = in ? (cc[i0 + u] >> 24) & open_heads : 0u;
-            qrow[u] = 0;
-            if (in) load_scores<G>(zown, i0 + u, z[u]);
+            hmo[u] = in ? (cc[i0 + u] >> 24) & open_heads : 0u;
+            if (in) load_scores<G>(zown, i0 + u, zo[u]);
           }
+        };
+        fetch(kHU * tid, hm, z);
+        for (int64_t base = 0; base < my_n; base += kHU * kThreads) {
+          const int64_t i0 = base + kHU * tid;
+          uint32_t hm_c[kHU];
+          float z_c[kHU][G];
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
-            if (!((open_heads >> h) & 1u)) continue;
-            const float zlo = S.st[h].zlo, zscale = S.st[h].zscale, zmx = S.zmax[h];
+          for (int u = 0; u < kHU; ++u) {
+            hm_c[u] = hm[u];
 #pragma unroll
-            for (int u = 0; u < kHU; ++u) {
-              if (!((hm[u] >> h) & 1u)) continue;
-              const uint32_t d = quant_bucket(z[u][h], zlo, zscale);
-              qrow[u] |= (uint64_t)d << (8 * h);
-              hist_add(S, h, d, mass_fixed(z[u][h], zmx));
+            for (int h = 0; h < G; ++h) z_c[u][h] = z[u][h];
+          }
+          if (base + kHU * kThreads < my_n) fetch(i0 + kHU * kThreads, hm, z);
+          uint64_t qrow[kHU];
+#pragma unroll
+          for (int u = 0; u < kHU; ++u) qrow[u] = 0;
+#pragma unroll
+          for (int u = 0; u < kHU; ++u) {
+            uint32_t d[G], c[G];
+            unsigned long long m[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              const bool v = (hm_c[u] >> h) & 1u;
+              const uint32_t b = quant_bucket(z_c[u][h], S.st[h].zlo, S.st[h].zscale);
+              qrow[u] |= (uint64_t)b << (8 * h);
+              d[h] = v ? b : (uint32_t)lane;  // spread the zero adds of absent heads
+              m[h] = v ? mass_fixed(z_c[u][h], S.zmax[h]) : 0ull;
+              c[h] = v ? 1u : 0u;
             }
+            hist_add_heads<G>(S, d, m, c);
           }
 #pragma unroll
           for (int u = 0; u < kHU; ++u)
@@ -928,53 +972,87 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
         uint64_t qb_pack = 0;
 #pragma unroll
         for (int h = 0; h < G; ++h) qb_pack |= (uint64_t)(S.st[h].qbeta & 0xffu) << (8 * h);
-        for (int64_t base = 0; base < my_n; base += kHU * kThreads) {
-          const int64_t i0 = base + kHU * tid;
-          uint32_t mem[kHU];
-          float z[kHU][G];
+        uint32_t mem[kHU];
+        float z[kHU][G];
+        auto fetch = [&](int64_t i0, uint32_t* memo, float (*zo)[G]) {
 #pragma unroll
           for (int u = 0; u < kHU; ++u) {
             const bool in = i0 + u < my_n;
             const uint32_t hm = in ? (cc[i0 + u] >> 24) & open_heads : 0u;
-            mem[u] = hm ? hm & bytes_eq(load_qrow<G>(qown, i0 + u), qb_pack) : 0u;
-            if (mem[u]) load_scores<G>(zown, i0 + u, z[u]);
+            memo[u] = hm ? hm & bytes_eq(load_qrow<G>(qown, i0 + u), qb_pack) : 0u;
+            if (in) load_scores<G>(zown, i0 + u, zo[u]);
+          }
+        };
+        fetch(kHU * tid, mem, z);
+        for (int64_t base = 0; base < my_n; base += kHU * kThreads) {
+          const int64_t i0 = base + kHU * tid;
+          uint32_t mem_c[kHU];
+          float z_c[kHU][G];
+#pragma unroll
+          for (int u = 0; u < kHU; ++u) {
+            mem_c[u] = mem[u];
+#pragma unroll
+            for (int h = 0; h < G; ++h) z_c[u][h] = z[u][h];
+          }
+          if (base + kHU * kThreads < my_n) fetch(i0 + kHU * kThreads, mem, z);
+          // members in the group's key interval, per candidate (bit h = head h)
+          uint32_t vm[kHU];
+#pragma unroll
+          for (int u = 0; u < kHU; ++u) {
+            vm[u] = 0u;
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              if (!((mem_c[u] >> h) & 1u)) continue;
+              const uint32_t key = order_key(z_c[u][h]);
+              if (key >= S.st[h].kgmin && key <= S.st[h].kgmax) vm[u] |= 1u << h;
+            }
           }
 #pragma unroll
-          for (int h = 0; h < G; ++h) {
-            if (!((open_heads >> h) & 1u)) continue;
-            const HeadState& st = S.st[h];
-            const bool gather = (gather_heads >> h) & 1u;
-            int sh = 0, w = 0;
-            radix_digit(st.kgmin, st.kgmax, &sh, &w);
+          for (int h = 0; h < G; ++h) {  // heads narrowed by another histogram pass
+            if (!((hist_heads >> h) & 1u)) continue;
+            int sh, w;
+            radix_digit(S.st[h].kgmin, S.st[h].kgmax, &sh, &w);
 #pragma unroll
-            for (int u = 0; u < kHU; ++u) {
-              bool v = (mem[u] >> h) & 1u;
-              uint32_t key = 0;
-              if (v) {
-                key = order_key(z[u][h]);
-                v = key >= st.kgmin && key <= st.kgmax;
+            for (int u = 0; u < kHU; ++u)
+              if ((vm[u] >> h) & 1u)
+                hist_add(S, h, (order_key(z_c[u][h]) >> sh) & ((1u << w) - 1u),
+                         mass_fixed(z_c[u][h], S.zmax[h]));
+          }
+          if (gather_heads) {
+            // ship the members to the heads' owners: lane h reserves the
+            // warp's slots for head h with one DSMEM atomic
+            unsigned mb[kHU][G];
+            unsigned cnt = 0;
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+#pragma unroll
+              for (int u = 0; u < kHU; ++u) {
+                mb[u][h] = ((gather_heads >> h) & 1u)
+                               ? __ballot_sync(0xffffffffu, (vm[u] >> h) & 1u)
+                               : 0u;
+                if (lane == h) cnt += __popc(mb[u][h]);
               }
-              if (gather) {  // one slot reservation per warp and head
-                const unsigned mb = __ballot_sync(0xffffffffu, v);
-                if (mb) {
-                  const int slot = h / C;
-                  const int leader = __ffs(mb) - 1;
-                  unsigned first_slot = 0;
-                  if (lane == leader)
-                    first_slot = atomicAdd(&cluster.map_shared_rank(&S, h % C)->mlist_n[slot],
-                                           (unsigned)__popc(mb));
-                  first_slot = __shfl_sync(0xffffffffu, first_slot, leader);
-                  if (v) {
-                    const unsigned k = first_slot + __popc(mb & ((1u << lane) - 1u));
-                    if (k < (unsigned)kGather) {
-                      Smem* O = cluster.map_shared_rank(&S, h % C);
-                      O->mz[slot * kGather + k] = z[u][h];
-                      O->mpos[slot * kGather + k] = ((uint32_t)rank << 24) | (uint32_t)(i0 + u);
-                    }
+            unsigned first_slot = 0;
+            if (lane < G && cnt)
+              first_slot = atomicAdd(&cluster.map_shared_rank(&S, lane % C)->mlist_n[lane / C], cnt);
+            const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+              if (!((gather_heads >> h) & 1u)) continue;
+              unsigned k0 = __shfl_sync(0xffffffffu, first_slot, h);
+              Smem* O = cluster.map_shared_rank(&S, h % C);
+              float* oz = list_z(*O) + (h / C) * kGather;
+              uint32_t* op = list_pos(*O, list_slots(G, C)) + (h / C) * kGather;
+#pragma unroll
+              for (int u = 0; u < kHU; ++u) {
+                if ((vm[u] >> h) & 1u) {
+                  const unsigned k = k0 + __popc(mb[u][h] & lt);
+                  if (k < (unsigned)kGather) {
+                    oz[k] = z_c[u][h];
+                    op[k] = ((uint32_t)rank << 24) | (uint32_t)(i0 + u);
                   }
                 }
-              } else if (v) {
-                hist_add(S, h, (key >> sh) & ((1u << w) - 1u), mass_fixed(z[u][h], S.zmax[h]));
+                k0 += __popc(mb[u][h]);
               }
             }
           }
@@ -983,7 +1061,8 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
       cluster.sync();  // every rank's histograms and shipped members complete
       for (int h = rank; h < G; h += C) {
         if ((hist_heads >> h) & 1u) owner_pass<G>(p, S, cluster, C, h);
-        else if ((gather_heads >> h) & 1u) owner_finish<G>(p, S, h, h / C, mk_u, seg);
+        else if ((gather_heads >> h) & 1u)
+          owner_finish<G>(p, S, h, h / C, list_slots(G, C), mk_u, seg);
       }
       cluster.sync();  // every owner published
       {  // copy the new states of the open heads from their owners
@@ -1140,6 +1219,7 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
         my_n = seg;
       }
     }
+    if (level > 1) cur ^= 1;  // the expanded segment is the next frontier
 
     if (level == 1 && p.list_mode) {
       // per-head ascending token lists: {0} (unless node 0 is kept) + tokens of
@@ -1197,16 +1277,20 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
         }
       }
     }
-    cur ^= 1;
     __syncthreads();
   }
   // no CTA may leave while another can still read its shared memory
   cluster.sync();
 }
 
+// Dynamic shared memory of a CTA: the struct plus its shipped-member lists.
+size_t smem_bytes(int G, int C) {
+  return sizeof(Smem) + (size_t)list_slots(G, C) * kGather * (sizeof(float) + sizeof(uint32_t));
+}
+
 template <typename T, int D, int G>
 cudaError_t launch_t(const TravParams& p, int64_t units, int C, cudaStream_t stream) {
-  const size_t smem = sizeof(Smem);
+  const size_t smem = smem_bytes(G, C);
   auto kern = traverse_kernel<T, D, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
@@ -1251,7 +1335,7 @@ template <typename T, int D, int G>
 int max_clusters_t(int C) {
   auto kern = traverse_kernel<T, D, G>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)sizeof(Smem)) != cudaSuccess)
+                           (int)smem_bytes(G, C)) != cudaSuccess)
     return (cudaGetLastError(), 0);
   if (C > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
                    cudaSuccess)
@@ -1259,7 +1343,7 @@ int max_clusters_t(int C) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)C, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = sizeof(Smem);
+  cfg.dynamicSmemBytes = smem_bytes(G, C);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = C;
