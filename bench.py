@@ -173,6 +173,25 @@ def oracle_rate(wl, n_queries: int, budget_s: float = 20.0):
 # the CUDA path
 # ---------------------------------------------------------------------------
 
+def max_over_ranks(x: float, device=None) -> float:
+    """The largest value of x over the ranks of the default process group (x
+    itself without one). Only this scalar crosses ranks: the replicas share no
+    data."""
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def throughput(queries_per_step: int, steps: int, world: int, ms_total_max: float) -> float:
+    """Whole-job queries/s: every rank runs `steps` steps of its own replica;
+    the job takes as long as the slowest rank."""
+    return queries_per_step * steps * world / (ms_total_max / 1e3)
+
+
 def workload_config(args, c):
     kv_gb = 2 * c.batch * c.n_kv_heads * c.n_tokens * c.head_dim * (2 if c.dtype == "bf16" else 4) / 1e9
     return {"workload": args.workload, "batch": c.batch, "context": c.n_tokens,
@@ -267,13 +286,10 @@ def run_zha(args, rank, world, dev):
     ms_ext = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
     ms_sel = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
     ms_att = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
-    if world > 1:
-        tt = torch.tensor([ms_total], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(tt.item())
+    ms_total = max_over_ranks(ms_total, dev)
     ms_step = ms_total / args.steps
     queries_per_step = B * Hq
-    value = queries_per_step * args.steps * world / (ms_total / 1e3)
+    value = throughput(queries_per_step, args.steps, world, ms_total)
 
     # ---- bytes touched per step (work counters of the last timed step) ----
     stats = torch.zeros(B * Hkv, L + 1, dtype=torch.int32, device=dev)
@@ -304,7 +320,7 @@ def run_zha(args, rank, world, dev):
         z.zha_dense_decode(cfg, cache, queries[i % n_steps_cap], out, wsd)
     e1.record()
     torch.cuda.synchronize()
-    dense_ms = e0.elapsed_time(e1) / nd
+    dense_ms = max_over_ranks(e0.elapsed_time(e1) / nd, dev)
     dense_bytes = B * Hkv * n_last * 2 * row + 2 * queries_per_step * row
 
     # ---- end to end through the API with host buffers ----
@@ -336,10 +352,7 @@ def run_zha(args, rank, world, dev):
     e1.record()
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / ne
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(e2e_ms, dev)
     h2d = kv_host[0].numel() * kv_host.element_size() + q_host[0].numel() * q_host.element_size()
     d2h = out_host[0].numel() * out_host.element_size()
 
