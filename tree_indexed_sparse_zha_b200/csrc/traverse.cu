@@ -59,6 +59,7 @@ constexpr int kBuckets = 1 << kDigit;     // == kThreads: one bucket per thread
 constexpr int kCandPerThread = 4;
 constexpr uint32_t kNodeMask = 0x00ffffffu;
 constexpr int kGather = 512;  // groups this small are finished by the head's owner alone
+constexpr int kSingleMax = 2048;  // frontiers this small are traversed by rank 0 alone
 static_assert(kBuckets == kThreads, "one histogram bucket per thread");
 
 enum HeadMode : int {
@@ -166,15 +167,21 @@ struct Smem {
   unsigned int mlist_n[kMaxGroup];
   alignas(16) unsigned long long mrank_m[kGather];   // member sort keys
   unsigned long long red_scan[kWarps];
+  // rank 0's hand-over of a grown frontier to the whole cluster
+  int sw_level;                         // level the cluster resumes at (0: finished)
+  int sw_cur;                           // candidate buffer holding the frontier
+  unsigned int sw_n;                    // frontier size
 };
 
-// Shipped-member lists after the struct: z[slots][kGather], then
-// position[slots][kGather] with position = (rank << 24) | segment index.
+// Shipped-member lists after the struct: z[slots][cap], then
+// position[slots][cap] with position = (rank << 24) | segment index. The area
+// holds list_slots(G, C) * kGather entries of each; while rank 0 works alone
+// it owns every head and splits the area into G slots of fewer entries.
 __device__ __forceinline__ float* list_z(Smem& S) {
   return reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(&S) + sizeof(Smem));
 }
-__device__ __forceinline__ uint32_t* list_pos(Smem& S, int slots) {
-  return reinterpret_cast<uint32_t*>(list_z(S) + slots * kGather);
+__device__ __forceinline__ uint32_t* list_pos(Smem& S, int slots, int cap) {
+  return reinterpret_cast<uint32_t*>(list_z(S) + slots * cap);
 }
 // owned heads per CTA (lists needed)
 __host__ __device__ __forceinline__ int list_slots(int G, int C) { return (G + C - 1) / C; }
@@ -291,8 +298,72 @@ __device__ __forceinline__ uint32_t quant_bucket(float z, float zlo, float zscal
   return f >= 255.0f ? 255u : (uint32_t)f;
 }
 
-// Score candidates [0, n) of a segment against G queries; 4 candidates per
-// thread so that each broadcast of q[i][0..G) feeds 4*G chains. The G scores
+// The canonical dot products of this thread's rows (up to K of them) with the
+// G queries, the rows' 16-byte chunks streamed through this thread's slots of
+// S.ring with DEPTH chunks per row (K * DEPTH <= 12): chunk ch of row k sits
+// in slot (ch % DEPTH) * K + k. Only this thread writes and reads its slots,
+// so waiting on its own cp.async groups suffices.
+template <typename T, int D, int G, int K, int DEPTH>
+__device__ __forceinline__ void stream_rows(Smem& S, const uint4* const* rows, const bool* ok,
+                                            float2 (*acc)[(G + 1) / 2], float* acc1) {
+  static_assert(K * DEPTH <= 3 * kCandPerThread, "ring slots per thread");
+  constexpr int kPer = Elem<T>::kPerChunk;
+  constexpr int kNch = D * (int)sizeof(T) / 16;
+  const int tid = threadIdx.x;
+  uint4* slots = &S.ring[0][0][0];  // slot s of this thread at slots[s * kThreads + tid]
+#pragma unroll
+  for (int st = 0; st < DEPTH - 1; ++st) {
+#pragma unroll
+    for (int k = 0; k < K; ++k)
+      if (ok[k] && st < kNch) cp_async16(&slots[(st * K + k) * kThreads + tid], rows[k] + st);
+    cp_async_commit();
+  }
+#pragma unroll 1
+  for (int ch = 0; ch < kNch; ++ch) {
+    if (ch + DEPTH - 1 < kNch) {
+      const int st = (ch + DEPTH - 1) % DEPTH;
+#pragma unroll
+      for (int k = 0; k < K; ++k)
+        if (ok[k]) cp_async16(&slots[(st * K + k) * kThreads + tid], rows[k] + ch + DEPTH - 1);
+    }
+    cp_async_commit();
+    cp_async_wait<DEPTH - 1>();  // this thread's copies of chunk ch have landed
+    float x[K][kPer];
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+      const uint4 c = ok[k] ? slots[((ch % DEPTH) * K + k) * kThreads + tid] : make_uint4(0, 0, 0, 0);
+      Elem<T>::unpack(c, x[k]);
+    }
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) {
+      const float* qv = S.q + (ch * kPer + e) * kMaxGroup;
+      if constexpr (G == 1) {
+#pragma unroll
+        for (int k = 0; k < K; ++k) acc1[k] = __fmaf_rn(qv[0], x[k][e], acc1[k]);
+      } else if constexpr (G == 2) {
+        const float2 q2 = *reinterpret_cast<const float2*>(qv);
+#pragma unroll
+        for (int k = 0; k < K; ++k) acc[k][0] = ffma2(q2, make_float2(x[k][e], x[k][e]), acc[k][0]);
+      } else {
+        float4 q4[G / 4];
+#pragma unroll
+        for (int j = 0; j < G / 4; ++j) q4[j] = *reinterpret_cast<const float4*>(qv + 4 * j);
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+          const float2 xx = make_float2(x[k][e], x[k][e]);
+#pragma unroll
+          for (int j = 0; j < G / 4; ++j) {
+            acc[k][2 * j] = ffma2(make_float2(q4[j].x, q4[j].y), xx, acc[k][2 * j]);
+            acc[k][2 * j + 1] = ffma2(make_float2(q4[j].z, q4[j].w), xx, acc[k][2 * j + 1]);
+          }
+        }
+      }
+    }
+  }
+}
+
+// Score candidates [0, n) of a segment against G queries; up to 4 candidates
+// per thread so that each broadcast of q[i][0..G) feeds 4*G chains. The G scores
 // of candidate i go to zseg[i*G .. i*G+G). lmax/lmin accumulate the extremes
 // over the candidates in each head's frontier.
 template <typename T, int D, int G>
@@ -300,8 +371,6 @@ __device__ __forceinline__ void score_segment(const TravParams& p, Smem& S, cons
                                               const uint32_t* cand, float* zseg, int64_t n,
                                               float lns, float* lmax, float* lmin, bool top,
                                               int64_t top_base) {
-  constexpr int kPer = Elem<T>::kPerChunk;
-  constexpr int kNch = D * (int)sizeof(T) / 16;
   const int tid = threadIdx.x;
   const uint64_t pol_z = policy_evict_last();
   for (int64_t base = 0; base < n; base += kThreads * kCandPerThread) {
@@ -326,57 +395,16 @@ __device__ __forceinline__ void score_segment(const TravParams& p, Smem& S, cons
 #pragma unroll
       for (int j = 0; j < (G + 1) / 2; ++j) acc[k][j] = make_float2(0.0f, 0.0f);
     }
-    // each thread streams its rows' 16-byte chunks through its own slots of a
-    // 3-stage shared-memory ring: two chunks in flight while one is used
-    uint4 cur[kCandPerThread];
-#pragma unroll
-    for (int st = 0; st < 2; ++st) {
-#pragma unroll
-      for (int k = 0; k < kCandPerThread; ++k)
-        if (ok[k] && st < kNch) cp_async16(&S.ring[st][k][tid], rows[k] + st);
-      cp_async_commit();
-    }
-#pragma unroll 1
-    for (int ch = 0; ch < kNch; ++ch) {
-      if (ch + 2 < kNch) {
-#pragma unroll
-        for (int k = 0; k < kCandPerThread; ++k)
-          if (ok[k]) cp_async16(&S.ring[(ch + 2) % 3][k][tid], rows[k] + ch + 2);
-      }
-      cp_async_commit();
-      cp_async_wait<2>();  // this thread's copies of chunk ch have landed
-#pragma unroll
-      for (int k = 0; k < kCandPerThread; ++k)
-        cur[k] = ok[k] ? S.ring[ch % 3][k][tid] : make_uint4(0, 0, 0, 0);
-      float x[kCandPerThread][kPer];
-#pragma unroll
-      for (int k = 0; k < kCandPerThread; ++k) Elem<T>::unpack(cur[k], x[k]);
-#pragma unroll
-      for (int e = 0; e < kPer; ++e) {
-        const float* qv = S.q + (ch * kPer + e) * kMaxGroup;
-        if constexpr (G == 1) {
-#pragma unroll
-          for (int k = 0; k < kCandPerThread; ++k) acc1[k] = __fmaf_rn(qv[0], x[k][e], acc1[k]);
-        } else if constexpr (G == 2) {
-          const float2 q2 = *reinterpret_cast<const float2*>(qv);
-#pragma unroll
-          for (int k = 0; k < kCandPerThread; ++k)
-            acc[k][0] = ffma2(q2, make_float2(x[k][e], x[k][e]), acc[k][0]);
-        } else {
-          float4 q4[G / 4];
-#pragma unroll
-          for (int j = 0; j < G / 4; ++j) q4[j] = *reinterpret_cast<const float4*>(qv + 4 * j);
-#pragma unroll
-          for (int k = 0; k < kCandPerThread; ++k) {
-            const float2 xx = make_float2(x[k][e], x[k][e]);
-#pragma unroll
-            for (int j = 0; j < G / 4; ++j) {
-              acc[k][2 * j] = ffma2(make_float2(q4[j].x, q4[j].y), xx, acc[k][2 * j]);
-              acc[k][2 * j + 1] = ffma2(make_float2(q4[j].z, q4[j].w), xx, acc[k][2 * j + 1]);
-            }
-          }
-        }
-      }
+    // each thread streams its rows' 16-byte chunks through its own 12 slots of
+    // a shared-memory ring: 11 chunks in flight with one row, 5 per row with
+    // two rows, 2 per row with three or four
+    const int kr = ok[3] ? 4 : ok[2] ? 3 : ok[1] ? 2 : ok[0] ? 1 : 0;
+    if (kr == 1) {
+      stream_rows<T, D, G, 1, 12>(S, rows, ok, acc, acc1);
+    } else if (kr == 2) {
+      stream_rows<T, D, G, 2, 6>(S, rows, ok, acc, acc1);
+    } else if (kr > 2) {
+      stream_rows<T, D, G, 4, 3>(S, rows, ok, acc, acc1);
     }
 #pragma unroll
     for (int k = 0; k < kCandPerThread; ++k) {
@@ -487,6 +515,62 @@ __device__ __forceinline__ void radix_digit(unsigned kgmin, unsigned kgmax, int*
   *sh = shift - *w;
 }
 
+// The state of a head after a pass found its crossing bucket beta (ok):
+// above / cabove are the mass and count ranked above the bucket, bcnt / bmass
+// the bucket's, [gmin, gmax] its key interval and tie_cnt[r] its members in
+// segment r.
+__device__ __forceinline__ HeadState narrow_state(const TravParams& p, const HeadState& s0,
+                                                  bool quant, bool ok, unsigned long long need,
+                                                  unsigned beta, unsigned long long above,
+                                                  unsigned cabove, unsigned bcnt,
+                                                  unsigned long long bmass, uint32_t gmin,
+                                                  uint32_t gmax, const unsigned* tie_cnt, int C,
+                                                  unsigned nh) {
+  HeadState ns = s0;
+  ns.need = need;
+  if (!ok) {  // cannot happen with exact sums; keep everything rather than loop
+    raise_status(p.status, ZHA_ERR_INTERNAL);
+    ns.mode = kModeAll;
+    ns.count = nh;
+    return ns;
+  }
+  ns.above = above;
+  ns.cabove = cabove;
+  ns.bmass = bmass;
+  ns.bcnt = bcnt;
+  ns.kgmin = gmin;
+  ns.kgmax = gmax;
+  if (quant) ns.qbeta = beta;
+  ns.zfree = quant ? 1 : 0;  // a final rule set now needs no scores in the expand
+  ns.mode = kModeRadix;
+  if (bcnt == 1u) {
+    ns.mode = kModeThr;  // the group's only member is the last kept candidate;
+    ns.kthr = ns.kgmin;  // no other candidate has a key in the group's interval
+    ns.count = ns.cabove + 1u;
+  } else if (ns.kgmin == ns.kgmax) {
+    // bcnt members share one key, hence one z and one mass: keep the first
+    // tie_need of them in node order
+    const unsigned long long mt = ns.bmass / bcnt;
+    const unsigned long long rem = need - ns.above;
+    const unsigned long long tn = mt ? (rem + mt - 1) / mt : bcnt;
+    ns.kthr = ns.kgmin;
+    if (tn >= bcnt) {
+      ns.mode = kModeThr;
+      ns.count = ns.cabove + bcnt;
+    } else {
+      ns.mode = kModeTie;
+      ns.count = ns.cabove + (unsigned)tn;
+      unsigned long long run = 0;
+      for (int r = 0; r < C; ++r) {
+        const unsigned long long cr = tie_cnt[r];
+        ns.quota[r] = (unsigned)(run >= tn ? 0ull : (tn - run < cr ? tn - run : cr));
+        run += cr;
+      }
+    }
+  }
+  return ns;
+}
+
 // Owner step of one pass for head h (every thread of the owner CTA calls it):
 // sums the C per-rank histograms of h through DSMEM, finds the bucket where
 // the mass in descending score order reaches the target, narrows the head's
@@ -584,51 +668,9 @@ __device__ __noinline__ void owner_pass(const TravParams& p, Smem& S, cg::cluste
     S.tie_cnt[tid] = R->hist_c[h][beta];
   }
   if (tie) __syncthreads();
-  if (tid == 0) {
-    HeadState ns = s0;
-    ns.need = need;
-    if (!ok) {  // cannot happen with exact sums; keep everything rather than loop
-      raise_status(p.status, ZHA_ERR_INTERNAL);
-      ns.mode = kModeAll;
-      ns.count = S.nh[h];
-    } else {
-      ns.above = S.found_u64[0];
-      ns.cabove = S.found[1];
-      ns.bmass = S.found_u64[1];
-      ns.bcnt = bcnt;
-      ns.kgmin = gmin;
-      ns.kgmax = gmax;
-      if (quant) ns.qbeta = beta;
-      ns.zfree = quant ? 1 : 0;  // a final rule set now needs no scores in the expand
-      ns.mode = kModeRadix;
-      if (bcnt == 1u) {
-        ns.mode = kModeThr;  // the group's only member is the last kept candidate;
-        ns.kthr = ns.kgmin;  // no other candidate has a key in the group's interval
-        ns.count = ns.cabove + 1u;
-      } else if (ns.kgmin == ns.kgmax) {
-        // bcnt members share one key, hence one z and one mass: keep the first
-        // tie_need of them in node order
-        const unsigned long long mt = ns.bmass / bcnt;
-        const unsigned long long rem = need - ns.above;
-        const unsigned long long tn = mt ? (rem + mt - 1) / mt : bcnt;
-        ns.kthr = ns.kgmin;
-        if (tn >= bcnt) {
-          ns.mode = kModeThr;
-          ns.count = ns.cabove + bcnt;
-        } else {
-          ns.mode = kModeTie;
-          ns.count = ns.cabove + (unsigned)tn;
-          unsigned long long run = 0;
-          for (int r = 0; r < C; ++r) {
-            const unsigned long long cr = S.tie_cnt[r];
-            ns.quota[r] = (unsigned)(run >= tn ? 0ull : (tn - run < cr ? tn - run : cr));
-            run += cr;
-          }
-        }
-      }
-    }
-    S.pub[h] = ns;
-  }
+  if (tid == 0)
+    S.pub[h] = narrow_state(p, s0, quant, ok, need, beta, S.found_u64[0], S.found[1], bcnt,
+                            S.found_u64[1], gmin, gmax, S.tie_cnt, C, S.nh[h]);
   __syncthreads();
 }
 
@@ -640,17 +682,17 @@ __device__ __noinline__ void owner_pass(const TravParams& p, Smem& S, cg::cluste
 // and publishes kModeGathered in S.pub[h].
 template <int G>
 __device__ __noinline__ void owner_finish(const TravParams& p, Smem& S, int h, int slot,
-                                          int slots, uint8_t* mk_u, int64_t seg) {
+                                          int slots, int cap, uint8_t* mk_u, int64_t seg) {
   static_assert(kGather == 2 * kThreads, "two sort slots per thread");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const HeadState s0 = S.st[h];
-  const int n = (int)(S.mlist_n[slot] < (unsigned)kGather ? S.mlist_n[slot] : kGather);
+  const int n = (int)(S.mlist_n[slot] < (unsigned)cap ? S.mlist_n[slot] : cap);
   int np2 = 2;
   while (np2 < n) np2 <<= 1;
   unsigned long long* key = S.mrank_m;  // sort keys, descending
   for (int i = tid; i < np2; i += kThreads)
-    key[i] = i < n ? ((unsigned long long)order_key(list_z(S)[slot * kGather + i]) << 32) |
-                         (0xffffffffu - list_pos(S, slots)[slot * kGather + i])
+    key[i] = i < n ? ((unsigned long long)order_key(list_z(S)[slot * cap + i]) << 32) |
+                         (0xffffffffu - list_pos(S, slots, cap)[slot * cap + i])
                    : 0ull;
   __syncthreads();
   for (int k = 2; k <= np2; k <<= 1) {
@@ -710,6 +752,194 @@ __device__ __noinline__ void owner_finish(const TravParams& p, Smem& S, int h, i
     S.pub[h] = ns;
   }
   __syncthreads();
+}
+
+// Single-CTA versions of the owner steps (rank 0 alone owns every head): warp
+// h handles head h, so the G heads are narrowed concurrently. Same results as
+// owner_pass / owner_finish with C = 1.
+constexpr int kWarpGather = kGather / kMaxGroup;  // members per head, single-CTA gathers
+
+template <int G>
+__device__ __noinline__ void owner_pass_warp(const TravParams& p, Smem& S, int h) {
+  const int lane = threadIdx.x & 31;
+  const HeadState s0 = S.st[h];
+  const bool quant = s0.mode == kModeQuant;
+  int nb = kBuckets;
+  if (!quant) {
+    int sh, w;
+    radix_digit(s0.kgmin, s0.kgmax, &sh, &w);
+    nb = 1 << w;
+  }
+  constexpr int kPer = kBuckets / 32;  // buckets per lane, lane-major
+  unsigned long long m[kPer];
+  unsigned int c[kPer];
+  unsigned long long tm = 0;
+  unsigned int tc = 0;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int d = lane * kPer + j;
+    m[j] = d < nb ? ((unsigned long long)S.hist_hi[h][d] << 32) | S.hist_lo[h][d] : 0ull;
+    c[j] = d < nb ? S.hist_c[h][d] : 0u;
+    tm += m[j];
+    tc += c[j];
+  }
+  unsigned long long xs = tm;  // inclusive suffix over lanes (higher lanes rank first)
+  unsigned int xc = tc;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const unsigned long long ym = __shfl_down_sync(0xffffffffu, xs, off);
+    const unsigned int yc = __shfl_down_sync(0xffffffffu, xc, off);
+    if (lane + off < 32) {
+      xs += ym;
+      xc += yc;
+    }
+  }
+  const unsigned long long total = __shfl_sync(0xffffffffu, xs, 0);
+  const unsigned long long need = quant ? ceil_mul_shift32(total, p.p_q) : s0.need;
+  unsigned long long run = s0.above + (xs - tm);
+  unsigned int runc = s0.cabove + (xc - tc);
+  int fbeta = -1;
+  unsigned long long fabove = 0, fbmass = 0;
+  unsigned int fcab = 0, fbcnt = 0;
+#pragma unroll
+  for (int j = kPer - 1; j >= 0; --j) {
+    const int d = lane * kPer + j;
+    if (d < nb && run < need && run + m[j] >= need) {
+      fbeta = d;
+      fabove = run;
+      fbmass = m[j];
+      fcab = runc;
+      fbcnt = c[j];
+    }
+    run += m[j];
+    runc += c[j];
+  }
+  const unsigned fmask = __ballot_sync(0xffffffffu, fbeta >= 0);
+  const bool ok = fmask != 0u;
+  const int src = ok ? __ffs(fmask) - 1 : 0;
+  const unsigned beta = (unsigned)__shfl_sync(0xffffffffu, fbeta, src);
+  const unsigned long long above = __shfl_sync(0xffffffffu, fabove, src);
+  const unsigned long long bmass = __shfl_sync(0xffffffffu, fbmass, src);
+  const unsigned cabove = __shfl_sync(0xffffffffu, fcab, src);
+  const unsigned bcnt = __shfl_sync(0xffffffffu, fbcnt, src);
+  if (lane == 0) {
+    uint32_t gmin = 0, gmax = 0;
+    if (ok) {
+      if (quant && s0.zscale == 0.0f) {
+        gmin = gmax = order_key(s0.zlo);
+      } else if (quant) {
+        quant_interval(s0.zlo, s0.zscale, beta, &gmin, &gmax);
+      } else {
+        int sh, w;
+        radix_digit(s0.kgmin, s0.kgmax, &sh, &w);
+        const uint32_t top = (uint32_t)(((unsigned long long)s0.kgmin >> (sh + w)) << (sh + w));
+        const uint32_t dlo = top | (beta << sh);
+        const uint32_t dhi = dlo | (uint32_t)((1ull << sh) - 1ull);
+        gmin = dlo > s0.kgmin ? dlo : s0.kgmin;
+        gmax = dhi < s0.kgmax ? dhi : s0.kgmax;
+      }
+    }
+    const unsigned tie_cnt[1] = {bcnt};
+    S.pub[h] = narrow_state(p, s0, quant, ok, need, beta, above, cabove, bcnt, bmass, gmin, gmax,
+                            tie_cnt, 1, S.nh[h]);
+  }
+  __syncwarp();
+}
+
+template <int G>
+__device__ __noinline__ void owner_finish_warp(const TravParams& p, Smem& S, int h, int slots,
+                                               int cap, uint8_t* mk_u, int64_t seg) {
+  const int lane = threadIdx.x & 31;
+  const HeadState s0 = S.st[h];
+  const int n = (int)(S.mlist_n[h] < (unsigned)cap ? S.mlist_n[h] : cap);
+  const float* mz = list_z(S) + h * cap;
+  const uint32_t* mpos = list_pos(S, slots, cap) + h * cap;
+  unsigned long long* mass = S.mrank_m + h * kWarpGather;  // by rank
+  const float zmax = S.zmax[h];
+  constexpr int kPerLane = kWarpGather / 32;
+  unsigned rk[kPerLane];
+#pragma unroll
+  for (int t = 0; t < kPerLane; ++t) {
+    const int i = lane + 32 * t;
+    rk[t] = 0u;
+    if (i < n) {
+      const float zi = mz[i];
+      const uint32_t pi = mpos[i];
+      for (int j = 0; j < n; ++j) {
+        const float zj = mz[j];
+        rk[t] += (zj > zi || (zj == zi && mpos[j] < pi)) ? 1u : 0u;
+      }
+      mass[rk[t]] = mass_fixed(zi, zmax);
+    }
+  }
+  __syncwarp();
+  // lane l owns ranks kPerLane*l .. kPerLane*l + kPerLane - 1
+  unsigned long long mr[kPerLane], tsum = 0;
+#pragma unroll
+  for (int t = 0; t < kPerLane; ++t) {
+    const int r = kPerLane * lane + t;
+    mr[t] = r < n ? mass[r] : 0ull;
+    tsum += mr[t];
+  }
+  unsigned long long x = tsum;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const unsigned long long y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  unsigned long long run = x - tsum;  // mass of lower ranks
+  const unsigned long long rem = s0.need - s0.above;
+  int kf = -1;
+#pragma unroll
+  for (int t = 0; t < kPerLane; ++t) {
+    const int r = kPerLane * lane + t;
+    if (r < n && run < rem && run + mr[t] >= rem) kf = r;
+    run += mr[t];
+  }
+  const unsigned kmask = __ballot_sync(0xffffffffu, kf >= 0);
+  const bool ok = kmask != 0u && n == (int)s0.bcnt;
+  unsigned k = kmask ? (unsigned)__shfl_sync(0xffffffffu, kf, __ffs(kmask) - 1) : 0u;
+  if (!ok) k = (unsigned)n - 1u;  // cannot happen with exact sums: keep the whole group
+#pragma unroll
+  for (int t = 0; t < kPerLane; ++t) {
+    const int i = lane + 32 * t;
+    if (i < n) {
+      const uint32_t pi = mpos[i];
+      mk_u[((int64_t)(pi >> 24) * seg + (pi & kNodeMask)) * G + h] = rk[t] <= k ? 1 : 0;
+    }
+  }
+  if (lane == 0) {
+    if (!ok) raise_status(p.status, ZHA_ERR_INTERNAL);
+    HeadState ns = s0;
+    ns.mode = kModeGathered;
+    ns.count = s0.cabove + k + 1u;
+    S.pub[h] = ns;
+  }
+  __syncwarp();
+}
+
+// After the hand-over barrier: reads where rank 0 left its frontier and copies
+// this rank's equal slice of it (rank 0's segment of buffer *cur) into this
+// rank's segment of the same buffer. Returns the slice length; *level = 0
+// when rank 0 finished alone.
+__device__ __noinline__ int64_t join_frontier(Smem& S, cg::cluster_group& cluster, int C,
+                                              int rank, uint32_t* cand_u, int64_t seg,
+                                              int* level, int* cur) {
+  const Smem* R0 = cluster.map_shared_rank(&S, 0);
+  *level = R0->sw_level;
+  *cur = R0->sw_cur;
+  const int64_t n = R0->sw_n;
+  int64_t len = 0;
+  if (*level > 0) {
+    const int64_t lo = n * rank / C, hi = n * (rank + 1) / C;
+    const uint32_t* src = cand_u + (int64_t)*cur * C * seg;  // rank 0's segment
+    uint32_t* dst = cand_u + ((int64_t)*cur * C + rank) * seg;
+    for (int64_t g = lo + threadIdx.x; g < hi; g += kThreads) dst[g - lo] = __ldcg(src + g);
+    len = hi - lo;
+    if (threadIdx.x < kMaxGroup) S.my_hcnt[threadIdx.x] = 0u;  // rank 0 carries the totals
+  }
+  __syncthreads();
+  return len;
 }
 
 // Final keep rule of one head for a candidate with order key `key`; *member
@@ -797,11 +1027,38 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
     return;  // uniform across the cluster and before any DSMEM access
   }
 
-  // my segment at the top level: a contiguous range of the complete top nodes
-  const int64_t top_lo = T_top * rank / C;
-  int64_t my_n = T_top * (rank + 1) / C - top_lo;
+  // Small frontiers are traversed by rank 0 alone (Ce = 1, CTA barriers
+  // only); when a frontier outgrows kSingleMax rank 0 hands it over and the
+  // whole cluster (Ce = C) takes equal slices of it. Every rank passes the
+  // hand-over barrier exactly once.
+  const bool single = C > 1 && T_top <= kSingleMax;
+  int Ce = single ? 1 : C;
+  int level = p.L;
   int cur = 0;
-  for (int level = p.L; level >= 1; --level) {
+  // my segment at the top level: a contiguous range of the complete top nodes
+  int64_t top_lo = single ? 0 : T_top * rank / C;
+  int64_t my_n = single ? T_top : T_top * (rank + 1) / C - top_lo;
+  bool joined = !single;  // passed the hand-over barrier
+  if (single && rank != 0) {
+    cluster.sync();  // hand-over: rank 0's frontier (or its finish) is published
+    joined = true;
+    my_n = join_frontier(S, cluster, C, rank, cand_u, seg, &level, &cur);
+    if (level > 0) Ce = C;
+    else if (!p.list_mode && tid == 0)
+      p.n_kept[(int64_t)unit * C + rank] = 0;  // rank 0 produced every kept node
+  }
+  for (; level >= 1; --level) {
+    if (Ce == 1 && single && level < p.L && my_n > kSingleMax) {  // rank 0 hands over
+      if (tid == 0) {
+        S.sw_level = level;
+        S.sw_cur = cur;
+        S.sw_n = (unsigned int)my_n;
+      }
+      cluster.sync();   // hand-over
+      joined = true;
+      my_n = my_n / C;  // rank 0's slice is the prefix of its own segment
+      Ce = C;
+    }
     const bool top = level == p.L;
     const T* lvl = static_cast<const T*>(p.tree) + p.level_off[level - 1] +
                    (int64_t)tree_unit * p.level_rows[level - 1] * D;
@@ -848,13 +1105,14 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
       }
       if (tid == 0) X.count = (unsigned int)my_n;
     }
-    cluster.sync();  // S1: every segment scored
+    if (Ce > 1) cluster.sync();  // S1: every segment scored
+    else __syncthreads();
     if (p.stats && tid == 0) atomicAdd(&p.stats[(int64_t)unit * p.L + (p.L - level)], (int)my_n);
 
     // ------------------------------------------------------------------
     // 2. distributed cut
     // ------------------------------------------------------------------
-    for (int e = tid; e < C * (3 * G + 1); e += kThreads) {  // one parallel DSMEM gather
+    for (int e = tid; e < Ce * (3 * G + 1); e += kThreads) {  // one parallel DSMEM gather
       const int r = e / (3 * G + 1), k = e % (3 * G + 1);
       const Xch* rx = &cluster.map_shared_rank(&S, r)->xch[level & 1];
       if (k == 0) S.seg_n[r] = rx->count;
@@ -866,7 +1124,7 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
     if (tid < G) {
       float mx = -INFINITY, mn = INFINITY;
       unsigned int n = 0;
-      for (int r = 0; r < C; ++r) {
+      for (int r = 0; r < Ce; ++r) {
         mx = fmaxf(mx, S.g_zmax[r][tid]);
         mn = fminf(mn, S.g_zmin[r][tid]);
         n += S.g_hcnt[r][tid];
@@ -891,6 +1149,9 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
       S.mlist_n[tid] = 0u;  // my gather lists (slots of the heads I own)
     }
     __syncthreads();
+    // entries per shipped-member list (rank 0 alone: one list per head, each
+    // finished by one warp)
+    const int cap = Ce > 1 ? kGather : kWarpGather;
     for (int pass = 0; pass < 40; ++pass) {  // every pass strictly narrows each group
       // heads whose group is still open: histogram pass, or (small group)
       // shipped to the owner who finishes the cut alone
@@ -900,7 +1161,7 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
         const int m = S.st[h].mode;
         if (m == kModeQuant) hist_heads |= 1u << h;
         else if (m == kModeRadix)
-          (S.st[h].bcnt <= (unsigned)kGather ? gather_heads : hist_heads) |= 1u << h;
+          (S.st[h].bcnt <= (unsigned)cap ? gather_heads : hist_heads) |= 1u << h;
       }
       const unsigned open_heads = hist_heads | gather_heads;
       if (!open_heads) break;  // uniform: every CTA holds the same states
@@ -1034,20 +1295,21 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
               }
             unsigned first_slot = 0;
             if (lane < G && cnt)
-              first_slot = atomicAdd(&cluster.map_shared_rank(&S, lane % C)->mlist_n[lane / C], cnt);
+              first_slot =
+                  atomicAdd(&cluster.map_shared_rank(&S, lane % Ce)->mlist_n[lane / Ce], cnt);
             const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
             for (int h = 0; h < G; ++h) {
               if (!((gather_heads >> h) & 1u)) continue;
               unsigned k0 = __shfl_sync(0xffffffffu, first_slot, h);
-              Smem* O = cluster.map_shared_rank(&S, h % C);
-              float* oz = list_z(*O) + (h / C) * kGather;
-              uint32_t* op = list_pos(*O, list_slots(G, C)) + (h / C) * kGather;
+              Smem* O = cluster.map_shared_rank(&S, h % Ce);
+              float* oz = list_z(*O) + (h / Ce) * cap;
+              uint32_t* op = list_pos(*O, list_slots(G, Ce), cap) + (h / Ce) * cap;
 #pragma unroll
               for (int u = 0; u < kHU; ++u) {
                 if ((vm[u] >> h) & 1u) {
                   const unsigned k = k0 + __popc(mb[u][h] & lt);
-                  if (k < (unsigned)kGather) {
+                  if (k < (unsigned)cap) {
                     oz[k] = z_c[u][h];
                     op[k] = ((uint32_t)rank << 24) | (uint32_t)(i0 + u);
                   }
@@ -1058,19 +1320,27 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
           }
         }
       }
-      cluster.sync();  // every rank's histograms and shipped members complete
-      for (int h = rank; h < G; h += C) {
-        if ((hist_heads >> h) & 1u) owner_pass<G>(p, S, cluster, C, h);
-        else if ((gather_heads >> h) & 1u)
-          owner_finish<G>(p, S, h, h / C, list_slots(G, C), mk_u, seg);
+      if (Ce > 1) cluster.sync();  // every rank's histograms and shipped members complete
+      else __syncthreads();
+      if (Ce > 1) {
+        for (int h = rank; h < G; h += Ce) {
+          if ((hist_heads >> h) & 1u) owner_pass<G>(p, S, cluster, Ce, h);
+          else if ((gather_heads >> h) & 1u)
+            owner_finish<G>(p, S, h, h / Ce, list_slots(G, Ce), cap, mk_u, seg);
+        }
+      } else if (warp < G) {  // one warp per head
+        if ((hist_heads >> warp) & 1u) owner_pass_warp<G>(p, S, warp);
+        else if ((gather_heads >> warp) & 1u)
+          owner_finish_warp<G>(p, S, warp, list_slots(G, Ce), cap, mk_u, seg);
       }
-      cluster.sync();  // every owner published
+      if (Ce > 1) cluster.sync();  // every owner published
+      else __syncthreads();
       {  // copy the new states of the open heads from their owners
         constexpr int kWords = (int)(sizeof(HeadState) / 4);
         for (int e = tid; e < G * kWords; e += kThreads) {
           const int h = e / kWords, k = e % kWords;
           if (!((open_heads >> h) & 1u)) continue;
-          const Smem* R = cluster.map_shared_rank(&S, h % C);
+          const Smem* R = cluster.map_shared_rank(&S, h % Ce);
           reinterpret_cast<unsigned int*>(&S.st[h])[k] =
               reinterpret_cast<const unsigned int*>(&R->pub[h])[k];
         }
@@ -1228,12 +1498,13 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
       const int64_t n1 = S.seg_n[rank];  // candidates of my segment at level 1
       if (tid == 0)
         S.node0 = (n1 > 0 && (cc[0] & kNodeMask) == 0u) ? km_seg[0] : 0u;
-      cluster.sync();  // every rank's kept counts published
+      if (Ce > 1) cluster.sync();  // every rank's kept counts published
+      else __syncthreads();
       unsigned int base[G], total[G];
       uint32_t node0 = 0;
 #pragma unroll
       for (int h = 0; h < G; ++h) base[h] = total[h] = 0u;
-      for (int r = 0; r < C; ++r) {
+      for (int r = 0; r < Ce; ++r) {
         const Smem* R = cluster.map_shared_rank(&S, r);
 #pragma unroll
         for (int h = 0; h < G; ++h) {
@@ -1265,7 +1536,7 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
           prun += tot;
         }
         if (rank == 0 && tid == 0 && off0 == 1 && p.idx_cap > 0) out[0] = 0;
-        if (rank == C - 1) {
+        if (rank == Ce - 1) {
           const int64_t tail_pos = off0 + (int64_t)b * total[h];
           for (int64_t j = tid; j < tail_len; j += kThreads)
             if (tail_pos + j < p.idx_cap) out[tail_pos + j] = (int32_t)(tail_start + j);
@@ -1278,6 +1549,10 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
       }
     }
     __syncthreads();
+  }
+  if (!joined) {  // rank 0 finished alone: release the waiting ranks
+    if (tid == 0) S.sw_level = 0;
+    cluster.sync();  // hand-over
   }
   // no CTA may leave while another can still read its shared memory
   cluster.sync();
