@@ -59,7 +59,7 @@ constexpr int kBuckets = 1 << kDigit;     // == kThreads: one bucket per thread
 constexpr int kCandPerThread = 4;
 constexpr uint32_t kNodeMask = 0x00ffffffu;
 constexpr int kGather = 512;  // groups this small are finished by the head's owner alone
-constexpr int kSingleMax = 2048;  // frontiers this small are traversed by rank 0 alone
+constexpr int kSingleMax = 512;  // frontiers this small are traversed by rank 0 alone
 static_assert(kBuckets == kThreads, "one histogram bucket per thread");
 
 enum HeadMode : int {
@@ -167,6 +167,7 @@ struct Smem {
   unsigned int mlist_n[kMaxGroup];
   alignas(16) unsigned long long mrank_m[kGather];   // member sort keys
   unsigned long long red_scan[kWarps];
+  unsigned int lm_n;                    // members staged in S.mrank_m before shipping
   // rank 0's hand-over of a grown frontier to the whole cluster
   int sw_level;                         // level the cluster resumes at (0: finished)
   int sw_cur;                           // candidate buffer holding the frontier
@@ -454,7 +455,7 @@ __device__ __forceinline__ void hist_add_heads(Smem& S, const uint32_t* d,
                                                const unsigned long long* m, const uint32_t* c) {
   unsigned old[G];
 #pragma unroll
-  for (int h = 0; h < G; ++h) old[h] = atomicAdd(&S.hist_lo[h][d[h]], (unsigned)m[h]);
+  for (int h = 0; h < G; ++h) old[h] = c[h] ? atomicAdd(&S.hist_lo[h][d[h]], (unsigned)m[h]) : 0u;
 #pragma unroll
   for (int h = 0; h < G; ++h) {
     const unsigned lo = (unsigned)m[h];
@@ -1166,6 +1167,7 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
       const unsigned open_heads = hist_heads | gather_heads;
       if (!open_heads) break;  // uniform: every CTA holds the same states
       const bool first = pass == 0;  // every open head is in kModeQuant
+      if (tid == 0) S.lm_n = 0u;
       if (hist_heads)
         for (int e = tid; e < G * kBuckets; e += kThreads) {
           (&S.hist_lo[0][0])[e] = 0u;
@@ -1233,29 +1235,28 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
         uint64_t qb_pack = 0;
 #pragma unroll
         for (int h = 0; h < G; ++h) qb_pack |= (uint64_t)(S.st[h].qbeta & 0xffu) << (8 * h);
+        // the next candidates' masks and bucket bytes are in flight while the
+        // current members' scores are loaded and shipped
         uint32_t mem[kHU];
-        float z[kHU][G];
-        auto fetch = [&](int64_t i0, uint32_t* memo, float (*zo)[G]) {
+        auto fetch = [&](int64_t i0, uint32_t* memo) {
 #pragma unroll
           for (int u = 0; u < kHU; ++u) {
             const bool in = i0 + u < my_n;
             const uint32_t hm = in ? (cc[i0 + u] >> 24) & open_heads : 0u;
             memo[u] = hm ? hm & bytes_eq(load_qrow<G>(qown, i0 + u), qb_pack) : 0u;
-            if (in) load_scores<G>(zown, i0 + u, zo[u]);
           }
         };
-        fetch(kHU * tid, mem, z);
+        fetch(kHU * tid, mem);
         for (int64_t base = 0; base < my_n; base += kHU * kThreads) {
           const int64_t i0 = base + kHU * tid;
           uint32_t mem_c[kHU];
           float z_c[kHU][G];
 #pragma unroll
-          for (int u = 0; u < kHU; ++u) {
-            mem_c[u] = mem[u];
+          for (int u = 0; u < kHU; ++u) mem_c[u] = mem[u];
+          if (base + kHU * kThreads < my_n) fetch(i0 + kHU * kThreads, mem);
 #pragma unroll
-            for (int h = 0; h < G; ++h) z_c[u][h] = z[u][h];
-          }
-          if (base + kHU * kThreads < my_n) fetch(i0 + kHU * kThreads, mem, z);
+          for (int u = 0; u < kHU; ++u)  // scores of this thread's group members only
+            if (mem_c[u]) load_scores<G>(zown, i0 + u, z_c[u]);
           // members in the group's key interval, per candidate (bit h = head h)
           uint32_t vm[kHU];
 #pragma unroll
@@ -1280,42 +1281,76 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
                          mass_fixed(z_c[u][h], S.zmax[h]));
           }
           if (gather_heads) {
-            // ship the members to the heads' owners: lane h reserves the
-            // warp's slots for head h with one DSMEM atomic
-            unsigned mb[kHU][G];
-            unsigned cnt = 0;
+            // stage the members locally: entry = z (low word) and
+            // (head << 28) | (rank << 24) | index (high word); a full stage
+            // ships the rest directly
 #pragma unroll
-            for (int h = 0; h < G; ++h)
+            for (int u = 0; u < kHU; ++u) {
+              const uint32_t gv = vm[u] & gather_heads;
+              const unsigned nb = __popc(gv);
+              unsigned excl = nb;
 #pragma unroll
-              for (int u = 0; u < kHU; ++u) {
-                mb[u][h] = ((gather_heads >> h) & 1u)
-                               ? __ballot_sync(0xffffffffu, (vm[u] >> h) & 1u)
-                               : 0u;
-                if (lane == h) cnt += __popc(mb[u][h]);
+              for (int off = 1; off < 32; off <<= 1) {
+                const unsigned y = __shfl_up_sync(0xffffffffu, excl, off);
+                if (lane >= off) excl += y;
               }
-            unsigned first_slot = 0;
-            if (lane < G && cnt)
-              first_slot =
-                  atomicAdd(&cluster.map_shared_rank(&S, lane % Ce)->mlist_n[lane / Ce], cnt);
-            const unsigned lt = (1u << lane) - 1u;
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-              if (!((gather_heads >> h) & 1u)) continue;
-              unsigned k0 = __shfl_sync(0xffffffffu, first_slot, h);
-              Smem* O = cluster.map_shared_rank(&S, h % Ce);
-              float* oz = list_z(*O) + (h / Ce) * cap;
-              uint32_t* op = list_pos(*O, list_slots(G, Ce), cap) + (h / Ce) * cap;
-#pragma unroll
-              for (int u = 0; u < kHU; ++u) {
-                if ((vm[u] >> h) & 1u) {
-                  const unsigned k = k0 + __popc(mb[u][h] & lt);
-                  if (k < (unsigned)cap) {
-                    oz[k] = z_c[u][h];
-                    op[k] = ((uint32_t)rank << 24) | (uint32_t)(i0 + u);
+              const unsigned wtot = __shfl_sync(0xffffffffu, excl, 31);
+              excl -= nb;
+              unsigned wbase = 0;
+              if (lane == 0 && wtot) wbase = atomicAdd(&S.lm_n, wtot);
+              wbase = __shfl_sync(0xffffffffu, wbase, 0);
+              uint32_t rest = gv;
+              unsigned k = wbase + excl;
+              while (rest) {
+                const int h = __ffs(rest) - 1;
+                rest &= rest - 1;
+                const uint32_t tag = ((uint32_t)h << 28) | ((uint32_t)rank << 24) | (uint32_t)(i0 + u);
+                if (k < (unsigned)kGather) {
+                  S.mrank_m[k] = ((unsigned long long)tag << 32) | __float_as_uint(z_c[u][h]);
+                } else {  // stage full: reserve one owner slot directly
+                  Smem* O = cluster.map_shared_rank(&S, h % Ce);
+                  const unsigned ko = atomicAdd(&O->mlist_n[h / Ce], 1u);
+                  if (ko < (unsigned)cap) {
+                    list_z(*O)[(h / Ce) * cap + ko] = z_c[u][h];
+                    list_pos(*O, list_slots(G, Ce), cap)[(h / Ce) * cap + ko] = tag & 0x0fffffffu;
                   }
                 }
-                k0 += __popc(mb[u][h]);
+                ++k;
               }
+            }
+          }
+        }
+        if (gather_heads) {
+          // ship the staged members: warp h reserves the owner's slots for head
+          // h with one DSMEM atomic and copies its members over
+          __syncthreads();
+          const unsigned n_st = S.lm_n < (unsigned)kGather ? S.lm_n : (unsigned)kGather;
+          for (int h = warp; h < G; h += kWarps) {
+            if (!((gather_heads >> h) & 1u)) continue;
+            unsigned cnt = 0;
+            for (unsigned e = lane; e < n_st; e += 32) cnt += (unsigned)(S.mrank_m[e] >> 60) == (unsigned)h;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+            if (!cnt) continue;
+            Smem* O = cluster.map_shared_rank(&S, h % Ce);
+            unsigned base = 0;
+            if (lane == 0) base = atomicAdd(&O->mlist_n[h / Ce], cnt);
+            base = __shfl_sync(0xffffffffu, base, 0);
+            float* oz = list_z(*O) + (h / Ce) * cap;
+            uint32_t* op = list_pos(*O, list_slots(G, Ce), cap) + (h / Ce) * cap;
+            for (unsigned e0 = 0; e0 < n_st; e0 += 32) {
+              const unsigned e = e0 + lane;
+              const unsigned long long v = e < n_st ? S.mrank_m[e] : 0ull;
+              const bool mine = e < n_st && (unsigned)(v >> 60) == (unsigned)h;
+              const unsigned mb = __ballot_sync(0xffffffffu, mine);
+              if (mine) {
+                const unsigned k = base + __popc(mb & ((1u << lane) - 1u));
+                if (k < (unsigned)cap) {
+                  oz[k] = __uint_as_float((uint32_t)v);
+                  op[k] = (uint32_t)(v >> 32) & 0x0fffffffu;
+                }
+              }
+              base += __popc(mb);
             }
           }
         }
