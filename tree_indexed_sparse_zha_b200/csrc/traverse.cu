@@ -295,8 +295,7 @@ __device__ __forceinline__ uint32_t bytes_nz(uint64_t a) {
 // operations on every CTA.
 __device__ __forceinline__ uint32_t quant_bucket(float z, float zlo, float zscale) {
   const float f = __fmul_rn(__fsub_rn(z, zlo), zscale);
-  if (!(f > 0.0f)) return 0u;
-  return f >= 255.0f ? 255u : (uint32_t)f;
+  return (uint32_t)fminf(fmaxf(f, 0.0f), 255.0f);  // NaN (inf * 0) maps to 0
 }
 
 // The canonical dot products of this thread's rows (up to K of them) with the
@@ -1218,7 +1217,8 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
               const uint32_t b = quant_bucket(z_c[u][h], S.st[h].zlo, S.st[h].zscale);
               qrow[u] |= (uint64_t)b << (8 * h);
               d[h] = v ? b : (uint32_t)lane;  // spread the zero adds of absent heads
-              m[h] = v ? mass_fixed(z_c[u][h], S.zmax[h]) : 0ull;
+              // computed for every head (independent chains), kept for present ones
+              m[h] = mass_fixed(z_c[u][h], S.zmax[h]) & (0ull - (unsigned long long)v);
               c[h] = v ? 1u : 0u;
             }
             hist_add_heads<G>(S, d, m, c);

@@ -26,7 +26,10 @@ constexpr int kMaxCluster = 16;   // CTAs cooperating on one traversal unit
 // exact power 2^n. Returns 0 below -87 (W. J. Cody and W. Waite, "Software
 // Manual for the Elementary Functions", 1980).
 __device__ __forceinline__ float exp_canon(float x) {
-  if (x < -87.0f) return 0.0f;
+  // branch-free, so that independent calls interleave; below -87 the result is
+  // selected away (the scaling below would not be a valid power of two there)
+  const bool zero = x < -87.0f;
+  x = zero ? 0.0f : x;
   const float n = rintf(__fmul_rn(x, 0x1.715476p+0f));
   float r = __fmaf_rn(-n, 0x1.62e4p-1f, x);
   r = __fmaf_rn(-n, 0x1.7f7d1cp-20f, r);
@@ -39,7 +42,7 @@ __device__ __forceinline__ float exp_canon(float x) {
   p = __fmaf_rn(p, r, 1.0f);
   p = __fmaf_rn(p, r, 1.0f);
   const int ni = __float2int_rn(n);  // in [-126, 0]
-  return __fmul_rn(p, __int_as_float((ni + 127) << 23));
+  return zero ? 0.0f : __fmul_rn(p, __int_as_float((ni + 127) << 23));
 }
 
 // Fixed-point node mass trunc(exp(z - zmax) * 2^40).
