@@ -43,6 +43,7 @@ struct AttParams {
   const int32_t* q_pos;    // tree stream with explicit positions (prefill)
   int64_t ncap;
   int Hq, Hkv, G, b, L, B;
+  int b_shift;             // log2(b) when b is a power of two, else -1
   int64_t span_L;
   float qscale;            // log2(e) / sqrt(d)
   // tree stream
@@ -96,7 +97,11 @@ __device__ __forceinline__ void row_of(const AttParams& p, const Span& s, int64_
     v -= s.tok0;
     const int64_t nrows = (s.n1 - s.n0) * p.b;
     if (v < nrows) {
-      const int64_t j = s.n0 + v / p.b;
+      // node slot and offset within the node (v < 2^31: a CTA's share of a unit)
+      const uint32_t vv = (uint32_t)v;
+      const uint32_t q = p.b_shift >= 0 ? vv >> p.b_shift : vv / (uint32_t)p.b;
+      const int off = (int)(vv - q * (uint32_t)p.b);
+      const int64_t j = s.n0 + q;
       uint32_t e;
       if (s.kept_local) {
         e = s.kept_local[j - s.n0];
@@ -106,7 +111,6 @@ __device__ __forceinline__ void row_of(const AttParams& p, const Span& s, int64_
         e = s.kept[r * s.stride + (j - s.segbase[r])];
       }
       const int64_t node = e & 0x00ffffffu;
-      const int off = (int)(v % p.b);
       *row = node * p.b + off;
       *mask = (node == 0 && off == 0) ? 0u : (e >> 24);
       return;
@@ -421,10 +425,12 @@ __global__ void __launch_bounds__(Cfg<T, D>::kThreads, 1) attend_kernel(AttParam
 template <int D>
 struct MmaCfg {
   static constexpr int kRowBytes = D * 2;
-  static constexpr int kStages = 3;
+  // 6 warps x 2 stages (one block in flight while one is computed): more
+  // warps to issue the per-block work than 4 x 3, with the same shared memory
+  static constexpr int kStages = 2;
   static constexpr int kStageBytes = 32 * kRowBytes * 2;             // K and V of 32 rows
   static constexpr int kWarpBytes = kStages * kStageBytes + kStages * 32;  // + row masks
-  static constexpr int kWarps = 4;
+  static constexpr int kWarps = 6;
   static constexpr int kKeptCap = 5120;   // kept-list entries staged in shared memory
   static constexpr int kThreads = 32 * kWarps;
   static constexpr int kKSteps = D / 16;   // QK k-steps
@@ -824,6 +830,7 @@ cudaError_t launch_attend(const Geometry& g, const AttendArgs& a, void* ws, size
   p.B = g.B;
   p.G = a.kind == kStreamList ? 1 : g.G;
   p.b = g.b;
+  p.b_shift = (g.b & (g.b - 1)) == 0 ? __builtin_ctz((unsigned)g.b) : -1;
   p.L = g.L;
   p.span_L = g.span[g.L];
   p.qscale = kLog2e * g.inv_sqrt_d;
