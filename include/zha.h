@@ -191,11 +191,40 @@ zha_status zha_decode_stats(const zha_config* cfg, const void* ws, size_t ws_byt
  * Extends the tree over the chunk, then for every token i of the chunk
  * (position chunk_start + i) and head h selects causally and attends:
  * q [T][Hq][d] -> out [T][Hq][d]. level_counts ([T][Hq][L]) is nullable.
- * ws: ZHA_OP_PREFILL workspace for max_queries = T. */
+ * ws: ZHA_OP_PREFILL workspace for max_queries = T.
+ * The top level of every (token, head) is first scored on the tensor cores
+ * (zha_prefill_top_scores) when the geometry allows it; a (token, KV head)
+ * whose tensor-core selection is certified skips the top level's canonical
+ * scoring. Certified or not, every selection equals the canonical one. */
 zha_status zha_prefill_chunk(const zha_config* cfg, const zha_cache* cache, const void* q,
                              int32_t seq, int64_t chunk_start, int64_t T, double p, void* out,
                              int32_t* level_counts, void* ws, size_t ws_bytes,
                              int32_t* dev_status, void* stream);
+
+/* Tensor-core top-level scores of a prefill chunk and their certificates
+ * (lefilia page, par. 1: a query scores the top nodes first; in a chunk all
+ * (token, head) queries of a KV head score the same top summaries, so this is
+ * one bf16 GEMM per KV head on tcgen05 with fp32 accumulation in TMEM).
+ *   - Input: the tree must already cover the chunk (zha_prefill_chunk extends
+ *     it; or zha_build_tree / zha_extend_tree); q [T][Hq][d] as in
+ *     zha_prefill_chunk, 16-byte aligned; positions chunk_start + i.
+ *   - z_top (nullable, device): [T][Hq][capacity / b^L] fp32; entry [i][h][n]
+ *     is the tensor-core score fl(fl(acc * 1/sqrt(d)) + L ln b) of top node n
+ *     for n < T_top(i) = (chunk_start + i + 1) / b^L; later entries untouched.
+ *     It differs from the canonical score by at most a bound derived from
+ *     |q| |s_n| (no rounding-order guarantee).
+ *   - certified (nullable, device): [T][Hq] int32, 1 when the canonical cut
+ *     over the top level is proven equal to the cut taken on z_top (the proof
+ *     is the same one zha_prefill_chunk relies on), else 0.
+ *   - ws: ZHA_OP_PREFILL workspace for max_queries >= T (not preserved).
+ *   - Errors: ZHA_ERR_UNSUPPORTED unless dtype is bf16, head_dim 128, L >= 2,
+ *     G <= 8 and capacity / b^L <= 1024; ZHA_ERR_INVALID_ARG for a bad chunk,
+ *     p or a misaligned q; ZHA_ERR_TIMEOUT in dev_status if the tensor-core
+ *     completion wait ran out. Asynchronous on `stream`. */
+zha_status zha_prefill_top_scores(const zha_config* cfg, const zha_cache* cache, const void* q,
+                                  int32_t seq, int64_t chunk_start, int64_t T, double p,
+                                  float* z_top, int32_t* certified, void* ws, size_t ws_bytes,
+                                  int32_t* dev_status, void* stream);
 
 /* Dense flash-decoding over every key [0, seq_len[b] - 1] (the baseline the
  * sparse path is measured against): q [B][Hq][d] -> out [B][Hq][d].

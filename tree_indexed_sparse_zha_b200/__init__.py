@@ -42,7 +42,7 @@ EXPORTS = (
     "zha_status_string", "zha_tree_layout", "zha_workspace_bytes", "zha_build_tree",
     "zha_extend_tree", "zha_select", "zha_attend", "zha_decode", "zha_decode_select",
     "zha_decode_attend", "zha_decode_stats", "zha_prefill_chunk", "zha_dense_decode",
-    "zha_decode_noalloc",
+    "zha_decode_noalloc", "zha_prefill_top_scores",
 )
 
 
@@ -107,6 +107,8 @@ def lib() -> ctypes.CDLL:
                                   i32),
             "zha_dense_decode": ([c_cfg, c_cache, vp, vp, vp, sz, vp], i32),
             "zha_decode_noalloc": ([c_cfg, c_cache, vp, d, vp, vp, vp, vp], i32),
+            "zha_prefill_top_scores": ([c_cfg, c_cache, vp, i32, i64, i64, d, vp, vp, vp, sz, vp,
+                                        vp], i32),
         }
         for name, (args, res) in sig.items():
             f = getattr(L, name)
@@ -273,6 +275,19 @@ def zha_dense_decode(cfg: zha_config, cache: Cache, q: torch.Tensor, out: torch.
     _check("zha_dense_decode", lib().zha_dense_decode(
         ctypes.byref(cfg), ctypes.byref(c), _ptr(q), _ptr(out), _ptr(ws), ws.numel(),
         _stream(stream)))
+
+
+def zha_prefill_top_scores(cfg: zha_config, cache: Cache, q: torch.Tensor, seq: int,
+                           chunk_start: int, p: float, z_top: Optional[torch.Tensor],
+                           certified: Optional[torch.Tensor], ws: torch.Tensor,
+                           dev_status: Optional[torch.Tensor] = None, stream=None):
+    """Tensor-core top-level scores (z_top [T][Hq][capacity // b**L] fp32) and
+    per-(token, head) certificates (certified [T][Hq] int32) of a prefill chunk
+    whose tree is already built."""
+    c = cache.c()
+    _check("zha_prefill_top_scores", lib().zha_prefill_top_scores(
+        ctypes.byref(cfg), ctypes.byref(c), _ptr(q), seq, chunk_start, q.shape[0], float(p),
+        _ptr(z_top), _ptr(certified), _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream)))
 
 
 def zha_decode_noalloc(cfg: zha_config, cache: Cache, q: torch.Tensor, p: float,

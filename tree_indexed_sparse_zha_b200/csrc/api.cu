@@ -114,7 +114,7 @@ static int64_t prefill_tile(const Geometry& g, int64_t T, int sms) {
 }
 
 struct PrefillLayout {
-  size_t old_len, q_seq, q_pos, dec, total;
+  size_t old_len, q_seq, q_pos, dec, top, top_bytes, total;
   int64_t tile;
   DecodeLayout d;
 };
@@ -132,6 +132,10 @@ static PrefillLayout prefill_layout(const Geometry& g, int64_t T, int sms) {
   P.dec = off;
   P.d = decode_layout(g, P.tile, kStreamTree, sms);
   off = align256(off + P.d.total);
+  // tensor-core top level of the whole chunk (scores, certificates, seeds)
+  P.top = off;
+  P.top_bytes = top_tc_ws_bytes(g, T);
+  off = align256(off + P.top_bytes);
   P.total = off;
   return P;
 }
@@ -292,14 +296,14 @@ static zha_status run_tree_select(const Geometry& g, const zha_cache* cache, con
                                   const int32_t* q_seq, const int32_t* q_pos, int64_t nq,
                                   uint64_t p_q, int32_t* level_counts, unsigned char* ws,
                                   const DecodeLayout& L, int32_t* dev_status, int sms,
-                                  cudaStream_t s) {
+                                  cudaStream_t s, const TopSeeds* seeds = nullptr) {
   TraverseOut to{};
   to.kept = reinterpret_cast<uint32_t*>(ws + L.kept);
   to.n_kept = reinterpret_cast<int32_t*>(ws + L.n_kept);
   to.stats = reinterpret_cast<int32_t*>(ws + L.stats);
   to.level_counts = level_counts;
   return cuda_status(launch_traverse(g, cache->tree, q, cache->seq_len, q_seq, q_pos, nq, p_q, 0,
-                                     to, ws + L.trav, L.kept - L.trav, dev_status, sms, s));
+                                     to, ws + L.trav, L.kept - L.trav, dev_status, sms, s, seeds));
 }
 
 static zha_status run_tree_attend(const Geometry& g, const zha_cache* cache, const void* q,
@@ -327,9 +331,9 @@ static zha_status run_tree_decode(const Geometry& g, const zha_cache* cache, con
                                   const int32_t* q_seq, const int32_t* q_pos, int64_t nq,
                                   uint64_t p_q, void* out, int32_t* level_counts,
                                   unsigned char* ws, const DecodeLayout& L, int32_t* dev_status,
-                                  int sms, cudaStream_t s) {
+                                  int sms, cudaStream_t s, const TopSeeds* seeds = nullptr) {
   zha_status st = run_tree_select(g, cache, q, q_seq, q_pos, nq, p_q, level_counts, ws, L,
-                                  dev_status, sms, s);
+                                  dev_status, sms, s, seeds);
   if (st != ZHA_OK) return st;
   return run_tree_attend(g, cache, q, q_seq, q_pos, nq, out, ws, L, sms, s);
 }
@@ -434,6 +438,15 @@ zha_status zha_prefill_chunk(const zha_config* cfg, const zha_cache* cache, cons
   if (cudaGetLastError() != cudaSuccess) return ZHA_ERR_CUDA;
   cudaError_t e = launch_tree(g, cache->k, cache->tree, cache->r, cache->seq_len, old_len, T, s);
   if (e != cudaSuccess) return ZHA_ERR_CUDA;
+  // the top level of every (token, KV head) of the chunk on the tensor cores;
+  // certified units skip it in the traversal, the rest score it canonically
+  TopSeeds seeds{};
+  const bool tc = P.top_bytes > 0 && (reinterpret_cast<uintptr_t>(q) & 15) == 0;
+  if (tc) {
+    e = launch_top_select(g, cache->tree, cache->seq_len, seq, q, chunk_start, T, p_q, w + P.top,
+                          P.top_bytes, &seeds, nullptr, nullptr, dev_status, s);
+    if (e != cudaSuccess) return ZHA_ERR_CUDA;
+  }
   const size_t row_bytes = (size_t)g.Hq * g.d * g.elem_bytes;
   for (int64_t i0 = 0; i0 < T; i0 += P.tile) {
     const int64_t n = (T - i0) < P.tile ? (T - i0) : P.tile;
@@ -441,13 +454,43 @@ zha_status zha_prefill_chunk(const zha_config* cfg, const zha_cache* cache, cons
                                                                       chunk_start + i0, n);
     if (cudaGetLastError() != cudaSuccess) return ZHA_ERR_CUDA;
     const DecodeLayout L = decode_layout(g, n, kStreamTree, sms);
+    TopSeeds ts{};
+    if (tc) {
+      ts.ok = seeds.ok + i0 * g.Hkv;
+      ts.mask = seeds.mask + i0 * g.Hkv * seeds.stride;
+      ts.cnt = seeds.cnt + i0 * g.Hkv * g.G;
+      ts.stride = seeds.stride;
+    }
     st = run_tree_decode(g, cache, static_cast<const unsigned char*>(q) + i0 * row_bytes, q_seq,
                          q_pos, n, p_q, static_cast<unsigned char*>(out) + i0 * row_bytes,
                          level_counts ? level_counts + i0 * g.Hq * g.L : nullptr, w + P.dec, L,
-                         dev_status, sms, s);
+                         dev_status, sms, s, tc ? &ts : nullptr);
     if (st != ZHA_OK) return st;
   }
   return ZHA_OK;
+}
+
+zha_status zha_prefill_top_scores(const zha_config* cfg, const zha_cache* cache, const void* q,
+                                  int32_t seq, int64_t chunk_start, int64_t T, double p,
+                                  float* z_top, int32_t* certified, void* ws, size_t ws_bytes,
+                                  int32_t* dev_status, void* stream) {
+  Geometry g;
+  zha_status st = make_geometry(cfg, &g);
+  if (st != ZHA_OK) return st;
+  if ((st = check_cache(cache, false)) != ZHA_OK) return st;
+  uint64_t p_q;
+  if (!q || !ws || T < 1 || seq < 0 || seq >= g.B || chunk_start < 0 ||
+      chunk_start + T > g.ncap || !check_p(p, &p_q) || (reinterpret_cast<uintptr_t>(q) & 15))
+    return ZHA_ERR_INVALID_ARG;
+  if (!top_tc_supported(g)) return ZHA_ERR_UNSUPPORTED;
+  const int sms = device_sm_count();
+  const PrefillLayout P = prefill_layout(g, T, sms);
+  if (ws_bytes < P.total) return ZHA_ERR_WORKSPACE;
+  TopSeeds seeds{};
+  return cuda_status(launch_top_select(g, cache->tree, cache->seq_len, seq, q, chunk_start, T,
+                                       p_q, static_cast<unsigned char*>(ws) + P.top, P.top_bytes,
+                                       &seeds, z_top, certified, dev_status,
+                                       (cudaStream_t)stream));
 }
 
 zha_status zha_dense_decode(const zha_config* cfg, const zha_cache* cache, const void* q,

@@ -101,6 +101,12 @@ struct TravParams {
   int32_t* level_counts;
   int32_t* stats;        // [units][L]: union candidates scored per level (nullable)
   int32_t* status;
+  // certified top-level selections (nullable): a unit with seed_ok != 0
+  // starts one level below the top
+  const int32_t* seed_ok;    // [units]
+  const uint8_t* seed_mask;  // [units][seed_stride] bit h: head h keeps top node i
+  const int32_t* seed_cnt;   // [units][G]
+  int64_t seed_stride;
 };
 
 // Cut state of one head. After every publish step it is identical on all CTAs
@@ -942,6 +948,37 @@ __device__ __noinline__ int64_t join_frontier(Smem& S, cg::cluster_group& cluste
   return len;
 }
 
+// A certified top-level selection (prefill on the tensor cores) expanded into
+// the frontier of the level below, as the expand step would write it: the b
+// children of every top node some head keeps, in node order, each carrying the
+// mask of the heads that keep its parent. Records the top level's per-head
+// counts and candidates. Returns the frontier size.
+template <int G>
+__device__ __noinline__ int64_t seed_frontier(const TravParams& p, Smem& S, int unit,
+                                              int64_t T_top, uint32_t* cn, int32_t* lc_base) {
+  const uint8_t* sm = p.seed_mask + (int64_t)unit * p.seed_stride;
+  const int b = p.b;
+  unsigned int run = 0;
+  for (int64_t base = 0; base < T_top; base += kThreads) {
+    const int64_t i = base + threadIdx.x;
+    const uint32_t m = i < T_top ? (uint32_t)sm[i] & ((1u << G) - 1u) : 0u;
+    unsigned int tot;
+    const unsigned int rk = block_excl_scan(m ? 1u : 0u, &tot, S);
+    if (m)
+      for (int c = 0; c < b; ++c)
+        cn[(int64_t)(run + rk) * b + c] = (m << 24) | ((uint32_t)i * (uint32_t)b + (uint32_t)c);
+    run += tot;
+  }
+  if (threadIdx.x < G) {
+    const int32_t k = p.seed_cnt[(int64_t)unit * G + threadIdx.x];
+    S.my_hcnt[threadIdx.x] = (unsigned int)k * (unsigned int)b;
+    if (lc_base) lc_base[(int64_t)threadIdx.x * p.L] = k;
+  }
+  if (p.stats && threadIdx.x == 0) atomicAdd(&p.stats[(int64_t)unit * p.L], (int)T_top);
+  __syncthreads();
+  return (int64_t)run * b;
+}
+
 // Final keep rule of one head for a candidate with order key `key`; *member
 // reports a kModeTie candidate whose keep depends on its rank among the ties.
 __device__ __forceinline__ bool keep_rule(int mode, unsigned kthr, uint32_t key, bool* member) {
@@ -1039,6 +1076,13 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
   int64_t top_lo = single ? 0 : T_top * rank / C;
   int64_t my_n = single ? T_top : T_top * (rank + 1) / C - top_lo;
   bool joined = !single;  // passed the hand-over barrier
+  // certified top level: its selection is given, rank 0 starts one level lower
+  // (uniform across the cluster: it depends on the unit only)
+  const bool seeded = p.seed_ok && p.L >= 2 && (C == 1 || single) && p.seed_ok[unit] != 0;
+  if (seeded && rank == 0) {
+    my_n = seed_frontier<G>(p, S, unit, T_top, cptr(0), lc_base);
+    level = p.L - 1;
+  }
   if (single && rank != 0) {
     cluster.sync();  // hand-over: rank 0's frontier (or its finish) is published
     joined = true;
@@ -1725,7 +1769,7 @@ cudaError_t launch_traverse(const Geometry& g, const void* tree, const void* q,
                             const int32_t* seq_len, const int32_t* q_seq, const int32_t* q_pos,
                             int64_t nq, uint64_t p_q, int list_mode, const TraverseOut& out,
                             void* ws, size_t ws_bytes, int32_t* status, int num_sms,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, const TopSeeds* seeds) {
   const int64_t units = nq * g.Hkv;
   if (units <= 0) return cudaSuccess;
   if (ws_bytes < traverse_ws_bytes(g, units, num_sms)) return cudaErrorInvalidValue;
@@ -1772,6 +1816,12 @@ cudaError_t launch_traverse(const Geometry& g, const void* tree, const void* q,
   p.level_counts = out.level_counts;
   p.stats = out.stats;
   p.status = status;
+  if (seeds && seeds->ok && g.L >= 2) {
+    p.seed_ok = seeds->ok;
+    p.seed_mask = seeds->mask;
+    p.seed_cnt = seeds->cnt;
+    p.seed_stride = seeds->stride;
+  }
   if (g.dtype == ZHA_BF16) {
     if (g.d == 128) return launch_g<__nv_bfloat16, 128>(g.G, p, units, C, stream);
     return launch_g<__nv_bfloat16, 64>(g.G, p, units, C, stream);

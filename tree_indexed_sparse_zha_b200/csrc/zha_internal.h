@@ -48,6 +48,17 @@ struct TraverseOut {
   int32_t* stats;          // [units][L] union candidates per level (nullable)
 };
 
+// Certified top-level selections (prefill, tensor-core scoring) of `units`
+// (query token, KV head) units, indexed like the traversal's units. When
+// ok[u] != 0 the canonical cut of every head of unit u at the top level is
+// known: mask[u][i] bit h says head h keeps top node i, cnt[u][h] counts them.
+struct TopSeeds {
+  const int32_t* ok;    // [units]
+  const uint8_t* mask;  // [units][stride]
+  const int32_t* cnt;   // [units][G]
+  int64_t stride;
+};
+
 // CTAs per traversal cluster for `units` (query token, KV head) units.
 int traverse_cluster_size(const Geometry& g, int64_t units, int num_sms);
 // Scratch bytes of the traversal (candidate segments, scores, keep bits).
@@ -63,7 +74,23 @@ cudaError_t launch_traverse(const Geometry& g, const void* tree, const void* q,
                             const int32_t* seq_len, const int32_t* q_seq, const int32_t* q_pos,
                             int64_t nq, uint64_t p_q, int list_mode, const TraverseOut& out,
                             void* ws, size_t ws_bytes, int32_t* status, int num_sms,
-                            cudaStream_t stream);
+                            cudaStream_t stream, const TopSeeds* seeds = nullptr);
+
+// ---- prefill top level on the tensor cores ----------------------------------
+// Top nodes per (sequence, KV head): ncap / b^L.
+int64_t top_cap(const Geometry& g);
+// bf16, head_dim 128, L >= 2, at most 8 query heads per KV head and 1024 top nodes.
+bool top_tc_supported(const Geometry& g);
+// Scratch of launch_top_select for n_tok query tokens (0 when unsupported).
+size_t top_tc_ws_bytes(const Geometry& g, int64_t n_tok);
+// Scores the top level of n_tok consecutive query tokens of sequence `seq`
+// (positions pos0 .., q [n_tok][Hq][d]) on the tensor cores and certifies each
+// (token, KV head) unit; *seeds points into ws afterwards. z_out ([n_tok][Hq]
+// [top_cap]) and cert_out ([n_tok][Hq]) are optional diagnostics.
+cudaError_t launch_top_select(const Geometry& g, const void* tree, const int32_t* seq_len,
+                              int seq, const void* q, int64_t pos0, int64_t n_tok, uint64_t p_q,
+                              void* ws, size_t ws_bytes, TopSeeds* seeds, float* z_out,
+                              int32_t* cert_out, int32_t* status, cudaStream_t stream);
 
 // ---- attention ------------------------------------------------------------
 enum StreamKind { kStreamTree = 0, kStreamDense = 1, kStreamList = 2 };
