@@ -9,6 +9,11 @@ head) queries. Inputs are synthetic (seeded Gaussian-mixture keys with planted
 needles) and resident in HBM; K+V (2.15 GB) is larger than L2, so no flush is
 needed between steps.
 
+--workload prefill-deep-1m-chunk4k times chunked prefill instead: a 4096-token
+chunk (16 query / 2 KV heads) after 1,048,576 cached tokens, one step being
+zha_prefill_chunk over the whole chunk (tree extension, tensor-core top level
+with certificates, traversal and sparse attention for all 65,536 queries).
+
 One JSON line on rank 0. Under torchrun every rank runs an independent replica
 (weak scaling, no data-path collective); timing is the max over ranks.
 --impl reference times the CPU oracle on the same metric (a bounded sample).
@@ -30,6 +35,11 @@ import torch  # noqa: E402
 
 WORKLOAD = "decode-deep-256k-b8"
 METRIC = "ZHA decode queries/s at 256K ctx (B=8, p=0.95); % of HBM roofline"
+PREFILL_METRIC = "ZHA chunked-prefill queries/s (4096-token chunk after 1M tokens, p=0.95)"
+
+
+def is_prefill(name: str) -> bool:
+    return name.startswith("prefill")
 
 
 def parse():
@@ -169,6 +179,35 @@ def oracle_rate(wl, n_queries: int, budget_s: float = 20.0):
     return done / el, done, el
 
 
+def oracle_prefill_rate(wl, n_queries: int, budget_s: float = 20.0):
+    """Times the CPU oracle on chunk queries of KV head 0 (tree over the cached
+    context and the chunk built untimed; select + fp64 attention per query)."""
+    import numpy as np  # noqa: F401
+
+    import oracle
+
+    c = wl.cfg
+    n = c.n_tokens + c.chunk
+    K = wl.K[0, 0].float().cpu().numpy()
+    V = wl.V[0, 0].float().cpu().numpy()
+    R = wl.R.float().cpu().numpy()
+    tr = oracle.build_tree(K, n, R, c.block, c.levels, True, c.capacity)
+    q = wl.queries(0).float().cpu().numpy()
+    done = 0
+    t0 = time.perf_counter()
+    i = 0
+    while done < n_queries and time.perf_counter() - t0 < budget_s and i < c.chunk:
+        for h in range(c.group):
+            idx, _, _, _ = oracle.select(q[i, h], tr, c.n_tokens + i, c.p)
+            oracle.attend(q[i, h], K, V, idx)
+            done += 1
+            if done >= n_queries:
+                break
+        i += 1
+    el = time.perf_counter() - t0
+    return done / el, done, el
+
+
 # ---------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------
@@ -193,6 +232,13 @@ def throughput(queries_per_step: int, steps: int, world: int, ms_total_max: floa
 
 
 def workload_config(args, c):
+    if is_prefill(args.workload):
+        kv_gb = 2 * c.n_kv_heads * c.capacity * c.head_dim * 2 / 1e9
+        return {"workload": args.workload, "batch": c.batch, "context": c.n_tokens,
+                "chunk": c.chunk, "heads": f"{c.n_q_heads}q/{c.n_kv_heads}kv",
+                "head_dim": c.head_dim, "tree": f"b={c.block},L={c.levels}", "p": c.p,
+                "queries_per_step": c.chunk * c.n_q_heads,
+                "l2": f"inputs larger than L2 (K+V {kv_gb:.2f} GB), no flush"}
     kv_gb = 2 * c.batch * c.n_kv_heads * c.n_tokens * c.head_dim * (2 if c.dtype == "bf16" else 4) / 1e9
     return {"workload": args.workload, "batch": c.batch, "context": c.n_tokens,
             "heads": f"{c.n_q_heads}q/{c.n_kv_heads}kv", "head_dim": c.head_dim,
@@ -398,6 +444,148 @@ def run_zha(args, rank, world, dev):
     return res, wl
 
 
+def run_prefill(args, rank, world, dev):
+    """One step = zha_prefill_chunk over the whole chunk: the tree extended over
+    the chunk, the top level of every (token, head) scored on the tensor cores
+    and certified, the traversal and sparse attention for every query."""
+    import tree_indexed_sparse_zha_b200 as z
+    from tree_indexed_sparse_zha_b200 import workloads as W
+
+    z.lib()  # fail loudly if the extension is missing
+    wl = W.make(args.workload, device=dev, n_tokens=args.n_tokens)
+    c = wl.cfg
+    cfg = z.make_config(c.head_dim, c.block, c.levels, c.n_q_heads, c.n_kv_heads, c.batch,
+                        c.capacity, c.torch_dtype)
+    Hq, Hkv, D, b, L, T, G = (c.n_q_heads, c.n_kv_heads, c.head_dim, c.block, c.levels, c.chunk,
+                              c.group)
+    start = c.n_tokens
+    len0 = torch.full((1,), start, dtype=torch.int32, device=dev)
+    len1 = torch.full((1,), start + T, dtype=torch.int32, device=dev)
+    cache = z.Cache(wl.K, wl.V, wl.R.float().contiguous(), z.alloc_tree(cfg, dev), len0)
+    ws = z.alloc_workspace(cfg, z.ZHA_OP_PREFILL, T, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    q = wl.queries(0)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+
+    # ---- tree over the cached context (rate reported; not part of a step) ----
+    z.zha_build_tree(cfg, cache)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    z.zha_build_tree(cfg, cache)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    build_ms = e0.elapsed_time(e1)
+
+    def one_step():
+        cache.seq_len = len1
+        z.zha_prefill_chunk(cfg, cache, q, 0, start, c.p, out, None, ws, st)
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {z.status_string(int(st.item()))}")
+    t_start, t_end = torch.cuda.Event(True), torch.cuda.Event(True)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    t_start.record(stream)
+    for _ in range(args.steps):
+        one_step()
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    ms_total = max_over_ranks(t_start.elapsed_time(t_end), dev)
+    ms_step = ms_total / args.steps
+    queries_per_step = T * Hq
+    value = throughput(queries_per_step, args.steps, world, ms_total)
+
+    # ---- the tensor-core top level alone (GEMM + certificates) ----
+    cert = torch.full((T, Hq), -1, dtype=torch.int32, device=dev)
+    z.zha_prefill_top_scores(cfg, cache, q, 0, start, c.p, None, cert, ws, st)
+    torch.cuda.synchronize()
+    nr = 20
+    e0.record(stream)
+    for _ in range(nr):
+        z.zha_prefill_top_scores(cfg, cache, q, 0, start, c.p, None, cert, ws, st)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    top_ms = max_over_ranks(e0.elapsed_time(e1) / nr, dev)
+    n_top = min((start + T) // b ** L, c.capacity // b ** L)
+    gemm_flops = 2.0 * T * Hq * n_top * D
+    # algorithmic bytes: query rows, top summaries, the fp32 scores written by
+    # the GEMM and read by the certifier, and the per-unit seeds
+    top_bytes = (T * Hq * D * 2 + Hkv * n_top * D * 2 + 2 * T * Hq * n_top * 4
+                 + T * Hkv * (n_top + 4 + 4 * G))
+    cert_heads = float((cert == 1).float().mean())
+    cert_units = float((cert == 1).view(T, Hkv, G).all(-1).float().mean())
+
+    # ---- end to end with host buffers: the chunk's K/V rows and queries in,
+    # the outputs back, every step ----
+    ne = min(3, args.steps)
+    kv_host = torch.stack([wl.K[0, :, start:start + T], wl.V[0, :, start:start + T]]).cpu()
+    kv_host = kv_host.pin_memory()
+    q_host = q.cpu().pin_memory()
+    out_host = torch.empty_like(q_host).pin_memory()
+    kv_dev = torch.empty_like(kv_host, device=dev)
+    q_dev = torch.empty_like(q)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(ne):
+        kv_dev.copy_(kv_host, non_blocking=True)
+        q_dev.copy_(q_host, non_blocking=True)
+        wl.K[0, :, start:start + T] = kv_dev[0]
+        wl.V[0, :, start:start + T] = kv_dev[1]
+        cache.seq_len = len1
+        z.zha_prefill_chunk(cfg, cache, q_dev, 0, start, c.p, out, None, ws, st)
+        out_host.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / ne, dev)
+    h2d = kv_host.numel() * kv_host.element_size() + q_host.numel() * q_host.element_size()
+    d2h = out_host.numel() * out_host.element_size()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {z.status_string(int(st.item()))}")
+
+    peak, peak_kind = measured_peaks()
+    roof = {"kernel": "tensor-core top level: top_score_tc_kernel + top_certify_kernel "
+                      "(zha_prefill_top_scores)", "bound": "hbm",
+            "achieved": top_bytes / (top_ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+            "peak_kind": peak_kind, "traffic": None}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    tile = max(1, min(T, (2 * sms) // Hkv))
+    tiles = (T + tile - 1) // tile
+    # fill, tree levels, top level (norms, GEMM, certificates), then per query
+    # tile positions, traversal, attention and combine
+    launches = 1 + L + 3 + 4 * tiles
+    res = {
+        "metric": PREFILL_METRIC, "value": value, "unit": "queries/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Gaussian-mixture keys, planted needles; no dataset)",
+        "config": workload_config(args, c),
+        "tensor_core_top_level": {
+            "ms": top_ms, "top_nodes": n_top, "gemm_flops": gemm_flops,
+            "gemm_tflops_incl_certify": gemm_flops / (top_ms / 1e3) / 1e12,
+            "certified_head_fraction": cert_heads, "certified_unit_fraction": cert_units},
+        "roofline": roof,
+        "tree_build": {"ms": build_ms, "tokens": Hkv * start},
+        "e2e": {"value": queries_per_step * world / (e2e_ms / 1e3), "unit": "queries/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches * args.steps,
+        "clocks": clocks,
+    }
+    return res, wl
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -410,10 +598,26 @@ def main():
 
         dev = "cuda" if torch.cuda.is_available() else "cpu"
         wl = W.make(args.workload, device=dev, n_tokens=args.n_tokens)
-        n = args.steps + args.warmup
+        c = wl.cfg
+        if is_prefill(args.workload):
+            rate, done, el = oracle_prefill_rate(wl, args.steps, budget_s=600.0)
+            line = {"impl": "reference", "metric": PREFILL_METRIC, "value": rate,
+                    "unit": "queries/s", "n_gpus": 1, "steps": args.steps,
+                    "warmup": args.warmup,
+                    "ms_per_step": el / done * c.chunk * c.n_q_heads * 1e3,
+                    "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                    "dtype": "f32 select / f64 attention", "data": "synthetic",
+                    "config": workload_config(args, c),
+                    "cpu_baseline": {"value": rate, "unit": "queries/s", "cores": 1,
+                                     "kind": "oracle",
+                                     "sample": f"{done} chunk queries (query heads of KV head "
+                                               f"0) in {el:.1f} s, tree built untimed"},
+                    "e2e": {"value": rate, "unit": "queries/s", "h2d_bytes_per_step": 0,
+                            "d2h_bytes_per_step": 0}}
+            print(json.dumps(line), flush=True)
+            return
         oracle_rate(wl, min(args.warmup, 2), budget_s=60.0)  # warm-up
         rate, done, el = oracle_rate(wl, args.steps, budget_s=600.0)
-        c = wl.cfg
         line = {"impl": "reference", "metric": METRIC, "value": rate, "unit": "queries/s",
                 "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": el / done * c.batch * c.n_q_heads * 1e3,
@@ -433,9 +637,15 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    res, wl = run_zha(args, rank, world, dev)
+    prefill = is_prefill(args.workload)
+    res, wl = (run_prefill if prefill else run_zha)(args, rank, world, dev)
     if rank == 0:
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and prefill:
+            rate, done, el = oracle_prefill_rate(wl, 200, budget_s=20.0)
+            res["cpu_baseline"] = {"value": rate, "unit": "queries/s", "cores": 1, "kind": "oracle",
+                                   "sample": f"{done} chunk queries of KV head 0 over {el:.1f} s "
+                                             "(tree built untimed)"}
+        elif world == 1 and not args.no_cpu_baseline:
             rate, done, el = oracle_rate(wl, 200, budget_s=20.0)
             res["cpu_baseline"] = {"value": rate, "unit": "queries/s", "cores": 1, "kind": "oracle",
                                    "sample": f"{done} queries of sequence 0 / KV head 0 over "

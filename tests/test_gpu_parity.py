@@ -205,3 +205,33 @@ def test_zero_query_all_ties():
     q = torch.zeros_like(wl.queries(0))
     for p in (0.3, 0.95):
         _decode_parity(wl, q, p, c.n_tokens)
+
+
+def test_select_one_cta_narrowed_groups():
+    """148 queries (one CTA per (query, KV head) unit, as a prefill tile runs)
+    at 131K context, small-norm queries and p = 0.5 / 0.95: the crossing
+    first-pass buckets hold hundreds of candidates, so a head's group is
+    narrowed by key-digit passes before its owner gathers it, and the other
+    members of the bucket (above and below the group) keep or lose their place
+    by key. Index lists must equal the oracle's exactly."""
+    wl = W.make("decode-deep-32k", n_tokens=131072)
+    c = wl.cfg
+    gpu = Gpu(wl)
+    ref = Ref(wl, c.n_tokens)
+    nq = 148
+    g = torch.Generator().manual_seed(7)
+    q = (0.05 * torch.randn(nq, c.n_q_heads, c.head_dim, generator=g)).to(c.torch_dtype)
+    pos = [c.n_tokens - 1 - i for i in range(nq)]
+    qf = q.float().numpy()
+    for p in (0.5, 0.95):
+        idx, n_idx, lcs, _ = gpu.select(q.to(gpu.dev), [0] * nq, pos, p, c.n_tokens + 2)
+        n_idx = n_idx.cpu().numpy()
+        lcs = lcs.cpu().numpy()
+        for i in (0, 1, 73, 147):
+            rows = idx[i].cpu().numpy()
+            for h in range(c.n_q_heads):
+                e_idx, e_counts, _, _ = ref.select(qf[i, h], 0, h, pos[i], p)
+                assert lcs[i, h].tolist() == e_counts.tolist(), (p, i, h)
+                assert n_idx[i, h] == len(e_idx), (p, i, h, n_idx[i, h], len(e_idx))
+                assert np.array_equal(rows[h, :n_idx[i, h]], e_idx), (p, i, h)
+        del idx

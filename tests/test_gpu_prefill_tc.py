@@ -169,3 +169,58 @@ def test_top_scores_unsupported_geometry():
     ws = z.alloc_workspace(gpu.cfg, z.ZHA_OP_PREFILL, 4, device=gpu.dev)
     with pytest.raises(z.ZhaError):
         z.zha_prefill_top_scores(gpu.cfg, gpu.cache, q, 0, 0, 0.95, None, None, ws, gpu.status)
+
+
+@pytest.mark.slow
+def test_prefill_full_size_sampled():
+    """The full chunked-prefill workload (a 4096-token chunk after 1,048,576
+    tokens, b = 4, L = 6, 257 top nodes for the last token), called as the
+    benchmark calls it: zha_prefill_chunk over the whole chunk. Sampled
+    (token, head) level counts and outputs against the oracle; exact index
+    lists of sampled tokens through zha_select, both with one token (a cluster
+    of CTAs per unit) and with a full 148-token tile (one CTA per unit, the
+    prefill configuration); then the tensor-core scores and certificates of
+    the whole chunk."""
+    wl = W.make("prefill-deep-1m-chunk4k")
+    c = wl.cfg
+    gpu = Gpu(wl)  # tree over the cached context
+    start = c.n_tokens
+    gpu.cache.seq_len.fill_(start + c.chunk)
+    q = wl.queries(0).to(gpu.dev)
+    out = torch.empty_like(q)
+    lc = torch.full((c.chunk, c.n_q_heads, c.levels), -1, dtype=torch.int32, device=gpu.dev)
+    ws = z.alloc_workspace(gpu.cfg, z.ZHA_OP_PREFILL, c.chunk, device=gpu.dev)
+    z.zha_prefill_chunk(gpu.cfg, gpu.cache, q, 0, start, c.p, out, lc, ws, gpu.status)
+    gpu.check_status()
+    ref = Ref(wl, start + c.chunk)
+    for kvh in range(c.n_kv_heads):
+        compare_tree(gpu, ref, 0, kvh)  # the chunk's nodes, extended in place
+    outn = out.float().cpu().numpy()
+    lcn = lc.cpu().numpy()
+    qf = q.float().cpu().numpy()
+    expect = {}
+
+    def oracle_sel(i, h):
+        if (i, h) not in expect:
+            expect[(i, h)] = ref.select(qf[i, h], 0, h, start + i, c.p)
+        return expect[(i, h)]
+
+    for i in (0, 2047, c.chunk - 1):
+        for h in range(c.n_q_heads):
+            e_idx, e_counts, _, _ = oracle_sel(i, h)
+            assert lcn[i, h].tolist() == e_counts.tolist(), (i, h)
+            o = ref.attend(qf[i, h], 0, h, e_idx)
+            assert np.abs(outn[i, h] - o).max() < TOL["bf16"], (i, h)
+    for nq, toks in ((1, (0,)), (148, (0, 77, 147))):
+        idx, n_idx, lcs, _ = gpu.select(q[:nq].contiguous(), [0] * nq,
+                                        [start + i for i in range(nq)], c.p, start + c.chunk + 2)
+        n_idx = n_idx.cpu().numpy()
+        for i in toks:
+            rows = idx[i].cpu().numpy()
+            for h in range(c.n_q_heads):
+                e_idx, _, _, _ = oracle_sel(i, h)
+                assert n_idx[i, h] == len(e_idx), (nq, i, h, n_idx[i, h], len(e_idx))
+                assert np.array_equal(rows[h, :n_idx[i, h]], e_idx), (nq, i, h)
+        del idx
+        torch.cuda.empty_cache()
+    _check_top_scores(wl, gpu, ref, start, [0, 4095], 0.5)

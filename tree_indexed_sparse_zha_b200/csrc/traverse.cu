@@ -68,8 +68,9 @@ enum HeadMode : int {
   kModeThr = 2,       // keep iff key >= kthr
   kModeTie = 3,       // keep iff key > kthr, or key == kthr within the segment's quota
   kModeQuant = 4,     // first pass pending: buckets are a linear map of z
-  kModeGathered = 5,  // keep iff first-pass bucket > qbeta, or == qbeta and the
-                      // owner marked the candidate kept
+  kModeGathered = 5,  // keep iff first-pass bucket > qbeta, or == qbeta and either
+                      // key > kgmax or key in [kgmin, kgmax] and the owner marked
+                      // the candidate kept
 };
 
 struct TravParams {
@@ -126,8 +127,9 @@ struct HeadState {
   unsigned int kthr;         // threshold key of the final rule
   unsigned int count;        // kept candidates (the level count)
   unsigned int qbeta;        // first-pass bucket of the group (0xffffffff: none)
-  int zfree;                 // kModeThr / kModeTie decided on the first pass: every
-                             // candidate's fate follows from its bucket alone
+  int zfree;                 // the final rule was set while the group was still the
+                             // whole first-pass bucket: every candidate's fate follows
+                             // from its bucket (and, kModeGathered, its mark) alone
   unsigned int quota[kMaxCluster];  // kModeTie: kept members of each segment
 };
 
@@ -1446,14 +1448,17 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
     }
     __syncthreads();
     // the rules as byte-parallel masks (bit h = head h)
-    uint32_t allm = 0, gathm = 0, thrz = 0, tiez = 0, needz = 0;
+    // A gathered group narrowed by radix passes (gathn) is a key sub-interval
+    // of its first-pass bucket: bucket members above it are kept, below it
+    // dropped, and only members inside it carry the owner's mark.
+    uint32_t allm = 0, gathz = 0, gathn = 0, thrz = 0, tiez = 0, needz = 0;
     uint64_t qb_pack = 0;
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       const HeadState& st = S.st[h];
       const uint32_t bit = 1u << h;
       if (st.mode == kModeAll) allm |= bit;
-      else if (st.mode == kModeGathered) gathm |= bit;
+      else if (st.mode == kModeGathered) (st.zfree ? gathz : gathn) |= bit;
       else if (st.mode == kModeThr) (st.zfree ? thrz : needz) |= bit;
       else if (st.mode == kModeTie) (st.zfree ? tiez : needz) |= bit;
       qb_pack |= (uint64_t)(st.qbeta & 0xffu) << (8 * h);
@@ -1467,7 +1472,7 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
       constexpr int kEU = 4;  // consecutive candidates per thread
       for (int64_t base = 0; base < my_n; base += kEU * kThreads) {
         const int64_t i0 = base + kEU * tid;
-        uint32_t km[kEU], cv[kEU], ties[kEU];
+        uint32_t km[kEU], cv[kEU], ties[kEU], eqm[kEU];
         uint64_t qrow[kEU], mrow[kEU];
 #pragma unroll
         for (int u = 0; u < kEU; ++u) {
@@ -1485,23 +1490,28 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
         for (int u = 0; u < kEU; ++u) {
           const uint32_t hm = cv[u] >> 24;
           const uint32_t gt = bytes_gt(qrow[u], qb_pack), eq = bytes_eq(qrow[u], qb_pack);
-          km[u] = hm & (allm | (gt & ~allm) | (eq & gathm & bytes_nz(mrow[u])) | (eq & thrz));
+          km[u] = hm & (allm | (gt & ~allm) | (eq & gathz & bytes_nz(mrow[u])) | (eq & thrz));
           ties[u] = hm & eq & tiez;
+          eqm[u] = hm & eq & (needz | gathn);
         }
-        if (needz) {  // rules narrowed below the first-pass bucket: compare scores
+        if (needz | gathn) {  // rules narrowed below the first-pass bucket: compare scores
 #pragma unroll
           for (int u = 0; u < kEU; ++u) {
-            if (i0 + u >= my_n) continue;
+            if (!eqm[u]) continue;  // (also every candidate past the segment's end)
             float z[G];
             load_scores<G>(zown, i0 + u, z);
-            const uint32_t hm = cv[u] >> 24;
 #pragma unroll
             for (int h = 0; h < G; ++h) {
               const HeadState& st = S.st[h];
-              if (!(((hm & needz) >> h) & 1u)) continue;
-              if ((uint32_t)((qrow[u] >> (8 * h)) & 0xffu) != st.qbeta) continue;
+              if (!((eqm[u] >> h) & 1u)) continue;
+              const uint32_t key = order_key(z[h]);
+              if ((gathn >> h) & 1u) {
+                if (key > st.kgmax || (key >= st.kgmin && ((mrow[u] >> (8 * h)) & 0xffu)))
+                  km[u] |= 1u << h;
+                continue;
+              }
               bool member;
-              if (keep_rule(st.mode, st.kthr, order_key(z[h]), &member)) km[u] |= 1u << h;
+              if (keep_rule(st.mode, st.kthr, key, &member)) km[u] |= 1u << h;
               if (member) ties[u] |= 1u << h;
             }
           }
