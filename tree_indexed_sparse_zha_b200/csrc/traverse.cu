@@ -1648,8 +1648,14 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
 }
 
 // Dynamic shared memory of a CTA: the struct plus its shipped-member lists.
+// A cluster's owners gather up to kGather members per owned head; a CTA
+// working alone (C = 1, or rank 0 on the small top levels) owns every head
+// with up to kWarpGather members each. Sizing C = 1 for the latter keeps two
+// CTAs per SM.
 size_t smem_bytes(int G, int C) {
-  return sizeof(Smem) + (size_t)list_slots(G, C) * kGather * (sizeof(float) + sizeof(uint32_t));
+  const size_t entries = C > 1 ? (size_t)list_slots(G, C) * kGather : 0;
+  const size_t alone = (size_t)list_slots(G, 1) * kWarpGather;
+  return sizeof(Smem) + (entries > alone ? entries : alone) * (sizeof(float) + sizeof(uint32_t));
 }
 
 template <typename T, int D, int G>
