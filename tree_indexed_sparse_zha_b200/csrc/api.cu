@@ -114,7 +114,7 @@ static int64_t prefill_tile(const Geometry& g, int64_t T, int sms) {
 }
 
 struct PrefillLayout {
-  size_t old_len, q_seq, q_pos, dec, top, top_bytes, total;
+  size_t old_len, q_seq, q_pos, dec, top, top_bytes, tatt, tatt_bytes, total;
   int64_t tile;
   DecodeLayout d;
 };
@@ -136,6 +136,10 @@ static PrefillLayout prefill_layout(const Geometry& g, int64_t T, int sms) {
   P.top = off;
   P.top_bytes = top_tc_ws_bytes(g, T);
   off = align256(off + P.top_bytes);
+  // tile attention (keep map and split partials of one query tile)
+  P.tatt = off;
+  P.tatt_bytes = tile_attend_ws_bytes(g, P.tile, sms);
+  off = align256(off + P.tatt_bytes);
   P.total = off;
   return P;
 }
@@ -461,10 +465,21 @@ zha_status zha_prefill_chunk(const zha_config* cfg, const zha_cache* cache, cons
       ts.cnt = seeds.cnt + i0 * g.Hkv * g.G;
       ts.stride = seeds.stride;
     }
-    st = run_tree_decode(g, cache, static_cast<const unsigned char*>(q) + i0 * row_bytes, q_seq,
-                         q_pos, n, p_q, static_cast<unsigned char*>(out) + i0 * row_bytes,
+    const unsigned char* q_tile = static_cast<const unsigned char*>(q) + i0 * row_bytes;
+    unsigned char* out_tile = static_cast<unsigned char*>(out) + i0 * row_bytes;
+    st = run_tree_select(g, cache, q_tile, q_seq, q_pos, n, p_q,
                          level_counts ? level_counts + i0 * g.Hq * g.L : nullptr, w + P.dec, L,
                          dev_status, sms, s, tc ? &ts : nullptr);
+    if (st != ZHA_OK) return st;
+    if (P.tatt_bytes > 0) {  // the tile's tokens share K/V blocks on tensor cores
+      st = cuda_status(launch_attend_tile(
+          g, cache->k, cache->v, cache->seq_len, seq, chunk_start + i0, n, q_tile, out_tile,
+          reinterpret_cast<const uint32_t*>(w + P.dec + L.kept),
+          reinterpret_cast<const int32_t*>(w + P.dec + L.n_kept), traverse_kept_stride(g),
+          traverse_cluster_size(g, L.units, sms), w + P.tatt, P.tatt_bytes, sms, s));
+    } else {
+      st = run_tree_attend(g, cache, q_tile, q_seq, q_pos, n, out_tile, w + P.dec, L, sms, s);
+    }
     if (st != ZHA_OK) return st;
   }
   return ZHA_OK;

@@ -121,6 +121,19 @@ size_t attend_ws_bytes(const Geometry& g, int kind, int64_t nq, int num_sms);
 cudaError_t launch_attend(const Geometry& g, const AttendArgs& a, void* ws, size_t ws_bytes,
                           int num_sms, cudaStream_t stream);
 
+// Prefill attention of a tile of n consecutive query tokens of sequence `seq`
+// (positions pos0 ..): all tokens' rows of a KV head share each K/V block on
+// tensor cores, masked by the traversal's kept level-1 lists (decode-mode
+// output of launch_traverse for the same tile).
+bool tile_attend_supported(const Geometry& g);
+int64_t tile_map_stride(const Geometry& g);
+size_t tile_attend_ws_bytes(const Geometry& g, int64_t n, int num_sms);
+cudaError_t launch_attend_tile(const Geometry& g, const void* k, const void* v,
+                               const int32_t* seq_len, int seq, int64_t pos0, int64_t n,
+                               const void* q, void* out, const uint32_t* kept,
+                               const int32_t* n_kept, int64_t kept_stride, int kept_segs,
+                               void* ws, size_t ws_bytes, int num_sms, cudaStream_t stream);
+
 int device_sm_count();
 
 }  // namespace zha
