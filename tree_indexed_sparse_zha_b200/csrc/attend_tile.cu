@@ -144,6 +144,14 @@ __global__ void __launch_bounds__(kTThreads, 1) attend_tile_kernel(TileParams p)
     tpos[k] = valid[k] ? t : -1;
     tstart[k] = p.span_L * ((tpos[k] + 1) / p.span_L);
   }
+  // the lowest tail start among the CTA's tokens (keys below it are decided by
+  // the keep map alone, except key 0)
+  int64_t tail_min;
+  {
+    int64_t t = p.pos0 + tok0;
+    if (t > nseq - 1) t = nseq - 1;
+    tail_min = ntok > 0 && t >= 0 ? p.span_L * ((t + 1) / p.span_L) : 0;
+  }
   // Q fragments of rows g (a0, a2) and g + 8 (a1, a3), exact bf16 inputs
   uint32_t qa[kTD / 16][4];
   {
@@ -226,20 +234,26 @@ __global__ void __launch_bounds__(kTThreads, 1) attend_tile_kernel(TileParams p)
       }
     }
     // ---- selection mask, scale, online softmax (rows g and g + 8) ----
+    // A thread's keys 2 t4 and 2 t4 + 1 of n-tile nt share one node (b >= 2):
+    // one keep byte per (row, n-tile). Blocks past key 0 and below every
+    // token's tail need nothing else; the others also test positions,
+    // relative to the block start.
     const int64_t k0 = kb * kTKB;
+    const bool plain = k0 > 0 && k0 + kTKB <= tail_min;
     float mb[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-    for (int nt = 0; nt < kTKB / 8; ++nt) {
+    for (int k = 0; k < 2; ++k) {
+      const uint8_t* mrow = mk + tl[k] * (kTKB / 2);
+      const int lim = (int)(tpos[k] - k0 < kTKB ? tpos[k] - k0 : kTKB);      // last key <= t
+      const int tst = (int)(tstart[k] - k0 < kTKB ? tstart[k] - k0 : kTKB);  // first tail key
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int kk = nt * 8 + 2 * t4 + j;
-        const int64_t key = k0 + kk;
-        const int nb = kk >> p.b_shift;
+      for (int nt = 0; nt < kTKB / 8; ++nt) {
+        const bool keep = (mrow[(nt * 8 + 2 * t4) >> p.b_shift] >> hh[k]) & 1u;
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const bool ok = key <= tpos[k] &&
-                          (key == 0 || key >= tstart[k] ||
-                           ((mk[tl[k] * (kTKB / 2) + nb] >> hh[k]) & 1u));
+        for (int j = 0; j < 2; ++j) {
+          const int kk = nt * 8 + 2 * t4 + j;
+          const bool ok = plain ? keep
+                                : kk <= lim && (keep || kk >= tst || (k0 == 0 && kk == 0));
           const float s = ok ? sc[nt][2 * k + j] * p.qscale : -INFINITY;
           sc[nt][2 * k + j] = s;
           mb[k] = fmaxf(mb[k], s);
