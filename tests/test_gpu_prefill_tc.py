@@ -224,3 +224,48 @@ def test_prefill_full_size_sampled():
         del idx
         torch.cuda.empty_cache()
     _check_top_scores(wl, gpu, ref, start, [0, 4095], 0.5)
+
+
+PREFILL_GEOMETRIES = [
+    # (context, chunk, block, levels, q heads, KV heads, head_dim, dtype)
+    (20000, 200, 8, 4, 8, 2, 128, "bf16"),     # G = 4, 8 keep bytes per 64-key block
+    (5000, 100, 2, 8, 16, 8, 128, "bf16"),     # G = 2, 32 keep bytes per block
+    (12000, 64, 16, 3, 16, 2, 128, "bf16"),    # b = 16: 4 keep bytes per block
+    (64, 200, 4, 3, 16, 2, 128, "bf16"),       # early tokens: 1 complete top node, then more
+    (9000, 80, 4, 4, 16, 2, 64, "bf16"),       # d = 64: gather attention, canonical top level
+    (3000, 60, 4, 3, 4, 1, 64, "f32"),         # fp32: gather attention, canonical top level
+]
+
+
+@pytest.mark.parametrize("geom", PREFILL_GEOMETRIES, ids=lambda g: "-".join(map(str, g)))
+def test_prefill_geometries(geom):
+    """zha_prefill_chunk on geometries off the benchmark's: other block sizes
+    and group sizes take other template instances of the tile attention and
+    certificate kernels; d = 64 and fp32 take the gather attention and the
+    canonical top level. Every (token, head) is checked against the oracle."""
+    n, chunk, b, L, hq, hkv, d, dt = geom
+    base = W.CONFIGS["prefill-deep-1m-chunk4k"]
+    wl = W.Workload(base.scaled(n, chunk=chunk, block=b, levels=L, n_q_heads=hq, n_kv_heads=hkv,
+                                head_dim=d, dtype=dt))
+    c = wl.cfg
+    gpu = Gpu(wl)
+    start = c.n_tokens
+    gpu.cache.seq_len.fill_(start + c.chunk)
+    q = wl.queries(0).to(gpu.dev)
+    out = torch.empty_like(q)
+    lc = torch.full((c.chunk, c.n_q_heads, c.levels), -1, dtype=torch.int32, device=gpu.dev)
+    ws = z.alloc_workspace(gpu.cfg, z.ZHA_OP_PREFILL, c.chunk, device=gpu.dev)
+    z.zha_prefill_chunk(gpu.cfg, gpu.cache, q, 0, start, c.p, out, lc, ws, gpu.status)
+    gpu.check_status()
+    ref = Ref(wl, start + c.chunk)
+    for kvh in range(c.n_kv_heads):
+        compare_tree(gpu, ref, 0, kvh)
+    out = out.float().cpu().numpy()
+    lc = lc.cpu().numpy()
+    qf = q.float().cpu().numpy()
+    for i in range(c.chunk):
+        for h in range(c.n_q_heads):
+            e_idx, e_counts, _, _ = ref.select(qf[i, h], 0, h, start + i, c.p)
+            assert lc[i, h].tolist() == e_counts.tolist(), (i, h)
+            o = ref.attend(qf[i, h], 0, h, e_idx)
+            assert np.abs(out[i, h] - o).max() < TOL[c.dtype], (i, h, np.abs(out[i, h] - o).max())
