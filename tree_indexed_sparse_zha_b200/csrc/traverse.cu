@@ -108,6 +108,11 @@ struct TravParams {
   const uint8_t* seed_mask;  // [units][seed_stride] bit h: head h keeps top node i
   const int32_t* seed_cnt;   // [units][G]
   int64_t seed_stride;
+  // one CTA per unit (C = 1): shipped-member lists of kGather entries per
+  // head in global memory (shared memory holds two CTAs per SM only with
+  // kWarpGather-entry lists)
+  float* glist_z;            // [units][G][kGather]
+  uint32_t* glist_pos;       // [units][G][kGather]
 };
 
 // Cut state of one head. After every publish step it is identical on all CTAs
@@ -683,24 +688,24 @@ __device__ __noinline__ void owner_pass(const TravParams& p, Smem& S, cg::cluste
 }
 
 // Owner step for a head whose group (at most kGather members) has been
-// shipped to this CTA's list S.mz/S.mpos[slot]: sorts the members by
+// shipped to the lists mz/mpos (listed entries): sorts the members by
 // (z desc, position asc) (bitonic network on (key << 32 | ~position)), finds
 // the shortest prefix whose mass reaches what the group must still cover,
 // marks every member's fate in mkbuf (the keep byte of (segment, index, head))
 // and publishes kModeGathered in S.pub[h].
 template <int G>
-__device__ __noinline__ void owner_finish(const TravParams& p, Smem& S, int h, int slot,
-                                          int slots, int cap, uint8_t* mk_u, int64_t seg) {
+__device__ __noinline__ void owner_finish(const TravParams& p, Smem& S, int h, const float* mz,
+                                          const uint32_t* mpos, unsigned listed, int cap,
+                                          uint8_t* mk_u, int64_t seg) {
   static_assert(kGather == 2 * kThreads, "two sort slots per thread");
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const HeadState s0 = S.st[h];
-  const int n = (int)(S.mlist_n[slot] < (unsigned)cap ? S.mlist_n[slot] : cap);
+  const int n = (int)(listed < (unsigned)cap ? listed : cap);
   int np2 = 2;
   while (np2 < n) np2 <<= 1;
   unsigned long long* key = S.mrank_m;  // sort keys, descending
   for (int i = tid; i < np2; i += kThreads)
-    key[i] = i < n ? ((unsigned long long)order_key(list_z(S)[slot * cap + i]) << 32) |
-                         (0xffffffffu - list_pos(S, slots, cap)[slot * cap + i])
+    key[i] = i < n ? ((unsigned long long)order_key(mz[i]) << 32) | (0xffffffffu - mpos[i])
                    : 0ull;
   __syncthreads();
   for (int k = 2; k <= np2; k <<= 1) {
@@ -1197,7 +1202,17 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
     __syncthreads();
     // entries per shipped-member list (rank 0 alone: one list per head, each
     // finished by one warp)
-    const int cap = Ce > 1 ? kGather : kWarpGather;
+    // one CTA per unit keeps kGather-entry lists in global memory; rank 0
+    // alone in a cluster keeps kWarpGather-entry lists in shared memory
+    const bool glob = C == 1 && p.glist_z != nullptr;
+    const int cap = (Ce > 1 || glob) ? kGather : kWarpGather;
+    auto list_zh = [&](Smem* O, int h) -> float* {
+      return glob ? p.glist_z + ((int64_t)unit * G + h) * kGather : list_z(*O) + (h / Ce) * cap;
+    };
+    auto list_ph = [&](Smem* O, int h) -> uint32_t* {
+      return glob ? p.glist_pos + ((int64_t)unit * G + h) * kGather
+                  : list_pos(*O, list_slots(G, Ce), cap) + (h / Ce) * cap;
+    };
     for (int pass = 0; pass < 40; ++pass) {  // every pass strictly narrows each group
       // heads whose group is still open: histogram pass, or (small group)
       // shipped to the owner who finishes the cut alone
@@ -1357,8 +1372,8 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
                   Smem* O = cluster.map_shared_rank(&S, h % Ce);
                   const unsigned ko = atomicAdd(&O->mlist_n[h / Ce], 1u);
                   if (ko < (unsigned)cap) {
-                    list_z(*O)[(h / Ce) * cap + ko] = z_c[u][h];
-                    list_pos(*O, list_slots(G, Ce), cap)[(h / Ce) * cap + ko] = tag & 0x0fffffffu;
+                    list_zh(O, h)[ko] = z_c[u][h];
+                    list_ph(O, h)[ko] = tag & 0x0fffffffu;
                   }
                 }
                 ++k;
@@ -1382,8 +1397,8 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
             unsigned base = 0;
             if (lane == 0) base = atomicAdd(&O->mlist_n[h / Ce], cnt);
             base = __shfl_sync(0xffffffffu, base, 0);
-            float* oz = list_z(*O) + (h / Ce) * cap;
-            uint32_t* op = list_pos(*O, list_slots(G, Ce), cap) + (h / Ce) * cap;
+            float* oz = list_zh(O, h);
+            uint32_t* op = list_ph(O, h);
             for (unsigned e0 = 0; e0 < n_st; e0 += 32) {
               const unsigned e = e0 + lane;
               const unsigned long long v = e < n_st ? S.mrank_m[e] : 0ull;
@@ -1407,8 +1422,16 @@ __global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
         for (int h = rank; h < G; h += Ce) {
           if ((hist_heads >> h) & 1u) owner_pass<G>(p, S, cluster, Ce, h);
           else if ((gather_heads >> h) & 1u)
-            owner_finish<G>(p, S, h, h / Ce, list_slots(G, Ce), cap, mk_u, seg);
+            owner_finish<G>(p, S, h, list_zh(&S, h), list_ph(&S, h), S.mlist_n[h / Ce], cap,
+                            mk_u, seg);
         }
+      } else if (glob) {
+        // the whole CTA sorts each gathered head's group in turn; one warp
+        // per head narrows the others
+        for (int h = 0; h < G; ++h)
+          if ((gather_heads >> h) & 1u)
+            owner_finish<G>(p, S, h, list_zh(&S, h), list_ph(&S, h), S.mlist_n[h], cap, mk_u, seg);
+        if (warp < G && ((hist_heads >> warp) & 1u)) owner_pass_warp<G>(p, S, warp);
       } else if (warp < G) {  // one warp per head
         if ((hist_heads >> warp) & 1u) owner_pass_warp<G>(p, S, warp);
         else if ((gather_heads >> warp) & 1u)
@@ -1769,9 +1792,11 @@ int traverse_cluster_size(const Geometry& g, int64_t units, int num_sms) {
 size_t traverse_ws_bytes(const Geometry& g, int64_t units, int num_sms) {
   const int C = traverse_cluster_size(g, units, num_sms);
   const size_t seg = (size_t)seg_capacity(g);
-  // candidates (two buffers), scores, first-pass buckets and owner marks
+  // candidates (two buffers), scores, first-pass buckets and owner marks,
+  // plus the global member lists of one-CTA units
   const size_t per = (size_t)C * seg * (2 * sizeof(uint32_t) + (size_t)g.G * (sizeof(float) + 2));
-  return per * (size_t)units + 256;
+  const size_t lists = C == 1 ? (size_t)g.G * kGather * (sizeof(float) + sizeof(uint32_t)) : 0;
+  return (per + lists) * (size_t)units + 512;
 }
 
 size_t traverse_kept_bytes(const Geometry& g, int64_t units, int num_sms) {
@@ -1821,6 +1846,13 @@ cudaError_t launch_traverse(const Geometry& g, const void* tree, const void* q,
   p.qbuf = reinterpret_cast<uint8_t*>(w);
   w += (size_t)units * C * p.seg * g.G;
   p.mkbuf = reinterpret_cast<uint8_t*>(w);
+  w += (size_t)units * C * p.seg * g.G;
+  if (C == 1) {
+    w = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(w) + 255) & ~(uintptr_t)255);
+    p.glist_z = reinterpret_cast<float*>(w);
+    w += sizeof(float) * (size_t)units * g.G * kGather;
+    p.glist_pos = reinterpret_cast<uint32_t*>(w);
+  }
   if (!list_mode) {
     if (!out.kept || !out.n_kept) return cudaErrorInvalidValue;
     p.kept = out.kept;
