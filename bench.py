@@ -231,20 +231,27 @@ def throughput(queries_per_step: int, steps: int, world: int, ms_total_max: floa
     return queries_per_step * steps * world / (ms_total_max / 1e3)
 
 
+L2_BYTES = 126e6
+
+
+def l2_note(kv_gb: float) -> str:
+    if kv_gb * 1e9 > L2_BYTES:
+        return f"inputs larger than L2 (K+V {kv_gb:.2f} GB), no flush"
+    return f"inputs fit in L2 (K+V {kv_gb:.3f} GB): a small diagnostic case, not a bench number"
+
+
 def workload_config(args, c):
     if is_prefill(args.workload):
         kv_gb = 2 * c.n_kv_heads * c.capacity * c.head_dim * 2 / 1e9
         return {"workload": args.workload, "batch": c.batch, "context": c.n_tokens,
                 "chunk": c.chunk, "heads": f"{c.n_q_heads}q/{c.n_kv_heads}kv",
                 "head_dim": c.head_dim, "tree": f"b={c.block},L={c.levels}", "p": c.p,
-                "queries_per_step": c.chunk * c.n_q_heads,
-                "l2": f"inputs larger than L2 (K+V {kv_gb:.2f} GB), no flush"}
+                "queries_per_step": c.chunk * c.n_q_heads, "l2": l2_note(kv_gb)}
     kv_gb = 2 * c.batch * c.n_kv_heads * c.n_tokens * c.head_dim * (2 if c.dtype == "bf16" else 4) / 1e9
     return {"workload": args.workload, "batch": c.batch, "context": c.n_tokens,
             "heads": f"{c.n_q_heads}q/{c.n_kv_heads}kv", "head_dim": c.head_dim,
             "tree": f"b={c.block},L={c.levels}", "p": c.p,
-            "queries_per_step": c.batch * c.n_q_heads,
-            "l2": f"inputs larger than L2 (K+V {kv_gb:.2f} GB), no flush"}
+            "queries_per_step": c.batch * c.n_q_heads, "l2": l2_note(kv_gb)}
 
 
 def run_zha(args, rank, world, dev):
