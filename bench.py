@@ -53,6 +53,9 @@ def parse():
     ap.add_argument("--n-tokens", type=int, default=None,
                     help="context length override (profiling captures on a smaller case); "
                          "the reported workload is the full one only without it")
+    ap.add_argument("--sweep", action="store_true",
+                    help="tree-geometry sweep of the decode workload (one JSON line per "
+                         "geometry): selectivity and queries/s against the dense kernel")
     return ap.parse_args()
 
 
@@ -593,6 +596,83 @@ def run_prefill(args, rank, world, dev):
     return res, wl
 
 
+# tree geometries of the sweep: b^L in [256, 16384], at most 8 levels
+SWEEP_GEOMETRIES = [(2, 8), (4, 4), (4, 5), (4, 6), (4, 7), (8, 3), (8, 4), (16, 2), (16, 3),
+                    (64, 2), (256, 1)]
+
+
+def run_sweep(args, dev):
+    """Decode steps (select + attend, cache fixed) of the 256K B = 8 workload
+    for each tree geometry, beside the dense kernel on the same cache."""
+    import tree_indexed_sparse_zha_b200 as z
+    from tree_indexed_sparse_zha_b200 import workloads as W
+
+    z.lib()
+    peak, peak_kind = measured_peaks()
+    base = W.CONFIGS[WORKLOAD]
+    n_tok = args.n_tokens or base.n_tokens
+    wl = W.make(WORKLOAD, device=dev, n_tokens=n_tok, steps=0)
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+    steps = min(args.steps, 50)
+    queries = [wl.queries(s) for s in range(1, steps + 1)]
+    for b, L in SWEEP_GEOMETRIES:
+        c = wl.cfg
+        cfg = z.make_config(c.head_dim, b, L, c.n_q_heads, c.n_kv_heads, c.batch, c.capacity,
+                            c.torch_dtype)
+        cache = z.Cache(wl.K, wl.V, wl.R.float().contiguous(), z.alloc_tree(cfg, dev),
+                        wl.seq_len.clone())
+        z.zha_build_tree(cfg, cache)
+        ws = z.alloc_workspace(cfg, z.ZHA_OP_DECODE, device=dev)
+        wsd = z.alloc_workspace(cfg, z.ZHA_OP_DENSE, device=dev)
+        st = torch.zeros(1, dtype=torch.int32, device=dev)
+        out = torch.empty_like(queries[0])
+        for i in range(args.warmup):
+            z.zha_decode(cfg, cache, queries[i % steps], c.p, out, None, ws, st)
+        torch.cuda.synchronize()
+        if int(st.item()) != 0:
+            raise RuntimeError(f"b={b} L={L}: {z.status_string(int(st.item()))}")
+        e0.record(stream)
+        for i in range(steps):
+            z.zha_decode(cfg, cache, queries[i], c.p, out, None, ws, st)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        stats = torch.zeros(c.batch * c.n_kv_heads, L + 1, dtype=torch.int32, device=dev)
+        z.zha_decode_stats(cfg, ws, stats)
+        z.zha_dense_decode(cfg, cache, queries[0], out, wsd)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i in range(steps):
+            z.zha_dense_decode(cfg, cache, queries[i], out, wsd)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        dense_ms = e0.elapsed_time(e1) / steps
+        stats = stats.cpu()
+        units = c.batch * c.n_kv_heads
+        row = c.head_dim * 2
+        top = n_tok // b ** L
+        tail = n_tok - b ** L * top
+        kept = int(stats[:, L].sum())
+        kv_rows = kept * b + units * (1 + tail)
+        # as the main bench: summary rows, kept-node indices read by both
+        # halves, selected K+V rows, and the query rows in and out of each half
+        touched = (int(stats[:, :L].sum()) * row + 2 * kept * 4 + kv_rows * 2 * row
+                   + 4 * c.batch * c.n_q_heads * row)
+        q = c.batch * c.n_q_heads
+        line = {"sweep": WORKLOAD, "block": b, "levels": L, "top_span": b ** L,
+                "context": n_tok, "p": c.p, "steps": steps,
+                "ms_per_step": ms, "queries_per_s": q / (ms / 1e3),
+                "dense_ms_per_step": dense_ms, "dense_queries_per_s": q / (dense_ms / 1e3),
+                "kv_fraction_read": kv_rows / (units * n_tok),
+                "summary_rows_scored": int(stats[:, :L].sum()),
+                "bytes_touched_per_step": touched,
+                "hbm_frac": touched / (ms / 1e3) / 1e9 / peak, "peak_kind": peak_kind}
+        print(json.dumps(line), flush=True)
+        del cache, ws, wsd
+        torch.cuda.empty_cache()
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -639,6 +719,12 @@ def main():
                 "e2e": {"value": rate, "unit": "queries/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
+        return
+    if args.sweep:
+        dev = torch.device("cuda", local)
+        torch.cuda.set_device(dev)
+        if rank == 0:
+            run_sweep(args, dev)
         return
     if world > 1:
         torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
