@@ -284,12 +284,16 @@ __global__ void __launch_bounds__(kTThreads, 1) attend_tile_kernel(TileParams p)
     }
 #pragma unroll
     for (int k = 0; k < 2; ++k) l_part[k] = l_part[k] * alpha[k] + lsum[k];
+    // the accumulators need rescaling only after a row's maximum moved (rare
+    // once a few blocks are in); multiplying by exactly 1 changes nothing
+    if (!__all_sync(0xffffffffu, alpha[0] == 1.0f && alpha[1] == 1.0f)) {
 #pragma unroll
-    for (int nt = 0; nt < kTD / 8; ++nt) {
-      o[nt][0] *= alpha[0];
-      o[nt][1] *= alpha[0];
-      o[nt][2] *= alpha[1];
-      o[nt][3] *= alpha[1];
+      for (int nt = 0; nt < kTD / 8; ++nt) {
+        o[nt][0] *= alpha[0];
+        o[nt][1] *= alpha[0];
+        o[nt][2] *= alpha[1];
+        o[nt][3] *= alpha[1];
+      }
     }
     // ---- O += P V: 4 k-steps of 16 keys x 16 n-tiles of 8 dims ----
 #pragma unroll
