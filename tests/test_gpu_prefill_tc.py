@@ -234,6 +234,8 @@ PREFILL_GEOMETRIES = [
     (64, 200, 4, 3, 16, 2, 128, "bf16"),       # early tokens: 1 complete top node, then more
     (9000, 80, 4, 4, 16, 2, 64, "bf16"),       # d = 64: gather attention, canonical top level
     (3000, 60, 4, 3, 4, 1, 64, "f32"),         # fp32: gather attention, canonical top level
+    (2, 100, 4, 3, 16, 2, 128, "bf16"),        # no complete top node for the first tokens
+    (5000, 1, 4, 3, 16, 2, 128, "bf16"),       # one token: clusters of CTAs, 16 kept segments
 ]
 
 
