@@ -85,6 +85,24 @@ struct Span {
   const int32_t* list;
 };
 
+// Exclusive prefix of the unit's kept-segment sizes into segbase[0 .. segs]
+// (called by one full warp): every lane loads one size at once, so the CTA
+// does not wait for the sizes one after another.
+__device__ __forceinline__ void seg_prefix(const AttParams& p, int unit, int64_t T_top,
+                                           unsigned int* segbase) {
+  const int lane = threadIdx.x & 31;
+  unsigned int v = (lane < p.kept_segs && T_top > 0)
+                       ? (unsigned int)p.n_kept[(int64_t)unit * p.kept_segs + lane]
+                       : 0u;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const unsigned int y = __shfl_up_sync(0xffffffffu, v, off);
+    if (lane >= off) v += y;
+  }
+  if (lane < p.kept_segs) segbase[lane + 1] = v;
+  if (lane == 0) segbase[0] = 0u;
+}
+
 // Row of virtual index v in the CTA share, with its head mask (0 = skip).
 __device__ __forceinline__ void row_of(const AttParams& p, const Span& s, int64_t v,
                                        int64_t* row, uint32_t* mask, uint32_t all) {
@@ -186,14 +204,7 @@ __global__ void __launch_bounds__(Cfg<T, D>::kThreads, 1) attend_kernel(AttParam
       const int64_t T_top = (t + 1) / p.span_L;
       s.tail_start = p.span_L * T_top;
       const int64_t tail_len = t + 1 - s.tail_start;
-      if (tid == 0) {
-        unsigned int acc = 0;
-        for (int r = 0; r < p.kept_segs; ++r) {
-          s_segbase[r] = acc;
-          acc += T_top > 0 ? (unsigned int)p.n_kept[(int64_t)unit * p.kept_segs + r] : 0u;
-        }
-        s_segbase[p.kept_segs] = acc;
-      }
+      if (tid < 32) seg_prefix(p, unit, T_top, s_segbase);
       __syncthreads();
       const int64_t nk = s_segbase[p.kept_segs];
       s.kept = p.kept + (int64_t)unit * p.kept_segs * p.kept_stride;
@@ -503,14 +514,7 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads, 1) attend_mma_kernel(AttP
     const int64_t T_top = (t + 1) / p.span_L;
     s.tail_start = p.span_L * T_top;
     const int64_t tail_len = t + 1 - s.tail_start;
-    if (tid == 0) {
-      unsigned int acc = 0;
-      for (int r = 0; r < p.kept_segs; ++r) {
-        s_segbase[r] = acc;
-        acc += T_top > 0 ? (unsigned int)p.n_kept[(int64_t)unit * p.kept_segs + r] : 0u;
-      }
-      s_segbase[p.kept_segs] = acc;
-    }
+    if (tid < 32) seg_prefix(p, unit, T_top, s_segbase);
     __syncthreads();
     const int64_t nk = s_segbase[p.kept_segs];
     s.kept = p.kept + (int64_t)unit * p.kept_segs * p.kept_stride;
