@@ -196,20 +196,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             smem_addr(mbar))
         : "memory");
     // bounded wait for phase 0 of the barrier (all MMAs complete)
-    int ok = 0;
-    for (long long it = 0; it < kMbarSpin && !ok; ++it) {
-      uint32_t r;
-      asm volatile(
-          "{\n\t.reg .pred p;\n\t"
-          "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-          "selp.b32 %0, 1, 0, p;\n\t"
-          "}\n"
-          : "=r"(r)
-          : "r"(smem_addr(mbar)), "r"(0u)
-          : "memory");
-      ok = (int)r;
+    auto wait_mma = [&]() -> int {
+      int ok = 0;
+      for (long long it = 0; it < kMbarSpin && !ok; ++it) {
+        uint32_t r;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.b32 %0, 1, 0, p;\n\t"
+            "}\n"
+            : "=r"(r)
+            : "r"(smem_addr(mbar)), "r"(0u)
+            : "memory");
+        ok = (int)r;
+      }
+      return ok;
+    };
+    const int ok = wait_mma();
+    if (!ok) {
+      raise_status(status, ZHA_ERR_TIMEOUT);
+      // give the MMAs in flight a second bounded wait before TMEM is freed
+      (void)wait_mma();
     }
-    if (!ok) raise_status(status, ZHA_ERR_TIMEOUT);
     *done_flag = ok;
   }
   __syncthreads();
