@@ -271,3 +271,51 @@ def test_prefill_geometries(geom):
             assert lc[i, h].tolist() == e_counts.tolist(), (i, h)
             o = ref.attend(qf[i, h], 0, h, e_idx)
             assert np.abs(out[i, h] - o).max() < TOL[c.dtype], (i, h, np.abs(out[i, h] - o).max())
+
+
+def test_tensor_core_wait_timeout_falls_back(monkeypatch):
+    """The tensor-core completion wait is bounded (1 s). A test hook makes it
+    wait for a barrier phase that never completes (the MMAs themselves finish;
+    nothing faults or hangs): the call reports ZHA_ERR_TIMEOUT, certifies
+    nothing, and zha_prefill_chunk still matches the oracle through the
+    canonical top level. Without the hook the next call is clean again."""
+    base = W.CONFIGS["prefill-deep-1m-chunk4k"]
+    wl = W.Workload(base.scaled(16256, chunk=64))
+    c = wl.cfg
+    gpu = Gpu(wl)
+    start = c.n_tokens
+    gpu.cache.seq_len.fill_(start + c.chunk)
+    z.zha_build_tree(gpu.cfg, gpu.cache)  # the tree covers the chunk too
+    q = wl.queries(0).to(gpu.dev)
+    ws = z.alloc_workspace(gpu.cfg, z.ZHA_OP_PREFILL, c.chunk, device=gpu.dev)
+    cert = torch.full((c.chunk, c.n_q_heads), -1, dtype=torch.int32, device=gpu.dev)
+
+    monkeypatch.setenv("ZHA_TEST_TC_WAIT_PARITY", "1")
+    gpu.status.zero_()
+    z.zha_prefill_top_scores(gpu.cfg, gpu.cache, q, 0, start, c.p, None, cert, ws, gpu.status)
+    torch.cuda.synchronize()
+    assert int(gpu.status.item()) == z.ZHA_ERR_TIMEOUT
+    assert (cert == 0).all()
+    out = torch.empty_like(q)
+    lc = torch.full((c.chunk, c.n_q_heads, c.levels), -1, dtype=torch.int32, device=gpu.dev)
+    gpu.status.zero_()
+    z.zha_prefill_chunk(gpu.cfg, gpu.cache, q, 0, start, c.p, out, lc, ws, gpu.status)
+    torch.cuda.synchronize()
+    assert int(gpu.status.item()) == z.ZHA_ERR_TIMEOUT
+    monkeypatch.delenv("ZHA_TEST_TC_WAIT_PARITY")
+
+    ref = Ref(wl, start + c.chunk)
+    outn = out.float().cpu().numpy()
+    lcn = lc.cpu().numpy()
+    qf = q.float().cpu().numpy()
+    for i in (0, c.chunk // 2, c.chunk - 1):
+        for h in range(c.n_q_heads):
+            e_idx, e_counts, _, _ = ref.select(qf[i, h], 0, h, start + i, c.p)
+            assert lcn[i, h].tolist() == e_counts.tolist(), (i, h)
+            o = ref.attend(qf[i, h], 0, h, e_idx)
+            assert np.abs(outn[i, h] - o).max() < TOL["bf16"], (i, h)
+
+    gpu.status.zero_()
+    z.zha_prefill_top_scores(gpu.cfg, gpu.cache, q, 0, start, c.p, None, cert, ws, gpu.status)
+    gpu.check_status()
+    assert float((cert == 1).float().mean()) > 0.3

@@ -15,6 +15,9 @@
 //    (kind::f16, fp32 accumulation in TMEM, M = 128, N <= 256, K = 16 per
 //    instruction) and commits to an mbarrier; four warps read the accumulator
 //    back with tcgen05.ld and write z~ = fl(fl(acc * inv_sqrt_d) + ln|node|).
+//    The completion wait is bounded (1 s): on a timeout the kernel reports
+//    ZHA_ERR_TIMEOUT, waits once more (bounded) for its MMAs, frees TMEM and
+//    marks the chunk's scores invalid, so no unit is certified.
 // 3. top_certify_kernel: one warp per (token, query head), one CTA per
 //    (token, KV head). The tensor core sums the exact bf16 products in its own
 //    order, the canonical path in a sequential fmaf chain; both are within
@@ -41,6 +44,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <cstdlib>
+
 #include "zha_device.cuh"
 #include "zha_internal.h"
 
@@ -52,9 +57,16 @@ constexpr int kTileN = 256;
 constexpr int kTcThreads = 128;
 constexpr uint32_t kTmemCols = 256;
 constexpr int kTcD = 128;                  // head_dim of the tensor-core path
-constexpr long long kMbarSpin = 1ll << 24; // bounded wait on the MMA completion
+constexpr long long kMbarSpin = 1ll << 24; // iteration cap of the MMA completion wait
+constexpr unsigned long long kWaitNs = 1000000000ull;  // and its time limit (1 s)
 constexpr int kCertPer = 32;               // top nodes per lane in the certifier
 constexpr int kTopCapMax = 32 * kCertPer;  // top nodes per unit on this path
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -88,8 +100,11 @@ __device__ __forceinline__ uint32_t sw128_offset(int r, int c, int rows) {
 }
 
 // |s_i| of every top-level summary of the sequence, per KV head: snorm[kvh][i].
+// It also sets *tc_valid = 1 ahead of the scoring kernel, which clears it if a
+// completion wait gives up.
 __global__ void top_norms_kernel(const __nv_bfloat16* top, int64_t top_stride, int64_t n_top,
-                                 int64_t cap, int Hkv, float* snorm) {
+                                 int64_t cap, int Hkv, float* snorm, int32_t* tc_valid) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) *tc_valid = 1;
   const int64_t w = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (w >= (int64_t)Hkv * cap) return;
@@ -116,7 +131,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     top_score_tc_kernel(const __nv_bfloat16* q, int64_t rows, int Hq, int G,
                         const __nv_bfloat16* top, int64_t top_stride, int64_t n_top,
                         float inv_sqrt_d, float lnsize, float* zt, int64_t zt_stride,
-                        int32_t* status) {
+                        int32_t* status, int32_t* tc_valid, uint32_t wait_parity) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   // tiles on 1024-byte boundaries: the swizzle pattern repeats every 1024 bytes
   unsigned char* base = reinterpret_cast<unsigned char*>(
@@ -195,8 +210,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
             smem_addr(mbar))
         : "memory");
-    // bounded wait for phase 0 of the barrier (all MMAs complete)
-    auto wait_mma = [&]() -> int {
+    // bounded wait (time and iterations) for the completion phase of the
+    // barrier. wait_parity is 0; a test sets 1, a phase that never completes,
+    // to run the timeout path without any fault
+    auto wait_mma = [&](uint32_t parity) -> int {
+      const unsigned long long t0 = global_ns();
       int ok = 0;
       for (long long it = 0; it < kMbarSpin && !ok; ++it) {
         uint32_t r;
@@ -206,17 +224,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             "selp.b32 %0, 1, 0, p;\n\t"
             "}\n"
             : "=r"(r)
-            : "r"(smem_addr(mbar)), "r"(0u)
+            : "r"(smem_addr(mbar)), "r"(parity)
             : "memory");
         ok = (int)r;
+        if (!ok && global_ns() - t0 > kWaitNs) break;
       }
       return ok;
     };
-    const int ok = wait_mma();
+    const int ok = wait_mma(wait_parity);
     if (!ok) {
       raise_status(status, ZHA_ERR_TIMEOUT);
-      // give the MMAs in flight a second bounded wait before TMEM is freed
-      (void)wait_mma();
+      *tc_valid = 0;  // the certifier then certifies nothing: canonical top level
+      // a second bounded wait for the MMAs in flight before TMEM is freed
+      (void)wait_mma(0u);
     }
     *done_flag = ok;
   }
@@ -285,6 +305,7 @@ struct CertParams {
   int32_t* cnt;             // [tokens * Hkv][G]
   float* z_out;             // nullable: [tokens][Hq][cap]
   int32_t* cert_out;        // nullable: [tokens][Hq]
+  const int32_t* tc_valid;  // 0: a scoring wait gave up, the scores are not to be used
 };
 
 __device__ __forceinline__ double warp_sum_d(double v) {
@@ -368,9 +389,11 @@ __global__ void __launch_bounds__(32 * kMaxGroup) top_certify_kernel(CertParams 
 
   const bool keep_all = p.p_q >= (1ull << 32);
   const double pr = (double)p.p_q * 0x1p-32;
-  bool cert = keep_all;
+  // scores of a chunk whose scoring wait gave up are not used: no certificate
+  const bool tc_ok = n > 0 && *p.tc_valid != 0;
+  bool cert = keep_all && tc_ok;
   uint32_t tau = 0u;  // candidate set: nodes whose order key is >= tau
-  if (!keep_all && finite && n > 0) {
+  if (!keep_all && finite && tc_ok) {
     // the smallest descending prefix whose softmax mass reaches p (approximate:
     // only the certificate below has to be exact)
     float w[PER];
@@ -481,7 +504,7 @@ bool top_tc_supported(const Geometry& g) {
 namespace {
 
 struct TopLayout {
-  size_t snorm, zt, ok, cnt, mask, total;
+  size_t snorm, zt, ok, cnt, mask, valid, total;
   int64_t zs;  // row stride of the score buffer (floats)
 };
 
@@ -502,6 +525,8 @@ TopLayout top_layout(const Geometry& g, int64_t n_tok) {
   off = align256_(off + sizeof(int32_t) * (size_t)n_tok * g.Hkv * g.G);
   T.mask = off;
   off = align256_(off + (size_t)n_tok * g.Hkv * cap);
+  T.valid = off;
+  off = align256_(off + sizeof(int32_t));
   T.total = off;
   return T;
 }
@@ -535,6 +560,13 @@ cudaError_t launch_top_select(const Geometry& g, const void* tree, const int32_t
   int32_t* ok = reinterpret_cast<int32_t*>(w + T.ok);
   int32_t* cnt = reinterpret_cast<int32_t*>(w + T.cnt);
   uint8_t* mask = reinterpret_cast<uint8_t*>(w + T.mask);
+  int32_t* tc_valid = reinterpret_cast<int32_t*>(w + T.valid);
+  // test hook: ZHA_TEST_TC_WAIT_PARITY=1 makes the scoring kernel wait for a
+  // barrier phase that never completes, so its bounded wait runs out (the
+  // MMAs themselves complete); the call then reports ZHA_ERR_TIMEOUT and the
+  // top level falls back to canonical scoring
+  const char* hook = getenv("ZHA_TEST_TC_WAIT_PARITY");
+  const uint32_t wait_parity = (hook && hook[0] == '1') ? 1u : 0u;
   seeds->ok = ok;
   seeds->mask = mask;
   seeds->cnt = cnt;
@@ -546,7 +578,7 @@ cudaError_t launch_top_select(const Geometry& g, const void* tree, const int32_t
   if (n_top > 0) {
     const int64_t warps = (int64_t)g.Hkv * cap;
     top_norms_kernel<<<(unsigned)((warps * 32 + 255) / 256), 256, 0, stream>>>(
-        top, top_stride, n_top, cap, g.Hkv, snorm);
+        top, top_stride, n_top, cap, g.Hkv, snorm, tc_valid);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const size_t smem = top_score_tc_smem();
@@ -557,7 +589,7 @@ cudaError_t launch_top_select(const Geometry& g, const void* tree, const int32_t
               (unsigned)g.Hkv);
     top_score_tc_kernel<<<grid, kTcThreads, smem, stream>>>(
         static_cast<const __nv_bfloat16*>(q), rows, g.Hq, g.G, top, top_stride, n_top,
-        g.inv_sqrt_d, g.lnsize[g.L - 1], zt, T.zs, status);
+        g.inv_sqrt_d, g.lnsize[g.L - 1], zt, T.zs, status, tc_valid, wait_parity);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   CertParams c{};
@@ -583,6 +615,7 @@ cudaError_t launch_top_select(const Geometry& g, const void* tree, const int32_t
   c.cnt = cnt;
   c.z_out = z_out;
   c.cert_out = cert_out;
+  c.tc_valid = tc_valid;
   const unsigned grid = (unsigned)(n_tok * g.Hkv), block = 32u * (unsigned)g.G;
   if (cap <= 32 * 4) top_certify_kernel<4><<<grid, block, 0, stream>>>(c);
   else if (cap <= 32 * 8) top_certify_kernel<8><<<grid, block, 0, stream>>>(c);
