@@ -77,3 +77,40 @@ def test_bad_arguments_rejected_before_launch(z):
     assert L.zha_dense_decode(ctypes.byref(cfg), ctypes.byref(c), ctypes.c_void_p(16),
                               ctypes.c_void_p(16), ctypes.c_void_p(16), 1, None) == \
         z.ZHA_ERR_WORKSPACE
+
+
+def test_prefill_top_scores_rejected_before_launch(z):
+    L = z.lib()
+    c = z.zha_cache(16, 16, 16, 16, 16)  # non-null dummies: never dereferenced here
+
+    def call(cfg, q, start, T, ws_bytes=1):
+        return L.zha_prefill_top_scores(ctypes.byref(cfg), ctypes.byref(c), ctypes.c_void_p(q),
+                                        0, start, T, 0.95, None, None, ctypes.c_void_p(256),
+                                        ws_bytes, None, None)
+
+    bf = z.make_config(128, 4, 3, 16, 2, 1, 40000, torch.bfloat16)
+    assert call(bf, 256, 30000, 100) == z.ZHA_ERR_WORKSPACE        # valid, workspace too small
+    assert call(bf, 258, 30000, 100) == z.ZHA_ERR_INVALID_ARG      # q not 16-byte aligned
+    assert call(bf, 256, 39990, 100) == z.ZHA_ERR_INVALID_ARG      # chunk past the capacity
+    assert call(bf, 256, 30000, 0) == z.ZHA_ERR_INVALID_ARG        # empty chunk
+    f32 = z.make_config(128, 4, 3, 16, 2, 1, 40000, torch.float32)
+    assert call(f32, 256, 30000, 100) == z.ZHA_ERR_UNSUPPORTED      # fp32: no tensor-core path
+    one = z.make_config(128, 256, 1, 16, 2, 1, 40000, torch.bfloat16)
+    assert call(one, 256, 30000, 100) == z.ZHA_ERR_UNSUPPORTED      # L = 1: no level below
+
+
+def test_prefill_workspace_never_shrinks_with_the_chunk(z):
+    # host-side sizing only (no device): a longer chunk never needs less
+    cfg = z.make_config(128, 4, 6, 16, 2, 1, 1048576 + 4096, torch.bfloat16)
+    sizes = [z.zha_workspace_bytes(cfg, z.ZHA_OP_PREFILL, T) for T in range(1, 401, 7)]
+    assert all(b >= a for a, b in zip(sizes, sizes[1:])), sizes
+
+
+def test_kernel_source_hash_is_stable():
+    import importlib
+    import sys
+
+    sys.path.insert(0, ROOT)
+    bench = importlib.import_module("bench")
+    h = bench.kernel_source_hash()
+    assert len(h) == 16 and h == bench.kernel_source_hash()
