@@ -195,7 +195,10 @@ zha_status zha_decode_stats(const zha_config* cfg, const void* ws, size_t ws_byt
  * The top level of every (token, head) is first scored on the tensor cores
  * (zha_prefill_top_scores) when the geometry allows it; a (token, KV head)
  * whose tensor-core selection is certified skips the top level's canonical
- * scoring. Certified or not, every selection equals the canonical one. */
+ * scoring. Certified or not, every selection equals the canonical one. If
+ * the tensor-core completion wait runs out (bounded at 1 s), dev_status gets
+ * ZHA_ERR_TIMEOUT, no unit is certified and the top level is scored
+ * canonically: the results stay exact. */
 zha_status zha_prefill_chunk(const zha_config* cfg, const zha_cache* cache, const void* q,
                              int32_t seq, int64_t chunk_start, int64_t T, double p, void* out,
                              int32_t* level_counts, void* ws, size_t ws_bytes,
@@ -215,7 +218,8 @@ zha_status zha_prefill_chunk(const zha_config* cfg, const zha_cache* cache, cons
  *     |q| |s_n| (no rounding-order guarantee).
  *   - certified (nullable, device): [T][Hq] int32, 1 when the canonical cut
  *     over the top level is proven equal to the cut taken on z_top (the proof
- *     is the same one zha_prefill_chunk relies on), else 0.
+ *     is the same one zha_prefill_chunk relies on), else 0. All 0 after a
+ *     ZHA_ERR_TIMEOUT, when z_top is not written.
  *   - ws: ZHA_OP_PREFILL workspace for max_queries >= T (not preserved).
  *   - Errors: ZHA_ERR_UNSUPPORTED unless dtype is bf16, head_dim 128, L >= 2,
  *     G <= 8 and capacity / b^L <= 1024; ZHA_ERR_INVALID_ARG for a bad chunk,
