@@ -8,9 +8,9 @@
  * query reads. Keys are cut into contiguous blocks of b tokens; each block gets
  * one summary key derived from 16 learned reference queries; blocks are grouped
  * level by level (a level-l node covers b^l tokens). A query scores the top
- * nodes, keeps the smallest set covering a fraction p of the estimated
- * attention mass, expands only the kept branches down to the raw KV entries,
- * and always keeps the first token. Paragraph 2 gives the operating point
+ * nodes, keeps the fewest nodes whose estimated attention mass reaches the
+ * fraction p, descends only into the kept branches until it reaches individual
+ * keys, and always keeps token 0. Paragraph 2 gives the operating point
  * p = 0.95 and the two geometries (b = 4, L = 6) and (b = 256, L = 1).
  *
  * Formulas the pages leave open are fixed by this library as:

@@ -12,9 +12,9 @@
  *             a query reads; keys are cut into contiguous blocks, each block is
  *             summarised by one key derived from 16 learned reference queries,
  *             and blocks are grouped level by level; a query scores the top
- *             nodes, keeps the smallest set covering a fraction p of the
- *             estimated attention mass, expands only those branches down to the
- *             raw KV entries, and always keeps the first token.
+ *             nodes, keeps the fewest nodes whose estimated attention mass
+ *             reaches the fraction p, descends only into the kept branches
+ *             until it reaches individual keys, and always keeps token 0.
  *   [lefilia] par. 2: p = 0.95; deep tree (blocks of 4, 6 levels) and wide tree
  *             (blocks of 256, 1 level).
  * The pages leave the formulas open. This library fixes them as:
@@ -114,9 +114,8 @@ float zo_inv_sqrt_d(int d) { return (float)(1.0 / sqrt((double)d)); }
 float zo_lnsize(int level, int b) { return (float)((double)level * log((double)b)); }
 
 /* ------------------------------------------------------------------------ */
-/* summary keys  [lefilia par. 1: "chacun resume par une cle de synthese     */
-/* issue de 16 requetes de reference apprises, puis regroupe niveau par      */
-/* niveau"]                                                                 */
+/* summary keys  [lefilia page, par. 1: one key per node, derived from 16  */
+/* learned reference queries; the tree is built one level at a time]        */
 /* ------------------------------------------------------------------------ */
 
 /*
@@ -188,8 +187,8 @@ int64_t zo_build_tree(const float* K, int64_t n, int d, const float* R, int b, i
 }
 
 /* ------------------------------------------------------------------------ */
-/* top-p cut at one level  [lefilia par. 1: "conserve le plus petit ensemble */
-/* couvrant une fraction p de la masse d'attention estimee"]                 */
+/* top-p cut at one level  [lefilia page, par. 1: the fewest nodes whose    */
+/* estimated attention mass reaches the fraction p]                          */
 /* ------------------------------------------------------------------------ */
 
 typedef struct {
@@ -272,9 +271,9 @@ int64_t zo_cut(const float* z, const int64_t* node, int64_t n, uint64_t p_q, int
 }
 
 /* ------------------------------------------------------------------------ */
-/* per-query traversal  [lefilia par. 1: "une requete evalue les noeuds du   */
-/* haut ... puis n'etend que ces branches jusqu'aux entrees KV brutes. Le    */
-/* premier token est toujours conserve"]                                     */
+/* per-query traversal  [lefilia page, par. 1: start from the top nodes,   */
+/* descend only into kept branches, down to the individual keys; token 0 is */
+/* always part of the selection]                                            */
 /* ------------------------------------------------------------------------ */
 
 /* z = (dot(q, s) * inv_sqrt_d) + lnsize_l, two separately rounded fp32 ops. */

@@ -2,9 +2,9 @@
 // together.
 //
 // lefilia.fr page "Zyphra presente Zyphra Hierarchical Attention (ZHA) ...",
-// paragraph 1: a query scores the top nodes, keeps the smallest set covering a
-// fraction p of the estimated attention mass, expands only the kept branches
-// down to the raw KV entries, and always keeps the first token.
+// paragraph 1: a query scores the top nodes, keeps the fewest nodes whose
+// estimated attention mass reaches the fraction p, descends only into the kept
+// branches until it reaches individual keys, and always keeps token 0.
 //
 // Unit of work: one query token and one KV head, i.e. the G = Hq/Hkv query
 // heads that read the same tree. At every level the unit's candidate list is
