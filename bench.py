@@ -123,11 +123,40 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def strip_c_comments(src: str) -> str:
+    """C/C++ source without its comments, each whitespace run folded to one
+    space; string and character literals are kept as written."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+            out.append(" ")
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        elif c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_hash() -> str:
+    """Hash of the decode-step kernels' code, comments and layout excluded, so
+    that recorded DRAM counters stay tied to the code they were taken on."""
     h = hashlib.sha256()
     for f in ("traverse.cu", "attend.cu", "zha_device.cuh"):
-        with open(os.path.join(ROOT, "tree_indexed_sparse_zha_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "tree_indexed_sparse_zha_b200", "csrc", f), encoding="utf-8") as fh:
+            h.update(strip_c_comments(fh.read()).encode())
+            h.update(b"\0")
     return h.hexdigest()[:16]
 
 

@@ -114,3 +114,19 @@ def test_kernel_source_hash_is_stable():
     bench = importlib.import_module("bench")
     h = bench.kernel_source_hash()
     assert len(h) == 16 and h == bench.kernel_source_hash()
+
+
+def test_kernel_source_hash_ignores_comments_only():
+    import importlib
+    import sys
+
+    sys.path.insert(0, ROOT)
+    bench = importlib.import_module("bench")
+    strip = bench.strip_c_comments
+    base = 'int f(int a) { return a + 1; } // tail\nconst char* s = "//x /*y*/";\n'
+    reworded = '/* lead */ int f(int a)  {\n  return a + 1; /* inline */ }\nconst char* s = "//x /*y*/";'
+    assert strip(base) == strip(reworded)
+    # literals that look like comments stay, and a code change shows
+    assert '"//x /*y*/"' in strip(base)
+    assert strip(base) != strip(base.replace("a + 1", "a + 2"))
+    assert strip("char c = '\\'';  // q") == "char c = '\\'';"
