@@ -716,7 +716,7 @@ def main():
         wl = W.make(args.workload, device=dev, n_tokens=args.n_tokens)
         c = wl.cfg
         if is_prefill(args.workload):
-            rate, done, el = oracle_prefill_rate(wl, args.steps, budget_s=600.0)
+            rate, done, el = oracle_prefill_rate(wl, args.steps, budget_s=180.0)
             line = {"impl": "reference", "metric": PREFILL_METRIC, "value": rate,
                     "unit": "queries/s", "n_gpus": 1, "steps": args.steps,
                     "warmup": args.warmup,
@@ -733,7 +733,7 @@ def main():
             print(json.dumps(line), flush=True)
             return
         oracle_rate(wl, min(args.warmup, 2), budget_s=60.0)  # warm-up
-        rate, done, el = oracle_rate(wl, args.steps, budget_s=600.0)
+        rate, done, el = oracle_rate(wl, args.steps, budget_s=180.0)
         line = {"impl": "reference", "metric": METRIC, "value": rate, "unit": "queries/s",
                 "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": el / done * c.batch * c.n_q_heads * 1e3,
