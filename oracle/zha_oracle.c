@@ -221,7 +221,9 @@ uint64_t zo_p_fixed(double p) { return (uint64_t)floor(p * 4294967296.0 + 0.5); 
  *   need = ceil(T * p_q / 2^32);  order by (z desc, node asc);
  *   k = smallest prefix length whose mass reaches need (all if p_q >= 2^32).
  * near_tie (nullable) is set to 1 if the cutoff score z_(k) lies within 1e-6
- * relative of a sorted neighbour (|dz| <= 1e-6 max(|z_(k)|, 1)).
+ * relative of a sorted neighbour (|dz| <= 1e-6 max(|z_(k)|, 1)), or if the
+ * target need lies within 1e-6 T of the prefix mass on either side of the
+ * cut (need - C_(k-1) or C_k - need, where C_j is the mass of the first j).
  * T_out / need_out (nullable) receive T and need.
  */
 int64_t zo_cut(const float* z, const int64_t* node, int64_t n, uint64_t p_q, int64_t* kept,
@@ -242,10 +244,11 @@ int64_t zo_cut(const float* z, const int64_t* node, int64_t n, uint64_t p_q, int
   const uint64_t need = (uint64_t)((prod + (((unsigned __int128)1 << 32) - 1)) >> 32);
   qsort(c, (size_t)n, sizeof(zo_cand), zo_cmp_cand);
   int64_t k;
-  if (p_q >= ((uint64_t)1 << 32)) {
+  const int all = p_q >= ((uint64_t)1 << 32);
+  uint64_t cum = 0; /* C_k, the mass of the kept prefix */
+  if (all) {
     k = n;
   } else {
-    uint64_t cum = 0;
     k = n;
     for (int64_t i = 0; i < n; ++i) {
       cum += c[i].mass;
@@ -261,6 +264,12 @@ int64_t zo_cut(const float* z, const int64_t* node, int64_t n, uint64_t p_q, int
     const float band = 1e-6f * (fabsf(zk) > 1.0f ? fabsf(zk) : 1.0f);
     if (k < n && fabsf(zk - c[k].z) <= band) *near_tie = 1;
     if (k >= 2 && fabsf(c[k - 2].z - zk) <= band) *near_tie = 1;
+    /* the cut's mass margin: C_(k-1) < need <= C_k, either side within 1e-6 T */
+    if (!all) {
+      const double mband = 1e-6 * (double)T;
+      const uint64_t prev = cum - c[k - 1].mass; /* C_(k-1) */
+      if ((double)(need - prev) <= mband || (double)(cum - need) <= mband) *near_tie = 1;
+    }
   }
   for (int64_t i = 0; i < k; ++i) kept[i] = c[i].node;
   qsort(kept, (size_t)k, sizeof(int64_t), zo_cmp_i64);

@@ -234,6 +234,29 @@ def test_cut_brute_force():
     assert checked > 300
 
 
+def test_cut_near_tie_flags():
+    """The near-tie flag, by hand: a cutoff score within 1e-6 relative of a
+    sorted neighbour, or a target mass within 1e-6 T of the prefix mass on
+    either side of the cut."""
+    nodes = np.arange(3, dtype=np.int64)
+    # masses 1, 0.61, 0.61: p = 0.6 keeps two, far from either prefix mass, and
+    # the third score sits 1e-7 below the cutoff score
+    z = np.array([0.0, -0.5, np.nextafter(np.float32(-0.5), np.float32(-1))], np.float32)
+    kept, T, need, tie = oracle.cut(z, nodes, 0.6)
+    assert kept.tolist() == [0, 1] and tie
+    z[2] = -0.6
+    assert oracle.cut(z, nodes, 0.6)[3] is False
+    # masses 1 and about 1/3: p = 0.75 puts the target on the first prefix
+    # mass (2^40), up to the rounding of -ln 3, with scores far apart
+    z2 = np.array([0.0, -np.log(3.0)], np.float32)
+    kept, T, need, tie = oracle.cut(z2, nodes[:2], 0.75)
+    assert abs(int(need) - 2**40) <= 1e-6 * T and tie
+    # p = 0.6: the target is 0.2 T below the first prefix mass, no flag
+    assert oracle.cut(z2, nodes[:2], 0.6)[3] is False
+    # p = 1 makes no cut, so no mass margin applies
+    assert oracle.cut(z2, nodes[:2], 1.0)[3] is False
+
+
 def test_cut_p_one_keeps_everything():
     z = np.array([0.0, -200.0, -100.0, 1.0], np.float32)  # two masses truncate to 0
     kept, T, need, _ = oracle.cut(z, np.arange(4), 1.0)
