@@ -149,6 +149,20 @@ def strip_c_comments(src: str) -> str:
     return " ".join("".join(out).split())
 
 
+def selection_per_query(lc, b: int, L: int, n: int) -> dict:
+    """Per-query selection figures from kept counts lc [B][Hq][L] (top level
+    first) of decode queries at position n - 1: the mean kept nodes per level
+    and the mean fraction of the n visible tokens selected. A query selects
+    b tokens per kept level-1 node, the tail past the last complete top node,
+    and token 0 when node (1, 0) is not kept, so the fraction is exact to
+    within one token per query."""
+    top = n // b ** L
+    tail = n - b ** L * top
+    k1 = lc[..., L - 1].double()
+    return {"mean_kept_per_level": [round(float(v), 3) for v in lc.double().mean(dim=(0, 1))],
+            "mean_selected_fraction": float(((b * k1 + tail) / n).mean())}
+
+
 def kernel_source_hash() -> str:
     """Hash of the decode-step kernels' code, comments and layout excluded, so
     that recorded DRAM counters stay tied to the code they were taken on."""
@@ -184,7 +198,8 @@ def recorded_traffic():
 
 def oracle_rate(wl, n_queries: int, budget_s: float = 20.0):
     """Times the CPU oracle (tree for one (sequence, KV head) built untimed, then
-    select + fp64 attention per query) on decode steps of that unit."""
+    select + fp64 attention per query) on decode steps of that unit. Returns
+    (queries/s, queries, seconds, queries flagged near-tie)."""
     import numpy as np
 
     import oracle
@@ -194,26 +209,28 @@ def oracle_rate(wl, n_queries: int, budget_s: float = 20.0):
     V = wl.V[0, 0].float().cpu().numpy()
     R = wl.R.float().cpu().numpy()
     tr = oracle.build_tree(K, c.n_tokens, R, c.block, c.levels, True, c.capacity)
-    done = 0
+    done = flagged = 0
     t0 = time.perf_counter()
     step = 1
     while done < n_queries and time.perf_counter() - t0 < budget_s:
         q = wl.queries(step)[0].float().cpu().numpy()
         t = c.n_tokens + step - 1
         for h in range(c.group):
-            idx, _, _, _ = oracle.select(q[h], tr, t, c.p)
+            idx, _, _, tie = oracle.select(q[h], tr, t, c.p)
             oracle.attend(q[h], K, V, idx)
+            flagged += tie
             done += 1
             if done >= n_queries:
                 break
         step += 1
     el = time.perf_counter() - t0
-    return done / el, done, el
+    return done / el, done, el, flagged
 
 
 def oracle_prefill_rate(wl, n_queries: int, budget_s: float = 20.0):
     """Times the CPU oracle on chunk queries of KV head 0 (tree over the cached
-    context and the chunk built untimed; select + fp64 attention per query)."""
+    context and the chunk built untimed; select + fp64 attention per query).
+    Returns (queries/s, queries, seconds, queries flagged near-tie)."""
     import numpy as np  # noqa: F401
 
     import oracle
@@ -225,19 +242,20 @@ def oracle_prefill_rate(wl, n_queries: int, budget_s: float = 20.0):
     R = wl.R.float().cpu().numpy()
     tr = oracle.build_tree(K, n, R, c.block, c.levels, True, c.capacity)
     q = wl.queries(0).float().cpu().numpy()
-    done = 0
+    done = flagged = 0
     t0 = time.perf_counter()
     i = 0
     while done < n_queries and time.perf_counter() - t0 < budget_s and i < c.chunk:
         for h in range(c.group):
-            idx, _, _, _ = oracle.select(q[i, h], tr, c.n_tokens + i, c.p)
+            idx, _, _, tie = oracle.select(q[i, h], tr, c.n_tokens + i, c.p)
             oracle.attend(q[i, h], K, V, idx)
+            flagged += tie
             done += 1
             if done >= n_queries:
                 break
         i += 1
     el = time.perf_counter() - t0
-    return done / el, done, el
+    return done / el, done, el, flagged
 
 
 # ---------------------------------------------------------------------------
@@ -389,6 +407,11 @@ def run_zha(args, rank, world, dev):
     cand_rows = int(stats[:, :L].sum())
     kept_nodes = int(stats[:, L].sum())
     kv_rows = kept_nodes * b + B * Hkv * (1 + tail)
+    # per-query kept counts of the last step's queries: one more select, untimed
+    lc = torch.zeros(B, Hq, L, dtype=torch.int32, device=dev)
+    z.zha_decode_select(cfg, cache, step_inputs(args.warmup + args.steps - 1)[3], c.p, lc, ws, st)
+    torch.cuda.synchronize()
+    per_query = selection_per_query(lc.cpu(), b, L, n_last)
     sel_bytes = cand_rows * row + kept_nodes * 4 + 2 * queries_per_step * row
     att_bytes = kv_rows * 2 * row + kept_nodes * 4 + 2 * queries_per_step * row
     ext_bytes = 0
@@ -467,7 +490,7 @@ def run_zha(args, rank, world, dev):
         "phases_ms": {"extend": ms_ext, "select": ms_sel, "attend": ms_att},
         "selection": {"summary_rows_scored": cand_rows, "kept_level1_nodes": kept_nodes,
                       "kv_rows_read": kv_rows,
-                      "kv_fraction_read": kv_rows / (B * Hkv * n_last)},
+                      "kv_fraction_read": kv_rows / (B * Hkv * n_last), **per_query},
         "roofline": roof,
         "dense": {"ms_per_step": dense_ms, "queries_per_s": queries_per_step * world / (dense_ms / 1e3),
                   "hbm_gbs": dense_bytes / (dense_ms / 1e3) / 1e9,
@@ -716,7 +739,7 @@ def main():
         wl = W.make(args.workload, device=dev, n_tokens=args.n_tokens)
         c = wl.cfg
         if is_prefill(args.workload):
-            rate, done, el = oracle_prefill_rate(wl, args.steps, budget_s=180.0)
+            rate, done, el, flagged = oracle_prefill_rate(wl, args.steps, budget_s=180.0)
             line = {"impl": "reference", "metric": PREFILL_METRIC, "value": rate,
                     "unit": "queries/s", "n_gpus": 1, "steps": args.steps,
                     "warmup": args.warmup,
@@ -725,7 +748,7 @@ def main():
                     "dtype": "f32 select / f64 attention", "data": "synthetic",
                     "config": workload_config(args, c),
                     "cpu_baseline": {"value": rate, "unit": "queries/s", "cores": 1,
-                                     "kind": "oracle",
+                                     "kind": "oracle", "near_tie_flagged": flagged,
                                      "sample": f"{done} chunk queries (query heads of KV head "
                                                f"0) in {el:.1f} s, tree built untimed"},
                     "e2e": {"value": rate, "unit": "queries/s", "h2d_bytes_per_step": 0,
@@ -733,7 +756,7 @@ def main():
             print(json.dumps(line), flush=True)
             return
         oracle_rate(wl, min(args.warmup, 2), budget_s=60.0)  # warm-up
-        rate, done, el = oracle_rate(wl, args.steps, budget_s=180.0)
+        rate, done, el, flagged = oracle_rate(wl, args.steps, budget_s=180.0)
         line = {"impl": "reference", "metric": METRIC, "value": rate, "unit": "queries/s",
                 "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": el / done * c.batch * c.n_q_heads * 1e3,
@@ -741,7 +764,7 @@ def main():
                 "vs_baseline": None, "dtype": "f32 select / f64 attention",
                 "data": "synthetic", "config": workload_config(args, c),
                 "cpu_baseline": {"value": rate, "unit": "queries/s", "cores": 1,
-                                 "kind": "oracle",
+                                 "kind": "oracle", "near_tie_flagged": flagged,
                                  "sample": f"{done} queries (the query heads of KV head 0 of "
                                            f"sequence 0, successive decode steps) in {el:.1f} s, "
                                            "tree built untimed"},
@@ -763,13 +786,15 @@ def main():
     res, wl = (run_prefill if prefill else run_zha)(args, rank, world, dev)
     if rank == 0:
         if world == 1 and not args.no_cpu_baseline and prefill:
-            rate, done, el = oracle_prefill_rate(wl, 200, budget_s=20.0)
+            rate, done, el, flagged = oracle_prefill_rate(wl, 200, budget_s=20.0)
             res["cpu_baseline"] = {"value": rate, "unit": "queries/s", "cores": 1, "kind": "oracle",
+                                   "near_tie_flagged": flagged,
                                    "sample": f"{done} chunk queries of KV head 0 over {el:.1f} s "
                                              "(tree built untimed)"}
         elif world == 1 and not args.no_cpu_baseline:
-            rate, done, el = oracle_rate(wl, 200, budget_s=20.0)
+            rate, done, el, flagged = oracle_rate(wl, 200, budget_s=20.0)
             res["cpu_baseline"] = {"value": rate, "unit": "queries/s", "cores": 1, "kind": "oracle",
+                                   "near_tie_flagged": flagged,
                                    "sample": f"{done} queries of sequence 0 / KV head 0 over "
                                              f"{el:.1f} s (tree built untimed)"}
         else:

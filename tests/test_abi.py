@@ -130,3 +130,17 @@ def test_kernel_source_hash_ignores_comments_only():
     assert '"//x /*y*/"' in strip(base)
     assert strip(base) != strip(base.replace("a + 1", "a + 2"))
     assert strip("char c = '\\'';  // q") == "char c = '\\'';"
+
+
+def test_bench_selection_per_query():
+    import importlib
+    import sys
+
+    sys.path.insert(0, ROOT)
+    bench = importlib.import_module("bench")
+    # b = 4, L = 2, n = 37: two complete top nodes (32 tokens) and a tail of 5
+    lc = torch.tensor([[[2, 3], [1, 4]]], dtype=torch.int32)  # [B=1][Hq=2][L=2]
+    r = bench.selection_per_query(lc, 4, 2, 37)
+    assert r["mean_kept_per_level"] == [1.5, 3.5]
+    # (4 * 3 + 5) / 37 and (4 * 4 + 5) / 37
+    assert abs(r["mean_selected_fraction"] - (17 / 37 + 21 / 37) / 2) < 1e-12
