@@ -149,18 +149,26 @@ def strip_c_comments(src: str) -> str:
     return " ".join("".join(out).split())
 
 
-def selection_per_query(lc, b: int, L: int, n: int) -> dict:
+def selection_per_query(lc, b: int, L: int, n: int, row: int) -> dict:
     """Per-query selection figures from kept counts lc [B][Hq][L] (top level
-    first) of decode queries at position n - 1: the mean kept nodes per level
-    and the mean fraction of the n visible tokens selected. A query selects
-    b tokens per kept level-1 node, the tail past the last complete top node,
-    and token 0 when node (1, 0) is not kept, so the fraction is exact to
-    within one token per query."""
+    first) of decode queries at position n - 1, with summary and K/V rows of
+    `row` bytes:
+    - the mean kept nodes per level and the mean fraction of the n visible
+      tokens selected. A query selects b tokens per kept level-1 node, the
+      tail past the last complete top node, and token 0 when node (1, 0) is
+      not kept, so the fraction is exact to within one token per query;
+    - the bytes the queries would touch if every query head read its own
+      summary rows (the top nodes, then b per node kept above level 1), its
+      own K and V rows and its index list: the sum over query heads, which
+      counts the GQA duplication that the shared reads avoid."""
     top = n // b ** L
     tail = n - b ** L * top
-    k1 = lc[..., L - 1].double()
+    k = lc.long()
+    sel = b * k[..., L - 1] + tail
+    scored = top + b * k[..., :L - 1].sum(-1)
     return {"mean_kept_per_level": [round(float(v), 3) for v in lc.double().mean(dim=(0, 1))],
-            "mean_selected_fraction": float(((b * k1 + tail) / n).mean())}
+            "mean_selected_fraction": float((sel.double() / n).mean()),
+            "bytes_per_q_head_sum": int((scored * row + sel * (2 * row + 8)).sum())}
 
 
 def kernel_source_hash() -> str:
@@ -411,7 +419,7 @@ def run_zha(args, rank, world, dev):
     lc = torch.zeros(B, Hq, L, dtype=torch.int32, device=dev)
     z.zha_decode_select(cfg, cache, step_inputs(args.warmup + args.steps - 1)[3], c.p, lc, ws, st)
     torch.cuda.synchronize()
-    per_query = selection_per_query(lc.cpu(), b, L, n_last)
+    per_query = selection_per_query(lc.cpu(), b, L, n_last, D * 2)
     sel_bytes = cand_rows * row + kept_nodes * 4 + 2 * queries_per_step * row
     att_bytes = kv_rows * 2 * row + kept_nodes * 4 + 2 * queries_per_step * row
     ext_bytes = 0

@@ -140,7 +140,10 @@ def test_bench_selection_per_query():
     bench = importlib.import_module("bench")
     # b = 4, L = 2, n = 37: two complete top nodes (32 tokens) and a tail of 5
     lc = torch.tensor([[[2, 3], [1, 4]]], dtype=torch.int32)  # [B=1][Hq=2][L=2]
-    r = bench.selection_per_query(lc, 4, 2, 37)
+    r = bench.selection_per_query(lc, 4, 2, 37, 256)
     assert r["mean_kept_per_level"] == [1.5, 3.5]
     # (4 * 3 + 5) / 37 and (4 * 4 + 5) / 37
     assert abs(r["mean_selected_fraction"] - (17 / 37 + 21 / 37) / 2) < 1e-12
+    # summary rows 2 + 4 * 2 and 2 + 4 * 1; K and V rows plus two 4-byte
+    # index entries per selected token
+    assert r["bytes_per_q_head_sum"] == (10 + 6) * 256 + (17 + 21) * (512 + 8)
