@@ -6,12 +6,13 @@
  * (ZHA), une voie vers une attention vraiment sous-quadratique", paragraph 1):
  * the KV cache stays complete and a tree over it only decides which keys each
  * query reads. Keys are cut into contiguous blocks of b tokens; each block gets
- * one summary key derived from 16 learned reference queries; blocks are grouped
- * level by level (a level-l node covers b^l tokens). A query scores the top
- * nodes, keeps the fewest nodes whose estimated attention mass reaches the
- * fraction p, descends only into the kept branches until it reaches individual
- * keys, and always keeps token 0. Paragraph 2 gives the operating point
- * p = 0.95 and the two geometries (b = 4, L = 6) and (b = 256, L = 1).
+ * one summary key derived from 16 learned reference queries; each higher level
+ * summarises groups of b nodes of the level below (a level-l node covers b^l
+ * tokens). A query scores the top nodes, keeps the fewest nodes whose
+ * estimated attention mass reaches the fraction p, descends only into the
+ * kept branches until it reaches individual keys, and always keeps token 0.
+ * Paragraph 2 gives the operating point p = 0.95 and the two geometries
+ * (b = 4, L = 6) and (b = 256, L = 1).
  *
  * Formulas the pages leave open are fixed by this library as:
  *   summary   s = (1/16) sum_r sum_c softmax_c(R_r . x_c / sqrt(d)) x_c over the
@@ -123,8 +124,9 @@ zha_status zha_workspace_bytes(const zha_config* cfg, int32_t op, int64_t max_qu
                                size_t* bytes);
 
 /* Build every complete node of every level for the first seq_len[b] tokens of
- * each sequence (lefilia.fr page, par. 1: blocks summarised, then grouped
- * level by level). Nodes that are not complete are left untouched. */
+ * each sequence (lefilia.fr page, par. 1: blocks are summarised, then each
+ * higher level summarises groups of b nodes below). Nodes that are not
+ * complete are left untouched. */
 zha_status zha_build_tree(const zha_config* cfg, const zha_cache* cache, void* stream);
 
 /* Build exactly the nodes that became complete when sequence b grew from

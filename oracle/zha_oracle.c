@@ -11,7 +11,8 @@
  *             the KV cache stays complete and the tree only decides which keys
  *             a query reads; keys are cut into contiguous blocks, each block is
  *             summarised by one key derived from 16 learned reference queries,
- *             and blocks are grouped level by level; a query scores the top
+ *             and each higher level summarises groups of b nodes of the level
+ *             below; a query scores the top
  *             nodes, keeps the fewest nodes whose estimated attention mass
  *             reaches the fraction p, descends only into the kept branches
  *             until it reaches individual keys, and always keeps token 0.

@@ -170,6 +170,31 @@ def _hand():
     return g, K, V
 
 
+def _arith(expr: str, names: dict) -> float:
+    """Value of a fixture's closed form: numbers, the given names, + - * / and
+    parentheses only."""
+    import ast
+    import operator
+
+    ops = {ast.Add: operator.add, ast.Sub: operator.sub, ast.Mult: operator.mul,
+           ast.Div: operator.truediv}
+
+    def ev(n):
+        if isinstance(n, ast.Expression):
+            return ev(n.body)
+        if isinstance(n, ast.BinOp) and type(n.op) in ops:
+            return ops[type(n.op)](ev(n.left), ev(n.right))
+        if isinstance(n, ast.UnaryOp) and isinstance(n.op, ast.USub):
+            return -ev(n.operand)
+        if isinstance(n, ast.Constant) and isinstance(n.value, (int, float)):
+            return float(n.value)
+        if isinstance(n, ast.Name) and n.id in names:
+            return names[n.id]
+        raise ValueError(f"unsupported expression: {expr}")
+
+    return ev(ast.parse(expr, mode="eval"))
+
+
 def test_hand_example():
     g, K, V = _hand()
     tr = oracle.build_tree(K, 16, np.zeros((16, g["d"]), np.float32), g["b"], g["L"], False)
@@ -182,7 +207,7 @@ def test_hand_example():
         assert idx.tolist() == case["S"], case["p"]
         assert counts.tolist() == case["level_counts"], case["p"]
         o = oracle.attend(q, K, V, idx)
-        o0 = eval(case["o0"], {"E2": e2, "E4": e4})
+        o0 = _arith(case["o0"], {"E2": e2, "E4": e4})
         assert abs(o[0] - o0) < 1e-12 and abs(o[1] - 1.0) < 1e-12
 
 
