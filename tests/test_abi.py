@@ -147,3 +147,16 @@ def test_bench_selection_per_query():
     # summary rows 2 + 4 * 2 and 2 + 4 * 1; K and V rows plus two 4-byte
     # index entries per selected token
     assert r["bytes_per_q_head_sum"] == (10 + 6) * 256 + (17 + 21) * (512 + 8)
+
+
+def test_binding_refuses_host_tensors(z):
+    # every pointer the library takes is device memory: a host tensor is
+    # refused in the binding, before any call into the library
+    with pytest.raises(ValueError, match="device"):
+        z._ptr(torch.zeros(4))
+    cfg = z.make_config(64, 4, 3, 1, 1, 1, 1024, torch.float32)
+    host = z.Cache(torch.zeros(1, 1, 1024, 64), torch.zeros(1, 1, 1024, 64),
+                   torch.zeros(16, 64), torch.zeros(8), torch.zeros(1, dtype=torch.int32))
+    with pytest.raises(ValueError, match="cache.k"):
+        z.zha_build_tree(cfg, host)
+    assert z._ptr(None) is None

@@ -127,12 +127,20 @@ def _check(fn: str, status: int):
         raise ZhaError(fn, status)
 
 
+def _device_tensor(t: torch.Tensor, what: str = "tensor") -> torch.Tensor:
+    """Every pointer the library takes is CUDA device memory read or written by
+    its kernels: a host tensor is refused here, before any launch."""
+    if not t.is_cuda:
+        raise ValueError(f"libzha takes CUDA device tensors; {what} is on {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"libzha needs contiguous tensors; {what} is not")
+    return t
+
+
 def _ptr(t: Optional[torch.Tensor]):
     if t is None:
         return None
-    if not t.is_contiguous():
-        raise ValueError("libzha needs contiguous tensors")
-    return ctypes.c_void_p(t.data_ptr())
+    return ctypes.c_void_p(_device_tensor(t).data_ptr())
 
 
 def _stream(stream) -> ctypes.c_void_p:
@@ -155,6 +163,8 @@ class Cache:
     seq_len: torch.Tensor     # [B] int32
 
     def c(self) -> zha_cache:
+        for name in ("k", "v", "r", "tree", "seq_len"):
+            _device_tensor(getattr(self, name), f"cache.{name}")
         return zha_cache(self.k.data_ptr(), self.v.data_ptr(), self.r.data_ptr(),
                          self.tree.data_ptr(), self.seq_len.data_ptr())
 
