@@ -128,10 +128,14 @@ def _check(fn: str, status: int):
 
 
 def _device_tensor(t: torch.Tensor, what: str = "tensor") -> torch.Tensor:
-    """Every pointer the library takes is CUDA device memory read or written by
-    its kernels: a host tensor is refused here, before any launch."""
+    """Every pointer the library takes is memory of the current CUDA device,
+    read or written by its kernels: a host tensor, or one on another device, is
+    refused here, before any launch."""
     if not t.is_cuda:
         raise ValueError(f"libzha takes CUDA device tensors; {what} is on {t.device}")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"libzha launches on the current device "
+                         f"(cuda:{torch.cuda.current_device()}); {what} is on {t.device}")
     if not t.is_contiguous():
         raise ValueError(f"libzha needs contiguous tensors; {what} is not")
     return t
