@@ -998,7 +998,7 @@ __device__ __forceinline__ bool keep_rule(int mode, unsigned kthr, uint32_t key,
 }
 
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads, 2) traverse_kernel(TravParams p) {
+__global__ void __launch_bounds__(kThreads, 2) traverse_kernel(const __grid_constant__ TravParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   Smem& S = *reinterpret_cast<Smem*>(smem_raw);
   cg::cluster_group cluster = cg::this_cluster();
