@@ -19,6 +19,7 @@ One JSON line on rank 0. Under torchrun every rank runs an independent replica
 --impl reference times the CPU oracle on the same metric (a bounded sample).
 """
 import argparse
+import datetime
 import hashlib
 import json
 import os
@@ -787,7 +788,7 @@ def main():
             run_sweep(args, dev)
         return
     if world > 1:
-        torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     prefill = is_prefill(args.workload)
