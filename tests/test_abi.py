@@ -160,3 +160,28 @@ def test_binding_refuses_host_tensors(z):
     with pytest.raises(ValueError, match="cache.k"):
         z.zha_build_tree(cfg, host)
     assert z._ptr(None) is None
+
+
+def test_bench_clock_sampler_parses_nvidia_smi(tmp_path, monkeypatch):
+    import importlib
+    import sys
+    import time
+
+    sys.path.insert(0, ROOT)
+    bench = importlib.import_module("bench")
+    fake = tmp_path / "nvidia-smi"
+    fake.write_text("#!/bin/sh\n"
+                    "echo '0, 1965, 1965, 700.1, 0x0, Not Active, Not Active, Not Active, Not Active'\n"
+                    "echo '0, 1800, 1965, 990.5, 0x4, Not Active, Not Active, Not Active, Active'\n"
+                    "echo '0, 1900, 1965, 950.0, 0x4, Not Active, Not Active, Not Active, Active'\n"
+                    "echo 'garbled line'\n"
+                    "exec sleep 30\n")
+    fake.chmod(0o755)
+    monkeypatch.setenv("PATH", f"{tmp_path}:{os.environ['PATH']}")
+    s = bench.ClockSampler(0)
+    s.start()
+    deadline = time.time() + 10
+    while len(s.lines) < 4 and time.time() < deadline:
+        time.sleep(0.05)
+    r = s.stop()
+    assert r == {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
