@@ -185,3 +185,32 @@ def test_bench_clock_sampler_parses_nvidia_smi(tmp_path, monkeypatch):
         time.sleep(0.05)
     r = s.stop()
     assert r == {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+
+
+def _ptxas_frame(report: str, mangled_part: str):
+    """(stack frame bytes, spill store bytes) of the kernel whose mangled name
+    contains mangled_part, from a ptxas -v report."""
+    lines = report.splitlines()
+    for i, ln in enumerate(lines):
+        if "Function properties for" in ln and mangled_part in ln and i + 1 < len(lines):
+            m = re.search(r"(\d+) bytes stack frame, (\d+) bytes spill stores", lines[i + 1])
+            if m:
+                return int(m.group(1)), int(m.group(2))
+    return None
+
+
+def test_traversal_stack_frame_stays_small(z):
+    # The traversal hands its parameter block by reference to non-inlined
+    # helpers; unless the parameter is grid-constant, every thread copies the
+    # whole block to its stack at launch (a 784-byte frame for the bf16,
+    # d = 128, 8-head instance, against 304 bytes with it).
+    from tree_indexed_sparse_zha_b200 import build as B
+
+    path = B.ptxas_report_path(os.path.join(B.CSRC, "traverse.cu"))
+    if not os.path.exists(path):
+        B.build(force=True)
+    with open(path) as f:
+        report = f.read()
+    frame = _ptxas_frame(report, "traverse_kernelI13__nv_bfloat16Li128ELi8E")
+    assert frame is not None, "traverse_kernel<bf16, 128, 8> missing from the ptxas report"
+    assert frame[0] <= 384 and frame[1] <= 64, frame

@@ -24,6 +24,10 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
+def ptxas_report_path(src: str) -> str:
+    return os.path.join(OBJ_DIR, os.path.basename(src) + ".ptxas.txt")
+
+
 def needs_build() -> bool:
     if not os.path.exists(LIB):
         return True
@@ -41,11 +45,19 @@ def build(force: bool = False, verbose: bool = False) -> str:
     nvcc = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
     os.makedirs(OBJ_DIR, exist_ok=True)
     inc = ["-I", os.path.join(ROOT, "include")]
-    extra = ["-Xptxas=-v"] if verbose else []
 
     def compile_one(src):
+        # ptxas's resource report (registers, stack frame, spills per kernel)
+        # is kept beside the object as <source>.ptxas.txt
         obj = os.path.join(OBJ_DIR, os.path.basename(src) + ".o")
-        subprocess.check_call([nvcc, *NVCC_FLAGS, *extra, *inc, "-c", src, "-o", obj])
+        r = subprocess.run([nvcc, *NVCC_FLAGS, "-Xptxas=-v", *inc, "-c", src, "-o", obj],
+                           capture_output=True, text=True)
+        with open(ptxas_report_path(src), "w") as f:
+            f.write(r.stderr)
+        if verbose or r.returncode:
+            sys.stderr.write(r.stdout + r.stderr)
+        if r.returncode:
+            raise subprocess.CalledProcessError(r.returncode, r.args)
         return obj
 
     with ThreadPoolExecutor(max_workers=len(sources())) as ex:
