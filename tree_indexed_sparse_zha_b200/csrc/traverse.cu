@@ -40,6 +40,8 @@
 //   z = (dot(q, s) * inv_sqrt_d) + fp32(l ln b),  M = trunc(exp(z - zmax) 2^40),
 //   need = ceil(T p_q / 2^32); keep the shortest prefix of (z desc, node asc)
 //   whose mass reaches need (every candidate when p_q >= 2^32).
+#include <atomic>
+
 #include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -1759,21 +1761,25 @@ int max_clusters_g(int G, int C) {
   }
 }
 
+// Cached per (dtype, d, G, C) for the process; every device is assumed to be
+// the same part. Calls from several host threads may query concurrently and
+// store the same value, so the cache entries are relaxed atomics.
 int max_clusters(const Geometry& g, int C) {
-  static int cache[2][2][4][kMaxCluster + 1];  // dtype, d, G, C (0 = not queried)
+  static std::atomic<int> cache[2][2][4][kMaxCluster + 1];  // 0 = not queried
   const int i0 = g.dtype == ZHA_BF16, i1 = g.d == 128;
   const int i2 = g.G == 1 ? 0 : g.G == 2 ? 1 : g.G == 4 ? 2 : 3;
-  int& v = cache[i0][i1][i2][C];
-  if (v == 0) {
-    int n;
+  std::atomic<int>& v = cache[i0][i1][i2][C];
+  int n = v.load(std::memory_order_relaxed);
+  if (n == 0) {
     if (g.dtype == ZHA_BF16)
       n = g.d == 128 ? max_clusters_g<__nv_bfloat16, 128>(g.G, C)
                      : max_clusters_g<__nv_bfloat16, 64>(g.G, C);
     else
       n = g.d == 128 ? max_clusters_g<float, 128>(g.G, C) : max_clusters_g<float, 64>(g.G, C);
-    v = n > 0 ? n : -1;
+    if (n <= 0) n = -1;
+    v.store(n, std::memory_order_relaxed);
   }
-  return v;
+  return n;
 }
 
 }  // namespace
