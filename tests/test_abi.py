@@ -47,6 +47,13 @@ def test_tree_layout_host_only(z):
 def test_status_strings(z):
     assert z.status_string(0) == "ok"
     assert "capacity" in z.status_string(z.ZHA_ERR_CAPACITY)
+    codes = [z.ZHA_ERR_INVALID_ARG, z.ZHA_ERR_UNSUPPORTED, z.ZHA_ERR_CUDA, z.ZHA_ERR_CAPACITY,
+             z.ZHA_ERR_WORKSPACE, z.ZHA_ERR_TIMEOUT, z.ZHA_ERR_INTERNAL]
+    texts = [z.status_string(c) for c in codes]
+    assert len(set(texts)) == len(codes) and "unknown status" not in texts
+    # device statuses are OR-ed flags: any set flag is named, the lowest first
+    assert z.status_string(z.ZHA_ERR_TIMEOUT | z.ZHA_ERR_CAPACITY) == texts[3]
+    assert z.status_string(1 << 20) == "unknown status"
 
 
 @pytest.mark.parametrize("field,value,code", [
