@@ -152,6 +152,23 @@ def strip_c_comments(src: str) -> str:
     return " ".join("".join(out).split())
 
 
+def decode_step_bytes(cand_rows: int, kept_nodes: int, b: int, tail: int, units: int,
+                      queries: int, row: int):
+    """Algorithmic bytes of one decode step, counted once per unit (a sequence
+    and KV head, whose query heads share every read), with rows of `row` bytes:
+    - selection: the distinct summary rows scored, the kept level-1 node list
+      written (4 bytes per node), and the query rows read and the output rows
+      written;
+    - attention: the K and V rows of the kept nodes' tokens, the causal tail
+      and token 0, the kept node list read back, and the query and output rows.
+    Token 0 is counted once per unit even when its node is kept, at most one
+    row over per unit. Returns (selection bytes, attention bytes, K/V rows)."""
+    kv_rows = kept_nodes * b + units * (1 + tail)
+    sel = cand_rows * row + kept_nodes * 4 + 2 * queries * row
+    att = kv_rows * 2 * row + kept_nodes * 4 + 2 * queries * row
+    return sel, att, kv_rows
+
+
 def selection_per_query(lc, b: int, L: int, n: int, row: int) -> dict:
     """Per-query selection figures from kept counts lc [B][Hq][L] (top level
     first) of decode queries at position n - 1, with summary and K/V rows of
@@ -417,14 +434,13 @@ def run_zha(args, rank, world, dev):
     row = D * 2
     cand_rows = int(stats[:, :L].sum())
     kept_nodes = int(stats[:, L].sum())
-    kv_rows = kept_nodes * b + B * Hkv * (1 + tail)
+    sel_bytes, att_bytes, kv_rows = decode_step_bytes(cand_rows, kept_nodes, b, tail, B * Hkv,
+                                                      queries_per_step, row)
     # per-query kept counts of the last step's queries: one more select, untimed
     lc = torch.zeros(B, Hq, L, dtype=torch.int32, device=dev)
     z.zha_decode_select(cfg, cache, step_inputs(args.warmup + args.steps - 1)[3], c.p, lc, ws, st)
     torch.cuda.synchronize()
     per_query = selection_per_query(lc.cpu(), b, L, n_last, D * 2)
-    sel_bytes = cand_rows * row + kept_nodes * 4 + 2 * queries_per_step * row
-    att_bytes = kv_rows * 2 * row + kept_nodes * 4 + 2 * queries_per_step * row
     ext_bytes = 0
     step_bytes = sel_bytes + att_bytes + ext_bytes
     peak, peak_kind = measured_peaks()

@@ -221,3 +221,21 @@ def test_traversal_stack_frame_stays_small(z):
     frame = _ptxas_frame(report, "traverse_kernelI13__nv_bfloat16Li128ELi8E")
     assert frame is not None, "traverse_kernel<bf16, 128, 8> missing from the ptxas report"
     assert frame[0] <= 384 and frame[1] <= 64, frame
+
+
+def test_bench_decode_step_bytes():
+    import importlib
+    import sys
+
+    sys.path.insert(0, ROOT)
+    bench = importlib.import_module("bench")
+    # by hand: 2 units, b = 4, 10 kept level-1 nodes, a tail of 3 tokens,
+    # 100 summary rows, 16 queries, 256-byte rows
+    sel, att, kv = bench.decode_step_bytes(100, 10, 4, 3, 2, 16, 256)
+    assert kv == 10 * 4 + 2 * (1 + 3)
+    assert sel == 100 * 256 + 10 * 4 + 2 * 16 * 256
+    assert att == kv * 512 + 10 * 4 + 2 * 16 * 256
+    # the counts of a measured 256K decode step (16 units, 128 queries) give
+    # the bytes that step reported
+    sel, att, kv = bench.decode_step_bytes(1397720, 1048300, 4, 205, 16, 128, 256)
+    assert kv == 4196496 and sel + att == 2514939744
