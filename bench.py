@@ -733,12 +733,10 @@ def run_sweep(args, dev):
         top = n_tok // b ** L
         tail = n_tok - b ** L * top
         kept = int(stats[:, L].sum())
-        kv_rows = kept * b + units * (1 + tail)
-        # as the main bench: summary rows, kept-node indices read by both
-        # halves, selected K+V rows, and the query rows in and out of each half
-        touched = (int(stats[:, :L].sum()) * row + 2 * kept * 4 + kv_rows * 2 * row
-                   + 4 * c.batch * c.n_q_heads * row)
         q = c.batch * c.n_q_heads
+        sel_b, att_b, kv_rows = decode_step_bytes(int(stats[:, :L].sum()), kept, b, tail, units,
+                                                  q, row)
+        touched = sel_b + att_b
         line = {"sweep": WORKLOAD, "block": b, "levels": L, "top_span": b ** L,
                 "context": n_tok, "p": c.p, "steps": steps,
                 "ms_per_step": ms, "queries_per_s": q / (ms / 1e3),
