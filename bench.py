@@ -157,14 +157,14 @@ def decode_step_bytes(cand_rows: int, kept_nodes: int, b: int, tail: int, units:
     """Algorithmic bytes of one decode step, counted once per unit (a sequence
     and KV head, whose query heads share every read), with rows of `row` bytes:
     - selection: the distinct summary rows scored, the kept level-1 node list
-      written (4 bytes per node), and the query rows read and the output rows
-      written;
+      written (4 bytes per node) and the query rows read;
     - attention: the K and V rows of the kept nodes' tokens, the causal tail
-      and token 0, the kept node list read back, and the query and output rows.
+      and token 0, the kept node list read back, the query rows read and the
+      output rows written.
     Token 0 is counted once per unit even when its node is kept, at most one
     row over per unit. Returns (selection bytes, attention bytes, K/V rows)."""
     kv_rows = kept_nodes * b + units * (1 + tail)
-    sel = cand_rows * row + kept_nodes * 4 + 2 * queries * row
+    sel = cand_rows * row + kept_nodes * 4 + queries * row
     att = kv_rows * 2 * row + kept_nodes * 4 + 2 * queries * row
     return sel, att, kv_rows
 
@@ -286,6 +286,131 @@ def oracle_prefill_rate(wl, n_queries: int, budget_s: float = 20.0):
     return done / el, done, el, flagged
 
 
+def host_cpu():
+    """(usable host cores, CPU model name)."""
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return max(1, cores), model
+
+
+def _widen_bf16(raw):
+    import numpy as np
+
+    return (raw.view(np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def _oracle_worker(shm_name, shape, R, n_tree, b, L, cap, p, warm, steps, barrier, out_q):
+    """One host core: rebuilds the unit's tree with the oracle and runs its
+    warm-up steps (untimed), waits for every worker, then runs select + fp64
+    attention over its timed steps."""
+    import numpy as np
+    from multiprocessing import shared_memory
+
+    import oracle
+
+    shm = shared_memory.SharedMemory(name=shm_name)
+    try:
+        n = int(np.prod(shape))
+        raw = np.ndarray((2 * n,), dtype=np.int16, buffer=shm.buf)
+        K = _widen_bf16(raw[:n].copy()).reshape(shape)
+        V = _widen_bf16(raw[n:].copy()).reshape(shape)
+    finally:
+        shm.close()
+    tr = oracle.build_tree(K, n_tree, R, b, L, True, cap)
+    for step in warm:
+        for q, t in step:
+            oracle.attend(q, K, V, oracle.select(q, tr, t, p)[0])
+    barrier.wait()
+    t0 = time.perf_counter()
+    done = flagged = 0
+    for step in steps:
+        for q, t in step:
+            idx, _, _, tie = oracle.select(q, tr, t, p)
+            oracle.attend(q, K, V, idx)
+            done += 1
+            flagged += tie
+    out_q.put((done, time.perf_counter() - t0, flagged))
+
+
+def oracle_steps_parallel(wl, steps, n_tree, workers, warm=()):
+    """Times the CPU oracle over `steps` (each a list of (q fp32[d], t)
+    queries of sequence 0 / KV head 0) on `workers` host processes at once,
+    steps dealt round-robin. A harness around the oracle, not oracle code:
+    each worker rebuilds the unit's tree untimed, then all start together.
+    Returns (queries done, wall seconds of the timed part, queries flagged
+    near-tie)."""
+    import multiprocessing as mp
+    from multiprocessing import shared_memory
+
+    c = wl.cfg
+    K = wl.K[0, 0].cpu().contiguous().view(torch.int16).numpy()
+    V = wl.V[0, 0].cpu().contiguous().view(torch.int16).numpy()
+    R = wl.R.float().cpu().numpy()
+    shm = shared_memory.SharedMemory(create=True, size=K.nbytes + V.nbytes)
+    procs = []
+    try:
+        buf = memoryview(shm.buf)
+        buf[:K.nbytes] = K.tobytes()
+        buf[K.nbytes:K.nbytes + V.nbytes] = V.tobytes()
+        del buf
+        ctx = mp.get_context("spawn")  # never fork a process holding a CUDA context
+        barrier = ctx.Barrier(workers + 1)
+        out_q = ctx.Queue()
+        for w in range(workers):
+            pr = ctx.Process(target=_oracle_worker,
+                             args=(shm.name, K.shape, R, n_tree, c.block, c.levels, c.capacity,
+                                   c.p, list(warm[w::workers]), steps[w::workers], barrier,
+                                   out_q))
+            pr.start()
+            procs.append(pr)
+        barrier.wait(timeout=900)
+        t0 = time.perf_counter()
+        res = [out_q.get(timeout=1800) for _ in range(workers)]
+        el = time.perf_counter() - t0
+        for pr in procs:
+            pr.join(timeout=60)
+    finally:
+        for pr in procs:
+            if pr.is_alive():
+                pr.kill()
+        shm.close()
+        shm.unlink()
+    return sum(r[0] for r in res), el, sum(r[2] for r in res)
+
+
+def decode_oracle_steps(wl, n_steps):
+    """Reference-arm steps of the decode workload: step s is the G query heads
+    of sequence 0 / KV head 0 at decode step s (one sixteenth of a workload
+    step's queries)."""
+    c = wl.cfg
+    out = []
+    for s in range(1, n_steps + 1):
+        q = wl.queries(((s - 1) % max(c.steps, 1)) + 1)[0].float().cpu().numpy()
+        t = c.n_tokens + ((s - 1) % max(c.steps, 1))
+        out.append([(q[h], t) for h in range(c.group)])
+    return out
+
+
+def prefill_oracle_steps(wl, n_steps):
+    """Reference-arm steps of the prefill workload: step i is the G query heads
+    of KV head 0 for chunk token i."""
+    c = wl.cfg
+    q = wl.queries(0).float().cpu().numpy()
+    return [[(q[i % c.chunk, h], c.n_tokens + i % c.chunk) for h in range(c.group)]
+            for i in range(n_steps)]
+
+
 # ---------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------
@@ -332,6 +457,117 @@ def workload_config(args, c):
             "queries_per_step": c.batch * c.n_q_heads, "l2": l2_note(kv_gb)}
 
 
+def tree_build_work(n_tokens: int, b: int, L: int, D: int, units: int, elem: int = 2):
+    """Algorithmic work of building every complete node over n_tokens tokens of
+    `units` (sequence, KV head) units: (bytes, flops). Bytes: the keys read,
+    every summary row read as a child of the level above, every summary row
+    written. Flops: per child of a node, 16 reference-query dot products of
+    length D and its share of the weighted sum (D), two flops per FMA."""
+    rows = [units * (n_tokens // b ** l) for l in range(1, L + 1)]
+    children = units * n_tokens + sum(rows[:-1])  # inputs of levels 1..L
+    nbytes = (units * n_tokens + sum(rows[:-1]) + sum(rows)) * D * elem
+    flops = 2.0 * (16 * D + D) * children
+    return nbytes, flops
+
+
+def fp32_peak_tflops(dev) -> float:
+    """FP32 FMA peak of the device at its top SM clock: SMs x 128 lanes x 2 flops."""
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    return sms * 128 * 2 * 1.965e9 / 1e12
+
+
+def time_tree_build(cfg, cache, stream, reps: int = 3) -> float:
+    import tree_indexed_sparse_zha_b200 as z
+
+    z.zha_build_tree(cfg, cache)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+    e0.record(stream)
+    for _ in range(reps):
+        z.zha_build_tree(cfg, cache)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def tree_builds_other_workloads(dev, peak_gbs: float) -> dict:
+    """Tree-build rate of the other workloads' caches (the 32K decode, the wide
+    256K tree and the 1M-token prefill context), built from scratch."""
+    import tree_indexed_sparse_zha_b200 as z
+    from tree_indexed_sparse_zha_b200 import workloads as W
+
+    out = {}
+    stream = torch.cuda.current_stream()
+    for name in ("decode-deep-32k", "decode-wide-256k-b8", "prefill-deep-1m-chunk4k"):
+        wl = W.make(name, device=dev, steps=0, chunk=0)
+        c = wl.cfg
+        cfg = z.make_config(c.head_dim, c.block, c.levels, c.n_q_heads, c.n_kv_heads, c.batch,
+                            c.capacity, c.torch_dtype)
+        cache = z.Cache(wl.K, wl.V, wl.R.float().contiguous(), z.alloc_tree(cfg, dev),
+                        wl.seq_len.clone())
+        ms = time_tree_build(cfg, cache, stream)
+        nbytes, flops = tree_build_work(c.n_tokens, c.block, c.levels, c.head_dim,
+                                        c.batch * c.n_kv_heads)
+        out[name] = {"ms": ms, "tokens": c.batch * c.n_kv_heads * c.n_tokens,
+                     "gb_per_s": nbytes / (ms / 1e3) / 1e9,
+                     "hbm_frac": nbytes / (ms / 1e3) / 1e9 / peak_gbs,
+                     "tflops": flops / (ms / 1e3) / 1e12,
+                     "fp32_frac": flops / (ms / 1e3) / 1e12 / fp32_peak_tflops(dev)}
+        del wl, cache
+        torch.cuda.empty_cache()
+    return out
+
+
+def wide_p_sweep(dev, peak: float, steps: int = 20, warmup: int = 3) -> list:
+    """The wide-tree 256K workload (b = 256, one level, 8 sequences): decode
+    steps (select + attend) at every p of its sweep, queries/s and the HBM
+    fraction of the bytes each step touches."""
+    import tree_indexed_sparse_zha_b200 as z
+    from tree_indexed_sparse_zha_b200 import workloads as W
+
+    wl = W.make("decode-wide-256k-b8", device=dev)
+    c = wl.cfg
+    cfg = z.make_config(c.head_dim, c.block, c.levels, c.n_q_heads, c.n_kv_heads, c.batch,
+                        c.capacity, c.torch_dtype)
+    cache = z.Cache(wl.K, wl.V, wl.R.float().contiguous(), z.alloc_tree(cfg, dev),
+                    wl.seq_len.clone())
+    z.zha_build_tree(cfg, cache)
+    ws = z.alloc_workspace(cfg, z.ZHA_OP_DECODE, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    q = wl.queries(0)
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+    B, Hq, Hkv, D, b, L = c.batch, c.n_q_heads, c.n_kv_heads, c.head_dim, c.block, c.levels
+    n = c.n_tokens
+    res = []
+    for p in c.p_sweep:
+        for _ in range(warmup):
+            z.zha_decode(cfg, cache, q, p, out, None, ws, st)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(steps):
+            z.zha_decode(cfg, cache, q, p, out, None, ws, st)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        stats = torch.zeros(B * Hkv, L + 1, dtype=torch.int32, device=dev)
+        z.zha_decode_stats(cfg, ws, stats)
+        stats = stats.cpu()
+        top = n // b ** L
+        sel_b, att_b, kv_rows = decode_step_bytes(int(stats[:, :L].sum()), int(stats[:, L].sum()),
+                                                  b, n - b ** L * top, B * Hkv, B * Hq, D * 2)
+        res.append({"p": p, "ms_per_step": ms, "queries_per_s": B * Hq / (ms / 1e3),
+                    "bytes_touched_per_step": sel_b + att_b,
+                    "kv_fraction_read": kv_rows / (B * Hkv * n),
+                    "hbm_frac": (sel_b + att_b) / (ms / 1e3) / 1e9 / peak})
+    if int(st.item()) != 0:
+        raise RuntimeError(f"wide sweep: device status {z.status_string(int(st.item()))}")
+    del cache, ws, wl
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_zha(args, rank, world, dev):
     import tree_indexed_sparse_zha_b200 as z
     from tree_indexed_sparse_zha_b200 import workloads as W
@@ -365,9 +601,7 @@ def run_zha(args, rank, world, dev):
     torch.cuda.synchronize()
     build_ms = e0.elapsed_time(e1)
     n_tok = B * Hkv * c.n_tokens
-    sum_rows = sum(B * Hkv * (c.n_tokens // b ** l) for l in range(1, L + 1))
-    build_bytes = (n_tok + sum_rows * 2 - B * Hkv * (c.n_tokens // b ** L)) * D * 2
-    build_flops = 2.0 * 16 * D * (n_tok + sum_rows - B * Hkv * (c.n_tokens // b ** L))
+    build_bytes, build_flops = tree_build_work(c.n_tokens, b, L, D, B * Hkv)
 
     def step_inputs(i):
         s = (i % n_steps_cap) + 1  # wrap: rebuilt nodes are identical
@@ -524,12 +758,16 @@ def run_zha(args, rank, world, dev):
                   "hbm_frac": dense_bytes / (dense_ms / 1e3) / 1e9 / peak},
         "tree_build": {"ms": build_ms, "gb_per_s": build_bytes / (build_ms / 1e3) / 1e9,
                        "tflops": build_flops / (build_ms / 1e3) / 1e12,
+                       "fp32_frac": build_flops / (build_ms / 1e3) / 1e12 / fp32_peak_tflops(dev),
                        "tokens": n_tok},
         "e2e": {"value": queries_per_step * world / (e2e_ms / 1e3), "unit": "queries/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "gpu_launches": 4 * args.steps,
         "clocks": clocks,
     }
+    if args.n_tokens is None:  # the other workloads at their full sizes
+        res["decode_wide_p_sweep"] = wide_p_sweep(dev, peak)
+        res["tree_build_other_workloads"] = tree_builds_other_workloads(dev, peak)
     return res, wl
 
 
@@ -750,6 +988,30 @@ def run_sweep(args, dev):
         torch.cuda.empty_cache()
 
 
+def cpu_baseline(wl, prefill: bool) -> dict:
+    """The oracle on the host: every usable core at once (a bounded sample,
+    a few steps per process), beside one core as the oracle stands."""
+    c = wl.cfg
+    cores, model = host_cpu()
+    workers = min(cores, 8 if prefill else 32)
+    steps = (prefill_oracle_steps if prefill else decode_oracle_steps)(wl, 3 * workers)
+    n_tree = c.n_tokens + c.chunk if prefill else c.n_tokens
+    done, el, flagged = oracle_steps_parallel(wl, steps, n_tree, workers)
+    if prefill:
+        r1, d1, e1, f1 = oracle_prefill_rate(wl, 200, budget_s=15.0)
+        what = "chunk queries of KV head 0"
+    else:
+        r1, d1, e1, f1 = oracle_rate(wl, 200, budget_s=15.0)
+        what = "decode queries of sequence 0 / KV head 0"
+    return {"value": done / el, "unit": "queries/s", "cores": workers, "cpu_model": model,
+            "host_cores": cores, "kind": "oracle", "near_tie_flagged": flagged,
+            "sample": f"{done} {what} on {workers} processes in {el:.1f} s (trees built "
+                      "untimed)",
+            "single_core": {"value": r1, "unit": "queries/s", "cores": 1,
+                            "near_tie_flagged": f1,
+                            "sample": f"{d1} {what} in {e1:.1f} s (tree built untimed)"}}
+
+
 def main():
     args = parse()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -763,36 +1025,36 @@ def main():
         dev = "cuda" if torch.cuda.is_available() else "cpu"
         wl = W.make(args.workload, device=dev, n_tokens=args.n_tokens)
         c = wl.cfg
-        if is_prefill(args.workload):
-            rate, done, el, flagged = oracle_prefill_rate(wl, args.steps, budget_s=180.0)
-            line = {"impl": "reference", "metric": PREFILL_METRIC, "value": rate,
-                    "unit": "queries/s", "n_gpus": 1, "steps": args.steps,
-                    "warmup": args.warmup,
-                    "ms_per_step": el / done * c.chunk * c.n_q_heads * 1e3,
-                    "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                    "dtype": "f32 select / f64 attention", "data": "synthetic",
-                    "config": workload_config(args, c),
-                    "cpu_baseline": {"value": rate, "unit": "queries/s", "cores": 1,
-                                     "kind": "oracle", "near_tie_flagged": flagged,
-                                     "sample": f"{done} chunk queries (query heads of KV head "
-                                               f"0) in {el:.1f} s, tree built untimed"},
-                    "e2e": {"value": rate, "unit": "queries/s", "h2d_bytes_per_step": 0,
-                            "d2h_bytes_per_step": 0}}
-            print(json.dumps(line), flush=True)
-            return
-        oracle_rate(wl, min(args.warmup, 2), budget_s=60.0)  # warm-up
-        rate, done, el, flagged = oracle_rate(wl, args.steps, budget_s=180.0)
-        line = {"impl": "reference", "metric": METRIC, "value": rate, "unit": "queries/s",
-                "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": el / done * c.batch * c.n_q_heads * 1e3,
-                "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "f32 select / f64 attention",
-                "data": "synthetic", "config": workload_config(args, c),
-                "cpu_baseline": {"value": rate, "unit": "queries/s", "cores": 1,
-                                 "kind": "oracle", "near_tie_flagged": flagged,
-                                 "sample": f"{done} queries (the query heads of KV head 0 of "
-                                           f"sequence 0, successive decode steps) in {el:.1f} s, "
-                                           "tree built untimed"},
+        cores, model = host_cpu()
+        prefill = is_prefill(args.workload)
+        # workers hold the unit's K/V in fp32 and its tree: about 0.6 GB each at
+        # 256K context, 1.5 GB at 1M
+        workers = min(cores, 8 if prefill else 32, max(args.steps, 1))
+        make_steps = prefill_oracle_steps if prefill else decode_oracle_steps
+        all_steps = make_steps(wl, args.warmup + args.steps)
+        n_tree = c.n_tokens + c.chunk if prefill else c.n_tokens
+        done, el, flagged = oracle_steps_parallel(wl, all_steps[args.warmup:], n_tree, workers,
+                                                  warm=all_steps[:args.warmup])
+        rate = done / el
+        step_desc = (f"the {c.group} query heads of KV head 0 for one chunk token"
+                     if prefill else
+                     f"the {c.group} query heads of sequence 0 / KV head 0 at one decode step")
+        frac = (f"1/{c.chunk * c.n_kv_heads} of a chunk's queries" if prefill
+                else f"1/{c.batch * c.n_kv_heads} of a workload step's queries")
+        line = {"impl": "reference", "metric": PREFILL_METRIC if prefill else METRIC,
+                "value": rate, "unit": "queries/s", "n_gpus": 1, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+                "step": f"{step_desc} ({frac}); steps dealt over {workers} host processes",
+                "queries_timed": done,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f32 select / f64 attention", "data": "synthetic",
+                "config": workload_config(args, c),
+                "cpu_baseline": {"value": rate, "unit": "queries/s", "cores": workers,
+                                 "cpu_model": model, "host_cores": cores, "kind": "oracle",
+                                 "near_tie_flagged": flagged,
+                                 "sample": f"{done} queries ({args.steps} steps of {step_desc}) "
+                                           f"in {el:.1f} s on {workers} processes, trees built "
+                                           "untimed"},
                 "e2e": {"value": rate, "unit": "queries/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
@@ -810,18 +1072,8 @@ def main():
     prefill = is_prefill(args.workload)
     res, wl = (run_prefill if prefill else run_zha)(args, rank, world, dev)
     if rank == 0:
-        if world == 1 and not args.no_cpu_baseline and prefill:
-            rate, done, el, flagged = oracle_prefill_rate(wl, 200, budget_s=20.0)
-            res["cpu_baseline"] = {"value": rate, "unit": "queries/s", "cores": 1, "kind": "oracle",
-                                   "near_tie_flagged": flagged,
-                                   "sample": f"{done} chunk queries of KV head 0 over {el:.1f} s "
-                                             "(tree built untimed)"}
-        elif world == 1 and not args.no_cpu_baseline:
-            rate, done, el, flagged = oracle_rate(wl, 200, budget_s=20.0)
-            res["cpu_baseline"] = {"value": rate, "unit": "queries/s", "cores": 1, "kind": "oracle",
-                                   "near_tie_flagged": flagged,
-                                   "sample": f"{done} queries of sequence 0 / KV head 0 over "
-                                             f"{el:.1f} s (tree built untimed)"}
+        if world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(wl, prefill)
         else:
             res["cpu_baseline"] = None
         print(json.dumps(res), flush=True)

@@ -130,7 +130,10 @@ zha_status zha_workspace_bytes(const zha_config* cfg, int32_t op, int64_t max_qu
 zha_status zha_build_tree(const zha_config* cfg, const zha_cache* cache, void* stream);
 
 /* Build exactly the nodes that became complete when sequence b grew from
- * old_len[b] (device int32) to seq_len[b] tokens. max_new_tokens is a host
+ * old_len[b] (device int32) to seq_len[b] tokens (lefilia.fr page, par. 1:
+ * the tree covers the whole cache, so a node is summarised as soon as its b
+ * children exist; the summary formula above is the same one the build uses).
+ * max_new_tokens is a host
  * upper bound on seq_len[b] - old_len[b] over all b (it sizes the launch);
  * growth beyond it is left unbuilt. */
 zha_status zha_extend_tree(const zha_config* cfg, const zha_cache* cache, const int32_t* old_len,
@@ -151,7 +154,9 @@ zha_status zha_select(const zha_config* cfg, const zha_cache* cache, const void*
                       void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
 
 /* Exact softmax attention of each query (i, h) over its list idx/n_idx (as
- * written by zha_select, ascending token positions of sequence q_seq[i]):
+ * written by zha_select, ascending token positions of sequence q_seq[i])
+ * (lefilia.fr page, par. 1: after the descent the query attends exactly over
+ * the raw K/V entries it selected; the cache itself is never pruned):
  * out[i][h] = sum_j softmax_j(q . k_j / sqrt(d)) v_j. fp32 accumulation.
  * ws/ws_bytes: ZHA_OP_ATTEND workspace for nq queries. */
 zha_status zha_attend(const zha_config* cfg, const zha_cache* cache, const void* q,
@@ -159,7 +164,9 @@ zha_status zha_attend(const zha_config* cfg, const zha_cache* cache, const void*
                       const int32_t* n_idx, void* out, void* ws, size_t ws_bytes,
                       int32_t* dev_status, void* stream);
 
-/* One decode step for every sequence: selection at position seq_len[b] - 1
+/* One decode step for every sequence (lefilia.fr page, par. 1 and 2: the
+ * top-p descent at p = 0.95 followed by exact attention over the selected raw
+ * keys, token 0 and the causal tail): selection at position seq_len[b] - 1
  * followed by attention over the selected keys, q [B][Hq][d] -> out [B][Hq][d].
  * The query heads sharing a KV head are traversed together and their
  * selections are read from HBM once (per-head masks). level_counts is
@@ -188,8 +195,11 @@ zha_status zha_decode_attend(const zha_config* cfg, const zha_cache* cache, cons
 zha_status zha_decode_stats(const zha_config* cfg, const void* ws, size_t ws_bytes,
                             int32_t* stats, void* stream);
 
-/* Chunked prefill of sequence `seq`: the caller has written the chunk's K and V
- * rows [chunk_start, chunk_start + T) and set seq_len[seq] = chunk_start + T.
+/* Chunked prefill of sequence `seq` (lefilia.fr page, par. 1: every query of
+ * the chunk descends the tree on its own and attends its selected keys,
+ * restricted causally to keys at or before its position): the caller has
+ * written the chunk's K and V rows [chunk_start, chunk_start + T) and set
+ * seq_len[seq] = chunk_start + T.
  * Extends the tree over the chunk, then for every token i of the chunk
  * (position chunk_start + i) and head h selects causally and attends:
  * q [T][Hq][d] -> out [T][Hq][d]. level_counts ([T][Hq][L]) is nullable.
@@ -233,10 +243,26 @@ zha_status zha_prefill_top_scores(const zha_config* cfg, const zha_cache* cache,
                                   int32_t* dev_status, void* stream);
 
 /* Dense flash-decoding over every key [0, seq_len[b] - 1] (the baseline the
- * sparse path is measured against): q [B][Hq][d] -> out [B][Hq][d].
+ * sparse path is measured against; lefilia.fr page, par. 2 and 4 compare the
+ * method with dense attention): q [B][Hq][d] -> out [B][Hq][d].
  * ws: ZHA_OP_DENSE workspace. */
 zha_status zha_dense_decode(const zha_config* cfg, const zha_cache* cache, const void* q,
                             void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* The token list each query head of the last zha_decode / zha_decode_select
+ * on ws attends (lefilia.fr page, par. 1: the raw keys under the kept
+ * level-1 nodes, plus the first token; the causal tail is the task's rule):
+ * for sequence s and head h, idx + (s*Hq + h)*idx_cap receives, ascending,
+ *   {0} U tokens of the level-1 nodes kept by h U [b^L T_top, seq_len[s] - 1]
+ * -- exactly the K/V rows zha_decode_attend reads for that head -- and
+ * n_idx[s*Hq + h] its length. It reads the kept level-1 node union and the
+ * per-head masks the traversal left in ws, so it must get the same cfg and
+ * cache (seq_len) and run after that selection with nothing touching ws in
+ * between. Lists longer than idx_cap are truncated and set ZHA_ERR_CAPACITY
+ * in *dev_status (nullable). idx, n_idx device int32. Asynchronous. */
+zha_status zha_decode_kept_lists(const zha_config* cfg, const zha_cache* cache, const void* ws,
+                                 size_t ws_bytes, int32_t* idx, int64_t idx_cap, int32_t* n_idx,
+                                 int32_t* dev_status, void* stream);
 
 /* zha_decode without a caller workspace. The pages describe no counterpart of
  * this call; it exists for callers that cannot hand the library a workspace --
@@ -250,7 +276,13 @@ zha_status zha_dense_decode(const zha_config* cfg, const zha_cache* cache, const
  *     (for example B = 1, Hkv = 2, G = 8, b = 4 fits up to about 180K tokens).
  *   - Set-up: the first call on each device looks up the array's device
  *     address (this loads its module on that device); make that first call
- *     with the device current and outside any stream capture.
+ *     with the device current and outside any stream capture. The address is
+ *     kept for the process, so the device must not be reset (cudaDeviceReset,
+ *     or its primary context destroyed) between calls.
+ *   - Memory: the 64 MiB are held on each device until the process exits.
+ *     Under the default lazy module loading only devices this entry point
+ *     ran on hold them; with CUDA_MODULE_LOADING=EAGER every process that
+ *     loads libzha holds them on every device it uses.
  *   - The scratch needs no clearing: every word is written before it is read.
  *   - Unlike the other entry points this one is NOT re-entrant: every call on
  *     a device shares the one array, so two calls whose executions overlap

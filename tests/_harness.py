@@ -51,14 +51,35 @@ class Gpu:
         assert st == 0, z.status_string(st)
 
     # -- calls ----------------------------------------------------------------
-    def decode(self, q: torch.Tensor, p: float):
+    def decode(self, q: torch.Tensor, p: float, lists: bool = False):
+        """zha_decode; with lists, also the per-head token lists the step's
+        attention read (zha_decode_kept_lists on the same workspace)."""
         c = self.c
         out = torch.empty_like(q)
         lc = torch.full((c.batch, c.n_q_heads, c.levels), -1, dtype=torch.int32, device=self.dev)
-        ws = z.alloc_workspace(self.cfg, z.ZHA_OP_DECODE, device=self.dev)
+        ws = self.decode_ws()
         z.zha_decode(self.cfg, self.cache, q, p, out, lc, ws, self.status)
         self.check_status()
-        return out.float().cpu().numpy(), lc.cpu().numpy()
+        if not lists:
+            return out.float().cpu().numpy(), lc.cpu().numpy()
+        idx, n_idx = self.kept_lists(ws)
+        return out.float().cpu().numpy(), lc.cpu().numpy(), idx, n_idx
+
+    def decode_ws(self) -> torch.Tensor:
+        if getattr(self, "_dws", None) is None:
+            self._dws = z.alloc_workspace(self.cfg, z.ZHA_OP_DECODE, device=self.dev)
+        return self._dws
+
+    def kept_lists(self, ws: torch.Tensor, cap: int = None):
+        """Per-head token lists [B][Hq][cap] and lengths [B][Hq] (device) of
+        the last decode selection on ws."""
+        c = self.c
+        cap = cap or int(self.cache.seq_len.max().item()) + 2
+        idx = torch.full((c.batch, c.n_q_heads, cap), -7, dtype=torch.int32, device=self.dev)
+        n_idx = torch.zeros(c.batch, c.n_q_heads, dtype=torch.int32, device=self.dev)
+        z.zha_decode_kept_lists(self.cfg, self.cache, ws, idx, n_idx, self.status)
+        self.check_status()
+        return idx, n_idx
 
     def dense(self, q: torch.Tensor):
         out = torch.empty_like(q)

@@ -28,7 +28,7 @@ def z():
 
 def test_exports_every_declared_symbol(z):
     names = _declared_functions()
-    assert len(names) == 15, names
+    assert len(names) == 16, names
     lib = z.lib()
     for n in names:
         assert hasattr(lib, n), n
@@ -80,6 +80,15 @@ def test_bad_arguments_rejected_before_launch(z):
         assert L.zha_decode(ctypes.byref(cfg), ctypes.byref(c), ctypes.c_void_p(16), p,
                             ctypes.c_void_p(16), None, ctypes.c_void_p(16), 1 << 40, None,
                             None) == z.ZHA_ERR_INVALID_ARG
+    # kept lists: null outputs, zero capacity and a short workspace
+    ws_need = z.zha_workspace_bytes(cfg, z.ZHA_OP_DECODE)
+    kl = L.zha_decode_kept_lists
+    assert kl(ctypes.byref(cfg), ctypes.byref(c), ctypes.c_void_p(16), ws_need, None, 8,
+              ctypes.c_void_p(16), None, None) == z.ZHA_ERR_INVALID_ARG
+    assert kl(ctypes.byref(cfg), ctypes.byref(c), ctypes.c_void_p(16), ws_need,
+              ctypes.c_void_p(16), 0, ctypes.c_void_p(16), None, None) == z.ZHA_ERR_INVALID_ARG
+    assert kl(ctypes.byref(cfg), ctypes.byref(c), ctypes.c_void_p(16), ws_need - 1,
+              ctypes.c_void_p(16), 8, ctypes.c_void_p(16), None, None) == z.ZHA_ERR_WORKSPACE
     # workspace too small
     assert L.zha_dense_decode(ctypes.byref(cfg), ctypes.byref(c), ctypes.c_void_p(16),
                               ctypes.c_void_p(16), ctypes.c_void_p(16), 1, None) == \
@@ -233,9 +242,9 @@ def test_bench_decode_step_bytes():
     # 100 summary rows, 16 queries, 256-byte rows
     sel, att, kv = bench.decode_step_bytes(100, 10, 4, 3, 2, 16, 256)
     assert kv == 10 * 4 + 2 * (1 + 3)
-    assert sel == 100 * 256 + 10 * 4 + 2 * 16 * 256
+    assert sel == 100 * 256 + 10 * 4 + 16 * 256  # queries read; outputs belong to attention
     assert att == kv * 512 + 10 * 4 + 2 * 16 * 256
     # the counts of a measured 256K decode step (16 units, 128 queries) give
     # the bytes that step reported
     sel, att, kv = bench.decode_step_bytes(1397720, 1048300, 4, 205, 16, 128, 256)
-    assert kv == 4196496 and sel + att == 2514939744
+    assert kv == 4196496 and sel + att == 2514939744 - 128 * 256

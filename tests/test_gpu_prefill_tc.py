@@ -175,12 +175,15 @@ def test_top_scores_unsupported_geometry():
 def test_prefill_full_size_sampled():
     """The full chunked-prefill workload (a 4096-token chunk after 1,048,576
     tokens, b = 4, L = 6, 257 top nodes for the last token), called as the
-    benchmark calls it: zha_prefill_chunk over the whole chunk. Sampled
-    (token, head) level counts and outputs against the oracle; exact index
-    lists of sampled tokens through zha_select, both with one token (a cluster
-    of CTAs per unit) and with a full 148-token tile (one CTA per unit, the
-    prefill configuration); then the tensor-core scores and certificates of
-    the whole chunk."""
+    benchmark calls it: zha_prefill_chunk over the whole chunk. 64 tokens x 16
+    heads (1024 queries: the first and last token, both sides of the first
+    tile edge 147/148, the rest seeded) against the oracle run over all host
+    cores: level counts and outputs. Exact index lists through zha_select for
+    the sampled tokens of two 148-token tiles (one CTA per unit, the prefill
+    configuration) and of one-token calls (a cluster of CTAs per unit); then
+    the tensor-core scores and certificates of the whole chunk."""
+    from _oracle_pool import run_units
+
     wl = W.make("prefill-deep-1m-chunk4k")
     c = wl.cfg
     gpu = Gpu(wl)  # tree over the cached context
@@ -192,37 +195,54 @@ def test_prefill_full_size_sampled():
     ws = z.alloc_workspace(gpu.cfg, z.ZHA_OP_PREFILL, c.chunk, device=gpu.dev)
     z.zha_prefill_chunk(gpu.cfg, gpu.cache, q, 0, start, c.p, out, lc, ws, gpu.status)
     gpu.check_status()
+    del ws
+    torch.cuda.empty_cache()
     ref = Ref(wl, start + c.chunk)
     for kvh in range(c.n_kv_heads):
         compare_tree(gpu, ref, 0, kvh)  # the chunk's nodes, extended in place
     outn = out.float().cpu().numpy()
     lcn = lc.cpu().numpy()
     qf = q.float().cpu().numpy()
-    expect = {}
-
-    def oracle_sel(i, h):
-        if (i, h) not in expect:
-            expect[(i, h)] = ref.select(qf[i, h], 0, h, start + i, c.p)
-        return expect[(i, h)]
-
-    for i in (0, 2047, c.chunk - 1):
-        for h in range(c.n_q_heads):
-            e_idx, e_counts, _, _ = oracle_sel(i, h)
-            assert lcn[i, h].tolist() == e_counts.tolist(), (i, h)
-            o = ref.attend(qf[i, h], 0, h, e_idx)
-            assert np.abs(outn[i, h] - o).max() < TOL["bf16"], (i, h)
-    for nq, toks in ((1, (0,)), (148, (0, 77, 147))):
-        idx, n_idx, lcs, _ = gpu.select(q[:nq].contiguous(), [0] * nq,
-                                        [start + i for i in range(nq)], c.p, start + c.chunk + 2)
+    rng = np.random.default_rng(4)
+    edges = [0, 1, 147, 148, 2047, 3948, 4094, c.chunk - 1]
+    rest = [int(i) for i in rng.permutation(c.chunk) if int(i) not in edges]
+    tokens = sorted(edges + rest[:64 - len(edges)])
+    # exact lists of the sampled tokens inside two 148-token tiles, and of two
+    # one-token calls
+    lists = {}
+    for lo, nq in ((0, 148), (3948, 148), (0, 1), (c.chunk - 1, 1)):
+        idx, n_idx, _, _ = gpu.select(q[lo:lo + nq].contiguous(), [0] * nq,
+                                      [start + lo + i for i in range(nq)], c.p,
+                                      start + c.chunk + 2)
         n_idx = n_idx.cpu().numpy()
-        for i in toks:
-            rows = idx[i].cpu().numpy()
-            for h in range(c.n_q_heads):
-                e_idx, _, _, _ = oracle_sel(i, h)
-                assert n_idx[i, h] == len(e_idx), (nq, i, h, n_idx[i, h], len(e_idx))
-                assert np.array_equal(rows[h, :n_idx[i, h]], e_idx), (nq, i, h)
+        for i in tokens:
+            if lo <= i < lo + nq:
+                for h in range(c.n_q_heads):
+                    lists[(nq, i, h)] = idx[i - lo, h, :n_idx[i - lo, h]].cpu().numpy()
         del idx
         torch.cuda.empty_cache()
+    # oracle tasks: per KV head, the tokens split into 4 tasks (each rebuilds
+    # the 1M-token tree)
+    R = wl.R.float().cpu().numpy()
+    tasks = []
+    for kvh in range(c.n_kv_heads):
+        for part in range(4):
+            qs = [((i, h), qf[i, h], start + i, c.p, "full") for i in tokens[part::4]
+                  for h in range(kvh * c.group, (kvh + 1) * c.group)]
+            tasks.append({"unit": (0, kvh), "k": wl.K[0, kvh], "v": wl.V[0, kvh],
+                          "dtype": c.dtype, "R": R, "n_tree": start + c.chunk, "b": c.block,
+                          "L": c.levels, "cap": c.capacity, "queries": qs})
+    n_list = 0
+    for _, results, _ in run_units(tasks):
+        for r in results:
+            i, h = r["key"]
+            assert lcn[i, h].tolist() == r["counts"].tolist(), (i, h)
+            assert np.abs(outn[i, h] - r["out"]).max() < TOL["bf16"], (i, h)
+            for nq in (148, 1):
+                if (nq, i, h) in lists:
+                    assert np.array_equal(lists[(nq, i, h)], r["idx"]), (nq, i, h)
+                    n_list += 1
+    assert n_list >= 16 * 8
     _check_top_scores(wl, gpu, ref, start, [0, 4095], 0.5)
 
 

@@ -42,7 +42,7 @@ EXPORTS = (
     "zha_status_string", "zha_tree_layout", "zha_workspace_bytes", "zha_build_tree",
     "zha_extend_tree", "zha_select", "zha_attend", "zha_decode", "zha_decode_select",
     "zha_decode_attend", "zha_decode_stats", "zha_prefill_chunk", "zha_dense_decode",
-    "zha_decode_noalloc", "zha_prefill_top_scores",
+    "zha_decode_noalloc", "zha_prefill_top_scores", "zha_decode_kept_lists",
 )
 
 
@@ -107,6 +107,7 @@ def lib() -> ctypes.CDLL:
                                   i32),
             "zha_dense_decode": ([c_cfg, c_cache, vp, vp, vp, sz, vp], i32),
             "zha_decode_noalloc": ([c_cfg, c_cache, vp, d, vp, vp, vp, vp], i32),
+            "zha_decode_kept_lists": ([c_cfg, c_cache, vp, sz, vp, i64, vp, vp, vp], i32),
             "zha_prefill_top_scores": ([c_cfg, c_cache, vp, i32, i64, i64, d, vp, vp, vp, sz, vp,
                                         vp], i32),
         }
@@ -272,6 +273,17 @@ def zha_decode_attend(cfg: zha_config, cache: Cache, q: torch.Tensor, out: torch
 def zha_decode_stats(cfg: zha_config, ws: torch.Tensor, stats: torch.Tensor, stream=None):
     _check("zha_decode_stats", lib().zha_decode_stats(
         ctypes.byref(cfg), _ptr(ws), ws.numel(), _ptr(stats), _stream(stream)))
+
+
+def zha_decode_kept_lists(cfg: zha_config, cache: Cache, ws: torch.Tensor, idx: torch.Tensor,
+                          n_idx: torch.Tensor, dev_status: Optional[torch.Tensor] = None,
+                          stream=None):
+    """Per-head token lists ([B][Hq][idx_cap] int32, lengths [B][Hq]) of the
+    last decode selection left in ws."""
+    c = cache.c()
+    _check("zha_decode_kept_lists", lib().zha_decode_kept_lists(
+        ctypes.byref(cfg), ctypes.byref(c), _ptr(ws), ws.numel(), _ptr(idx), idx.shape[-1],
+        _ptr(n_idx), _ptr(dev_status), _stream(stream)))
 
 
 def zha_prefill_chunk(cfg: zha_config, cache: Cache, q: torch.Tensor, seq: int, chunk_start: int,

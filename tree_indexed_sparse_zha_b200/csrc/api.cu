@@ -417,6 +417,24 @@ zha_status zha_decode_stats(const zha_config* cfg, const void* ws, size_t ws_byt
   return cuda_status(cudaGetLastError());
 }
 
+zha_status zha_decode_kept_lists(const zha_config* cfg, const zha_cache* cache, const void* ws,
+                                 size_t ws_bytes, int32_t* idx, int64_t idx_cap, int32_t* n_idx,
+                                 int32_t* dev_status, void* stream) {
+  Geometry g;
+  zha_status st = make_geometry(cfg, &g);
+  if (st != ZHA_OK) return st;
+  if (!cache || !cache->seq_len || !ws || !idx || idx_cap < 1 || !n_idx)
+    return ZHA_ERR_INVALID_ARG;
+  const int sms = device_sm_count();
+  const DecodeLayout L = decode_layout(g, g.B, kStreamTree, sms);
+  if (ws_bytes < L.total) return ZHA_ERR_WORKSPACE;
+  const unsigned char* w = static_cast<const unsigned char*>(ws);
+  return cuda_status(launch_kept_lists(
+      g, reinterpret_cast<const uint32_t*>(w + L.kept), reinterpret_cast<const int32_t*>(w + L.n_kept),
+      traverse_kept_stride(g), traverse_cluster_size(g, L.units, sms), cache->seq_len, idx, idx_cap,
+      n_idx, dev_status, (cudaStream_t)stream));
+}
+
 zha_status zha_prefill_chunk(const zha_config* cfg, const zha_cache* cache, const void* q,
                              int32_t seq, int64_t chunk_start, int64_t T, double p, void* out,
                              int32_t* level_counts, void* ws, size_t ws_bytes,

@@ -3,8 +3,11 @@
 // For callers that cannot hand the library a workspace: plugins loaded by a
 // host that owns the device allocator and exposes none of it, and hot paths
 // where an allocation is not allowed (cudaMalloc/cudaFree synchronise the
-// device). The scratch lives in this translation unit only, so its module --
-// and its memory -- is loaded only by programs that call this entry point.
+// device). The scratch is a static device array of this library: with the
+// CUDA runtime's default lazy module loading its 64 MiB are reserved on a
+// device only once a program calls this entry point there; with eager loading
+// (CUDA_MODULE_LOADING=EAGER) every process that loads libzha reserves them on
+// every device it uses, until exit.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -26,7 +29,10 @@ std::mutex g_mutex;
 void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of g_static_scratch on the current device, looked up once per
-// device (the first call on a device loads this module there).
+// device (the first call on a device loads this module there). The address is
+// kept for the life of the process: a device reset (cudaDeviceReset, or the
+// primary context destroyed and re-created) between calls would leave it
+// stale, so callers of this entry point must not reset the device.
 zha_status static_scratch(void** ptr) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) {

@@ -134,6 +134,14 @@ cudaError_t launch_attend_tile(const Geometry& g, const void* k, const void* v,
                                const int32_t* n_kept, int64_t kept_stride, int kept_segs,
                                void* ws, size_t ws_bytes, int num_sms, cudaStream_t stream);
 
+// Decode mode: each query head's token list (token 0, the tokens of the kept
+// level-1 nodes whose mask has the head's bit, the causal tail) from the
+// traversal's kept segments; idx [B][Hq][idx_cap], n_idx [B][Hq].
+cudaError_t launch_kept_lists(const Geometry& g, const uint32_t* kept, const int32_t* n_kept,
+                              int64_t stride, int segs, const int32_t* seq_len, int32_t* idx,
+                              int64_t idx_cap, int32_t* n_idx, int32_t* status,
+                              cudaStream_t stream);
+
 int device_sm_count();
 
 }  // namespace zha
