@@ -143,25 +143,171 @@ __device__ void node_small_b(const TreeParams& p, const float* Rt, float* abuf, 
   __syncwarp();
 }
 
+// ---------------------------------------------------------------------------
+// Level kernel for b <= 32: a CTA takes tiles of kTileRows consecutive child
+// rows (kTileRows / b whole nodes) of one unit. The rows are staged in shared
+// memory by cp.async, double-buffered so that the next tile's rows stream in
+// while the current one is reduced, in four phases:
+//   1. logits: thread (cg, rg) runs the 16 canonical chains of children
+//      4cg..4cg+3 against reference queries 4rg..4rg+3 -- every staged x
+//      chunk feeds 4 reference queries and every R value 4 children;
+//   2. softmax per (node, r) over the node's children, in child order;
+//   3. a_c = (sum_r w_rc in r order) / 16 per child;
+//   4. the weighted sum per (node, 16-byte output chunk), in child order,
+//      stored with one 16-byte write.
+// Each value is the same chain of the same rounded operations as in the
+// per-node formulation, so the stored summaries are bit-identical.
+// ---------------------------------------------------------------------------
+constexpr int kTileRows = 128;  // child rows per tile (a multiple of every b <= 32)
+constexpr int kTileThreads = 128;
+
 template <typename T, int D>
-__global__ void __launch_bounds__(256) tree_level_small_b(TreeParams p, int level) {
-  __shared__ __align__(16) float Rt[kNRef * D];
-  __shared__ float abuf[256];
-  load_rt<D>(p.r, Rt);
-  __syncthreads();
+struct TileCfg {
+  static constexpr int kPer = Elem<T>::kPerChunk;        // elements per 16-byte chunk
+  static constexpr int kNch = D * (int)sizeof(T) / 16;    // chunks per row
+  static constexpr int kStageBytes = kTileRows * D * (int)sizeof(T);
+  static constexpr int kRtBytes = kNRef * D * 4;
+  static constexpr int kWBytes = kTileRows * kNRef * 4;
+  static constexpr int kSmem = 2 * kStageBytes + kRtBytes + kWBytes + kTileRows * 4;
+};
+
+// Chunk ch of staged row r sits at chunk ch ^ ((r >> 2) & 7): the 8 rows one
+// warp reads at once in phase 1 (rows 4cg + k, 8 consecutive cg) then fall
+// in 8 different bank groups.
+__device__ __forceinline__ int tswz(int ch, int r) { return ch ^ ((r >> 2) & 7); }
+
+template <typename T, int D>
+__device__ __forceinline__ void stage_tile(const T* src, int rows, unsigned char* dst) {
+  using C = TileCfg<T, D>;
+  for (int e = threadIdx.x; e < rows * C::kNch; e += kTileThreads) {
+    const int r = e / C::kNch, ch = e % C::kNch;
+    cp_async16(dst + ((int64_t)r * C::kNch + tswz(ch, r)) * 16,
+               reinterpret_cast<const uint4*>(src + (int64_t)r * D) + ch);
+  }
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kTileThreads) tree_level_tiled(const __grid_constant__ TreeParams p,
+                                                                 int level) {
+  using C = TileCfg<T, D>;
+  constexpr int kPer = C::kPer, kNch = C::kNch;
+  extern __shared__ __align__(16) float sm[];
+  unsigned char* X0 = reinterpret_cast<unsigned char*>(sm);  // two stages of staged rows
+  float* Rt = reinterpret_cast<float*>(X0 + 2 * C::kStageBytes);  // [D][16]
+  float* W = Rt + kNRef * D;                                // [tile rows][16]
+  float* A = W + kTileRows * kNRef;                         // [tile rows]
+  const int tid = threadIdx.x;
   const int unit = blockIdx.y;
   const int seq = unit / p.Hkv;
+  const int b = p.b;
   const int64_t span = p.span[level];
   const int64_t n_new = clamp_len(p.seq_len[seq], p.ncap);
   const int64_t n_old = p.old_len ? clamp_len(p.old_len[seq], p.ncap) : 0;
   const int64_t lo = (n_old < n_new ? n_old : n_new) / span;
   const int64_t hi = n_new / span;
-  const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t node = lo + g / p.b;
-  const bool active = node < hi;
-  // whole warp idle -> leave (shuffles only mix lanes of one node group)
-  if (__all_sync(0xffffffffu, !active)) return;
-  node_small_b<T, D>(p, Rt, abuf + (threadIdx.x & ~31), level, unit, active ? node : lo, active);
+  const int64_t rows_total = (hi - lo) * b;  // child rows of the nodes to build
+  const int64_t n_tiles = (rows_total + kTileRows - 1) / kTileRows;
+  if ((int64_t)blockIdx.x >= n_tiles) return;  // uniform over the CTA
+  const T* cb = child_base<T, D>(p, level, unit) + lo * b * D;
+  T* ob = level_base<T, D>(p, level, unit) + lo * D;
+  load_rt<D>(p.r, Rt);
+  const int rg = tid & 3, cg = tid >> 2;  // phase-1 block: 4 children x 4 reference queries
+  const float inv_sqrt_d = p.inv_sqrt_d;
+
+  int64_t tile = blockIdx.x;
+  {
+    const int64_t r0 = tile * kTileRows;
+    const int rows = (int)(rows_total - r0 < kTileRows ? rows_total - r0 : kTileRows);
+    stage_tile<T, D>(cb + r0 * D, rows, X0);
+  }
+  cp_async_commit();
+  for (int it = 0; tile < n_tiles; ++it, tile += gridDim.x) {
+    unsigned char* X = X0 + (it & 1) * C::kStageBytes;
+    const int64_t r0 = tile * kTileRows;
+    const int rows = (int)(rows_total - r0 < kTileRows ? rows_total - r0 : kTileRows);
+    const int64_t next = tile + gridDim.x;
+    if (next < n_tiles) {  // the other stage was last read before the previous iteration's end
+      const int64_t n0 = next * kTileRows;
+      const int nrows = (int)(rows_total - n0 < kTileRows ? rows_total - n0 : kTileRows);
+      stage_tile<T, D>(cb + n0 * D, nrows, X0 + ((it + 1) & 1) * C::kStageBytes);
+    }
+    cp_async_commit();
+    cp_async_wait<1>();  // this tile's rows have landed (this thread's copies)
+    __syncthreads();     // ... and every thread's
+    // ---- 1. logits of children 4cg..4cg+3 against queries 4rg..4rg+3 ----
+    {
+      float2 acc[4][2];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[k][0] = acc[k][1] = make_float2(0.0f, 0.0f);
+#pragma unroll 2
+      for (int ch = 0; ch < kNch; ++ch) {
+        float x[4][kPer];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int r = 4 * cg + k;
+          Elem<T>::unpack(lds128(X + ((int64_t)r * kNch + tswz(ch, r)) * 16), x[k]);
+        }
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) {
+          const float4 rv = *reinterpret_cast<const float4*>(Rt + (ch * kPer + e) * kNRef + 4 * rg);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 xx = make_float2(x[k][e], x[k][e]);
+            acc[k][0] = ffma2(make_float2(rv.x, rv.y), xx, acc[k][0]);
+            acc[k][1] = ffma2(make_float2(rv.z, rv.w), xx, acc[k][1]);
+          }
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        *reinterpret_cast<float4*>(W + (4 * cg + k) * kNRef + 4 * rg) =
+            make_float4(__fmul_rn(acc[k][0].x, inv_sqrt_d), __fmul_rn(acc[k][0].y, inv_sqrt_d),
+                        __fmul_rn(acc[k][1].x, inv_sqrt_d), __fmul_rn(acc[k][1].y, inv_sqrt_d));
+    }
+    __syncthreads();
+    // ---- 2. softmax over each node's children, per reference query ----
+    const int nodes = rows / b;
+    for (int task = tid; task < nodes * kNRef; task += kTileThreads) {
+      const int n = task / kNRef, r = task % kNRef;
+      float* w = W + (n * b) * kNRef + r;
+      float mu = w[0];
+      for (int c = 1; c < b; ++c) mu = fmaxf(mu, w[c * kNRef]);
+      float Z = 0.0f;
+      for (int c = 0; c < b; ++c) {
+        const float e = exp_canon(__fsub_rn(w[c * kNRef], mu));
+        w[c * kNRef] = e;
+        Z = __fadd_rn(Z, e);
+      }
+      for (int c = 0; c < b; ++c) w[c * kNRef] = __fdiv_rn(w[c * kNRef], Z);
+    }
+    __syncthreads();
+    // ---- 3. child weights a_c ----
+    for (int c = tid; c < nodes * b; c += kTileThreads) {
+      float a = 0.0f;
+#pragma unroll
+      for (int r = 0; r < kNRef; ++r) a = __fadd_rn(a, W[c * kNRef + r]);
+      A[c] = __fmul_rn(a, 0.0625f);
+    }
+    __syncthreads();
+    // ---- 4. weighted sums, one 16-byte output chunk per task ----
+    for (int task = tid; task < nodes * kNch; task += kTileThreads) {
+      const int n = task / kNch, ch = task % kNch;
+      float s[kPer];
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) s[e] = 0.0f;
+      for (int c = 0; c < b; ++c) {
+        const int r = n * b + c;
+        float x[kPer];
+        Elem<T>::unpack(lds128(X + ((int64_t)r * kNch + tswz(ch, r)) * 16), x);
+        const float a = A[r];
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) s[e] = __fmaf_rn(a, x[e], s[e]);
+      }
+      *reinterpret_cast<uint4*>(ob + (r0 / b + n) * D + ch * kPer) = Elem<T>::pack(s);
+    }
+    __syncthreads();  // this stage is refilled two iterations on
+  }
+  cp_async_wait<0>();
 }
 
 // One CTA per unit walks every level; for small growth (decode steps).
@@ -275,10 +421,20 @@ cudaError_t launch_tree_t(const Geometry& g, const TreeParams& p, int64_t max_ne
     }
     if (nodes <= 0) break;
     if (small_b) {
-      const int64_t threads = nodes * g.b;
-      const int64_t blocks = (threads + 255) / 256;
-      dim3 grid((unsigned)blocks, (unsigned)units);
-      tree_level_small_b<T, D><<<grid, 256, 0, stream>>>(p, level);
+      using C = TileCfg<T, D>;
+      cudaError_t e = cudaFuncSetAttribute(tree_level_tiled<T, D>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+      if (e != cudaSuccess) return e;
+      int per_sm = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tree_level_tiled<T, D>,
+                                                        kTileThreads, C::kSmem);
+      if (e != cudaSuccess) return e;
+      // enough CTAs for one full wave over all units, each looping over tiles
+      const int64_t tiles = (nodes * g.b + kTileRows - 1) / kTileRows;
+      int64_t per_unit = ((int64_t)device_sm_count() * (per_sm > 0 ? per_sm : 1) + units - 1) / units;
+      if (per_unit > tiles) per_unit = tiles;
+      dim3 grid((unsigned)per_unit, (unsigned)units);
+      tree_level_tiled<T, D><<<grid, kTileThreads, C::kSmem, stream>>>(p, level);
     } else {
       const size_t smem = sizeof(float) * (kNRef * D + kNRef * g.b + g.b + 32 * kNRef + kNRef);
       cudaError_t e = cudaFuncSetAttribute(tree_level_large_b<T, D>,

@@ -99,6 +99,11 @@ struct Elem<float> {
     out[2] = __uint_as_float(c.z);
     out[3] = __uint_as_float(c.w);
   }
+  // pack kPerChunk floats into a 16-byte chunk
+  __device__ __forceinline__ static uint4 pack(const float* v) {
+    return make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]),
+                      __float_as_uint(v[3]));
+  }
   __device__ __forceinline__ static float load(const float* p) { return *p; }
   __device__ __forceinline__ static float to_f(float v) { return v; }
   __device__ __forceinline__ static float from_f(float v) { return v; }
@@ -112,6 +117,16 @@ struct Elem<__nv_bfloat16> {
                  e = bf16x2_to_f2(c.w);
     out[0] = a.x; out[1] = a.y; out[2] = b.x; out[3] = b.y;
     out[4] = d.x; out[5] = d.y; out[6] = e.x; out[7] = e.y;
+  }
+  // round kPerChunk floats to nearest-even bf16 and pack them (element 0 in
+  // the low half of the first word)
+  __device__ __forceinline__ static uint4 pack(const float* v) {
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      w[j] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * j])) |
+             ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v[2 * j + 1])) << 16);
+    return make_uint4(w[0], w[1], w[2], w[3]);
   }
   __device__ __forceinline__ static float load(const __nv_bfloat16* p) {
     return __bfloat162float(*p);
