@@ -85,14 +85,19 @@ static zha_status cuda_status(cudaError_t e) { return e == cudaSuccess ? ZHA_OK 
 struct DecodeLayout {
   size_t trav, kept, n_kept, stats, part, total;
   int64_t units;
+  bool dense;  // selection by decode_dense (decode steps), else the frontier traversal
 };
 
-static DecodeLayout decode_layout(const Geometry& g, int64_t nq, int kind, int sms) {
+// dense: the caller is a decode step (one query per sequence at seq_len - 1)
+static DecodeLayout decode_layout(const Geometry& g, int64_t nq, int kind, int sms,
+                                  bool decode = false) {
   DecodeLayout L{};
   L.units = nq * g.Hkv;
+  L.dense = decode && decode_dense_ok(g, L.units);
   size_t off = 0;
   L.trav = off;
-  off = align256(off + traverse_ws_bytes(g, L.units, sms));
+  off = align256(off + (L.dense ? decode_dense_ws_bytes(g, L.units)
+                                : traverse_ws_bytes(g, L.units, sms)));
   L.kept = off;
   off = align256(off + traverse_kept_bytes(g, L.units, sms));
   L.n_kept = off;
@@ -204,7 +209,7 @@ zha_status zha_workspace_bytes(const zha_config* cfg, int32_t op, int64_t max_qu
       *bytes = align256(attend_ws_bytes(g, kStreamList, max_queries, sms));
       return ZHA_OK;
     case ZHA_OP_DECODE:
-      *bytes = decode_layout(g, g.B, kStreamTree, sms).total;
+      *bytes = decode_layout(g, g.B, kStreamTree, sms, true).total;
       return ZHA_OK;
     case ZHA_OP_DENSE:
       *bytes = align256(attend_ws_bytes(g, kStreamDense, g.B, sms));
@@ -301,6 +306,12 @@ static zha_status run_tree_select(const Geometry& g, const zha_cache* cache, con
                                   uint64_t p_q, int32_t* level_counts, unsigned char* ws,
                                   const DecodeLayout& L, int32_t* dev_status, int sms,
                                   cudaStream_t s, const TopSeeds* seeds = nullptr) {
+  if (L.dense && !q_pos && !seeds)
+    return cuda_status(launch_decode_dense(
+        g, cache->tree, q, cache->seq_len, p_q, ws + L.trav, level_counts,
+        reinterpret_cast<int32_t*>(ws + L.stats), reinterpret_cast<uint32_t*>(ws + L.kept),
+        reinterpret_cast<int32_t*>(ws + L.n_kept), traverse_kept_stride(g),
+        traverse_cluster_size(g, L.units, sms), dev_status, sms, s));
   TraverseOut to{};
   to.kept = reinterpret_cast<uint32_t*>(ws + L.kept);
   to.n_kept = reinterpret_cast<int32_t*>(ws + L.n_kept);
@@ -362,7 +373,7 @@ zha_status zha_decode(const zha_config* cfg, const zha_cache* cache, const void*
   uint64_t p_q;
   if (!q || !out || !ws || !check_p(p, &p_q)) return ZHA_ERR_INVALID_ARG;
   const int sms = device_sm_count();
-  const DecodeLayout L = decode_layout(g, g.B, kStreamTree, sms);
+  const DecodeLayout L = decode_layout(g, g.B, kStreamTree, sms, true);
   if (ws_bytes < L.total) return ZHA_ERR_WORKSPACE;
   return run_tree_decode(g, cache, q, nullptr, nullptr, g.B, p_q, out, level_counts,
                          static_cast<unsigned char*>(ws), L, dev_status, sms,
@@ -379,7 +390,7 @@ zha_status zha_decode_select(const zha_config* cfg, const zha_cache* cache, cons
   uint64_t p_q;
   if (!q || !ws || !check_p(p, &p_q)) return ZHA_ERR_INVALID_ARG;
   const int sms = device_sm_count();
-  const DecodeLayout L = decode_layout(g, g.B, kStreamTree, sms);
+  const DecodeLayout L = decode_layout(g, g.B, kStreamTree, sms, true);
   if (ws_bytes < L.total) return ZHA_ERR_WORKSPACE;
   return run_tree_select(g, cache, q, nullptr, nullptr, g.B, p_q, level_counts,
                          static_cast<unsigned char*>(ws), L, dev_status, sms,
@@ -394,7 +405,7 @@ zha_status zha_decode_attend(const zha_config* cfg, const zha_cache* cache, cons
   if ((st = check_cache(cache, true)) != ZHA_OK) return st;
   if (!q || !out || !ws) return ZHA_ERR_INVALID_ARG;
   const int sms = device_sm_count();
-  const DecodeLayout L = decode_layout(g, g.B, kStreamTree, sms);
+  const DecodeLayout L = decode_layout(g, g.B, kStreamTree, sms, true);
   if (ws_bytes < L.total) return ZHA_ERR_WORKSPACE;
   return run_tree_attend(g, cache, q, nullptr, nullptr, g.B, out,
                          static_cast<unsigned char*>(ws), L, sms, (cudaStream_t)stream);
@@ -407,7 +418,7 @@ zha_status zha_decode_stats(const zha_config* cfg, const void* ws, size_t ws_byt
   if (st != ZHA_OK) return st;
   if (!ws || !stats) return ZHA_ERR_INVALID_ARG;
   const int sms = device_sm_count();
-  const DecodeLayout L = decode_layout(g, g.B, kStreamTree, sms);
+  const DecodeLayout L = decode_layout(g, g.B, kStreamTree, sms, true);
   if (ws_bytes < L.total) return ZHA_ERR_WORKSPACE;
   const unsigned char* w = static_cast<const unsigned char*>(ws);
   const int units = (int)L.units;
@@ -426,7 +437,7 @@ zha_status zha_decode_kept_lists(const zha_config* cfg, const zha_cache* cache, 
   if (!cache || !cache->seq_len || !ws || !idx || idx_cap < 1 || !n_idx)
     return ZHA_ERR_INVALID_ARG;
   const int sms = device_sm_count();
-  const DecodeLayout L = decode_layout(g, g.B, kStreamTree, sms);
+  const DecodeLayout L = decode_layout(g, g.B, kStreamTree, sms, true);
   if (ws_bytes < L.total) return ZHA_ERR_WORKSPACE;
   const unsigned char* w = static_cast<const unsigned char*>(ws);
   return cuda_status(launch_kept_lists(

@@ -226,16 +226,6 @@ __device__ __forceinline__ unsigned int block_excl_scan(unsigned int v, unsigned
   return wbase + x - v;
 }
 
-// ceil(T * pq / 2^32) without overflow.
-__device__ __forceinline__ unsigned long long ceil_mul_shift32(unsigned long long T,
-                                                               unsigned long long pq) {
-  const unsigned long long lo = T * pq;
-  const unsigned long long hi = __umul64hi(T, pq);
-  unsigned long long r = (hi << 32) | (lo >> 32);
-  if (lo & 0xffffffffull) r += 1;
-  return r;
-}
-
 // L2 eviction policy of the per-candidate scores, which every pass of the cut
 // re-reads (evict last).
 __device__ __forceinline__ uint64_t policy_evict_last() {
@@ -303,14 +293,6 @@ __device__ __forceinline__ uint32_t bytes_eq(uint64_t a, uint64_t b) {
 __device__ __forceinline__ uint32_t bytes_nz(uint64_t a) {
   return gather_bits(((uint64_t)__vcmpne4((unsigned)(a >> 32), 0u) << 32) |
                      __vcmpne4((unsigned)a, 0u));
-}
-
-// First-pass bucket of score z: a linear map of [zlo, zlo + 256 / zscale)
-// onto 0..255, clamped. Non-decreasing in z, and evaluated with the same
-// operations on every CTA.
-__device__ __forceinline__ uint32_t quant_bucket(float z, float zlo, float zscale) {
-  const float f = __fmul_rn(__fsub_rn(z, zlo), zscale);
-  return (uint32_t)fminf(fmaxf(f, 0.0f), 255.0f);  // NaN (inf * 0) maps to 0
 }
 
 // The canonical dot products of this thread's rows (up to K of them) with the
@@ -477,57 +459,6 @@ __device__ __forceinline__ void hist_add_heads(Smem& S, const uint32_t* d,
     if (hi) atomicAdd(&S.hist_hi[h][d[h]], hi);
     if (c[h]) atomicAdd(&S.hist_c[h][d[h]], c[h]);
   }
-}
-
-// Inverse of order_key.
-__device__ __forceinline__ float key_float(uint32_t k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
-}
-
-// Smallest key in [lo, hi] whose first-pass bucket is >= beta; the bucket of
-// key_float(hi) must be >= beta. Binary search over the key order.
-__device__ __forceinline__ uint32_t quant_first_key(float zlo, float zscale, uint32_t beta,
-                                                    uint32_t lo, uint32_t hi) {
-  while (lo < hi) {
-    const uint32_t mid = lo + (hi - lo) / 2;
-    if (quant_bucket(key_float(mid), zlo, zscale) >= beta) hi = mid;
-    else lo = mid + 1;
-  }
-  return lo;
-}
-
-// First key of bucket beta (beta >= 1): the search starts in a window of 512
-// keys around the estimate zlo + beta / zscale and widens to the whole key
-// range of the finite scores when the window does not bracket the boundary.
-__device__ __forceinline__ uint32_t quant_boundary(float zlo, float zscale, uint32_t beta) {
-  const uint32_t kneg = order_key(-INFINITY), kpos = order_key(INFINITY);
-  const uint32_t ke = order_key(__fadd_rn(zlo, __fdiv_rn((float)beta, zscale)));
-  uint32_t lo = ke > kneg + 256u ? ke - 256u : kneg;
-  uint32_t hi = ke < kpos - 256u ? ke + 256u : kpos;
-  if (lo < kneg || hi > kpos || lo > hi || quant_bucket(key_float(lo), zlo, zscale) >= beta ||
-      quant_bucket(key_float(hi), zlo, zscale) < beta) {
-    lo = kneg;
-    hi = kpos;
-  }
-  return quant_first_key(zlo, zscale, beta, lo, hi);
-}
-
-// Key interval [*klo, *khi] of the finite scores whose first-pass bucket is
-// beta (an interval, as the bucket map is non-decreasing in the score).
-__device__ __forceinline__ void quant_interval(float zlo, float zscale, uint32_t beta,
-                                               uint32_t* klo, uint32_t* khi) {
-  *klo = beta == 0u ? order_key(-INFINITY) : quant_boundary(zlo, zscale, beta);
-  *khi = beta >= (uint32_t)kBuckets - 1u || zscale == 0.0f
-             ? order_key(INFINITY)
-             : quant_boundary(zlo, zscale, beta + 1u) - 1u;
-}
-
-// Digit width and position of a kModeRadix pass over the group [kgmin, kgmax]
-// (kgmin < kgmax): the bits below the range's common prefix, 8 at a time.
-__device__ __forceinline__ void radix_digit(unsigned kgmin, unsigned kgmax, int* sh, int* w) {
-  const int shift = 32 - __clz(kgmin ^ kgmax);
-  *w = shift < kDigit ? shift : kDigit;
-  *sh = shift - *w;
 }
 
 // The state of a head after a pass found its crossing bucket beta (ok):

@@ -57,6 +57,81 @@ __device__ __forceinline__ uint32_t order_key(float z) {
 }
 
 // ---------------------------------------------------------------------------
+// top-p cut helpers (exact integer arithmetic and the score -> bucket maps)
+// ---------------------------------------------------------------------------
+
+constexpr int kCutDigit = 8;  // key bits resolved per radix pass (256 buckets)
+
+// ceil(T * pq / 2^32) without overflow.
+__device__ __forceinline__ unsigned long long ceil_mul_shift32(unsigned long long T,
+                                                               unsigned long long pq) {
+  const unsigned long long lo = T * pq;
+  const unsigned long long hi = __umul64hi(T, pq);
+  unsigned long long r = (hi << 32) | (lo >> 32);
+  if (lo & 0xffffffffull) r += 1;
+  return r;
+}
+
+// First-pass bucket of score z: a linear map of [zlo, zlo + 256 / zscale)
+// onto 0..255, clamped. Non-decreasing in z, and evaluated with the same
+// operations on every CTA.
+__device__ __forceinline__ uint32_t quant_bucket(float z, float zlo, float zscale) {
+  const float f = __fmul_rn(__fsub_rn(z, zlo), zscale);
+  return (uint32_t)fminf(fmaxf(f, 0.0f), 255.0f);  // NaN (inf * 0) maps to 0
+}
+
+// Inverse of order_key.
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Smallest key in [lo, hi] whose first-pass bucket is >= beta; the bucket of
+// key_float(hi) must be >= beta. Binary search over the key order.
+__device__ __forceinline__ uint32_t quant_first_key(float zlo, float zscale, uint32_t beta,
+                                                    uint32_t lo, uint32_t hi) {
+  while (lo < hi) {
+    const uint32_t mid = lo + (hi - lo) / 2;
+    if (quant_bucket(key_float(mid), zlo, zscale) >= beta) hi = mid;
+    else lo = mid + 1;
+  }
+  return lo;
+}
+
+// First key of bucket beta (beta >= 1): the search starts in a window of 512
+// keys around the estimate zlo + beta / zscale and widens to the whole key
+// range of the finite scores when the window does not bracket the boundary.
+__device__ __forceinline__ uint32_t quant_boundary(float zlo, float zscale, uint32_t beta) {
+  const uint32_t kneg = order_key(-INFINITY), kpos = order_key(INFINITY);
+  const uint32_t ke = order_key(__fadd_rn(zlo, __fdiv_rn((float)beta, zscale)));
+  uint32_t lo = ke > kneg + 256u ? ke - 256u : kneg;
+  uint32_t hi = ke < kpos - 256u ? ke + 256u : kpos;
+  if (lo < kneg || hi > kpos || lo > hi || quant_bucket(key_float(lo), zlo, zscale) >= beta ||
+      quant_bucket(key_float(hi), zlo, zscale) < beta) {
+    lo = kneg;
+    hi = kpos;
+  }
+  return quant_first_key(zlo, zscale, beta, lo, hi);
+}
+
+// Key interval [*klo, *khi] of the finite scores whose first-pass bucket is
+// beta (an interval, as the bucket map is non-decreasing in the score).
+__device__ __forceinline__ void quant_interval(float zlo, float zscale, uint32_t beta,
+                                               uint32_t* klo, uint32_t* khi) {
+  *klo = beta == 0u ? order_key(-INFINITY) : quant_boundary(zlo, zscale, beta);
+  *khi = beta >= 255u || zscale == 0.0f
+             ? order_key(INFINITY)
+             : quant_boundary(zlo, zscale, beta + 1u) - 1u;
+}
+
+// Digit width and position of a kModeRadix pass over the group [kgmin, kgmax]
+// (kgmin < kgmax): the bits below the range's common prefix, 8 at a time.
+__device__ __forceinline__ void radix_digit(unsigned kgmin, unsigned kgmax, int* sh, int* w) {
+  const int shift = 32 - __clz(kgmin ^ kgmax);
+  *w = shift < kCutDigit ? shift : kCutDigit;
+  *sh = shift - *w;
+}
+
+// ---------------------------------------------------------------------------
 // packed fp32x2 FMA (sm_100): two independent round-to-nearest FMAs, each
 // bit-identical to __fmaf_rn on its lane.
 // ---------------------------------------------------------------------------

@@ -76,6 +76,20 @@ cudaError_t launch_traverse(const Geometry& g, const void* tree, const void* q,
                             void* ws, size_t ws_bytes, int32_t* status, int num_sms,
                             cudaStream_t stream, const TopSeeds* seeds = nullptr);
 
+// ---- decode selection with every summary row scored up front ---------------
+// True when a decode step of `units` (sequence, KV head) units takes this path
+// (its shared-memory state fits and the tree prefix it reads is bounded).
+bool decode_dense_ok(const Geometry& g, int64_t units);
+size_t decode_dense_ws_bytes(const Geometry& g, int64_t units);
+// Decode mode only (query of sequence s at seq_len[s] - 1): writes the kept
+// level-1 union with per-head masks in `segs` ordered segments per unit, the
+// per-head level counts (nullable) and the rows scored per level (stats).
+cudaError_t launch_decode_dense(const Geometry& g, const void* tree, const void* q,
+                                const int32_t* seq_len, uint64_t p_q, void* ws,
+                                int32_t* level_counts, int32_t* stats, uint32_t* kept,
+                                int32_t* n_kept, int64_t kept_stride, int segs, int32_t* status,
+                                int num_sms, cudaStream_t stream);
+
 // ---- prefill top level on the tensor cores ----------------------------------
 // Top nodes per (sequence, KV head): ncap / b^L.
 int64_t top_cap(const Geometry& g);
