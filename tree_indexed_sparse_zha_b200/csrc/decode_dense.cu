@@ -80,12 +80,12 @@ __device__ __forceinline__ int64_t decode_top(const DenseParams& p, int seq) {
 }
 
 // ---------------------------------------------------------------------------
-// 1. scoring: tiles of 1024 contiguous rows of one level of one unit; each of
-//    the 256 threads runs the G chains of 4 rows (rows t, t+256, t+512, t+768
-//    of the tile). Rows are staged 64 bytes (4 chunks) at a time, two stages
+// 1. scoring: tiles of 512 contiguous rows of one level of one unit; each of
+//    the 128 threads runs the G chains of 4 rows (rows t, t+128, t+256, t+384
+//    of the tile), three CTAs per SM. Rows are staged 64 bytes (4 chunks) at a time, two stages
 //    in flight; a warp's load instruction covers 8 rows x 64 contiguous bytes.
 // ---------------------------------------------------------------------------
-constexpr int kSThreads = 256;
+constexpr int kSThreads = 128;
 constexpr int kSTile = 4 * kSThreads;          // rows per tile
 constexpr int kSStageBytes = kSTile * 64;      // 4 chunks of every row of a tile
 
@@ -96,7 +96,7 @@ struct ScoreCfg {
   static constexpr int kSteps = kNch / 4;       // stages per row
   static constexpr int kSmem = 2 * kSStageBytes + D * kMaxGroup * 4;
 };
-static_assert(kSThreads == 256, "tile mapping assumes 256 threads");
+static_assert(kSTile == 128 * (kSThreads / 32), "a warp stages 128 rows of the tile");
 
 // Chunk c (0..3) of staged row r sits at slot c ^ ((r >> 1) & 3) of the row's
 // 64 bytes: 8 consecutive rows read by 8 consecutive lanes then cover all 32
@@ -123,7 +123,7 @@ __device__ __forceinline__ void stage_rows(const T* lvl, int64_t r0, int n, int 
 }
 
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kSThreads, 1) dense_score_kernel(const __grid_constant__ DenseParams p) {
+__global__ void __launch_bounds__(kSThreads, 3) dense_score_kernel(const __grid_constant__ DenseParams p) {
   using C = ScoreCfg<T, D>;
   constexpr int kPer = C::kPer, kSteps = C::kSteps;
   extern __shared__ __align__(16) unsigned char sm[];
@@ -1068,6 +1068,7 @@ constexpr int kUThreads = 256;
 // is written with the mask of the heads that keep it.
 __global__ void __launch_bounds__(kUThreads) union_kernel(const __grid_constant__ DenseParams p) {
   __shared__ unsigned int s_warp[kUThreads / 32];
+  __shared__ uint32_t s_out[32 * kUThreads];  // one iteration's entries, written out coalesced
   const int r = blockIdx.x, unit = blockIdx.y;
   const int seq = unit / p.Hkv;
   const int G = p.G;
@@ -1107,15 +1108,17 @@ __global__ void __launch_bounds__(kUThreads) union_kernel(const __grid_constant_
       if (w2 < warp) wbase += s_warp[w2];
       tot += s_warp[w2];
     }
-    unsigned pos = run + wbase + x - f;
+    unsigned pos = wbase + x - f;  // within this iteration's entries
     while (any) {
       const int i = __ffs(any) - 1;
       any &= any - 1u;
       uint32_t mask = 0;
 #pragma unroll
       for (int h = 0; h < kMaxGroup; ++h) mask |= ((words[h] >> i) & 1u) << h;
-      out[pos++] = (mask << 24) | (uint32_t)(n0 + i);
+      s_out[pos++] = (mask << 24) | (uint32_t)(n0 + i);
     }
+    __syncthreads();
+    for (unsigned e = tid; e < tot; e += kUThreads) out[run + e] = s_out[e];
     run += tot;
     __syncthreads();
   }
@@ -1128,7 +1131,7 @@ cudaError_t launch_score(const DenseParams& p, int units, int sms, cudaStream_t 
   auto kern = dense_score_kernel<T, D, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
-  int per = sms / units;
+  int per = 3 * sms / units;  // three CTAs per SM
   if (per < 1) per = 1;
   dense_score_kernel<T, D, G><<<dim3((unsigned)per, (unsigned)units), kSThreads, C::kSmem, s>>>(p);
   return cudaGetLastError();

@@ -315,13 +315,15 @@ template <typename T, int D>
 __global__ void __launch_bounds__(128) tree_extend_fused(TreeParams p) {
   __shared__ __align__(16) float Rt[kNRef * D];
   __shared__ float abuf[128];
-  load_rt<D>(p.r, Rt);
-  __syncthreads();
   const int unit = blockIdx.x;
   const int seq = unit / p.Hkv;
   const int64_t n_new = clamp_len(p.seq_len[seq], p.ncap);
   const int64_t n_old0 = p.old_len ? clamp_len(p.old_len[seq], p.ncap) : 0;
   const int64_t n_old = n_old0 < n_new ? n_old0 : n_new;
+  // most single-token steps complete no node: leave before staging R
+  if (n_old / p.span[1] >= n_new / p.span[1]) return;  // uniform over the CTA
+  load_rt<D>(p.r, Rt);
+  __syncthreads();
   const int groups = blockDim.x / p.b;
   for (int level = 1; level <= p.L; ++level) {
     const int64_t lo = n_old / p.span[level];
