@@ -195,7 +195,7 @@ def kernel_source_hash() -> str:
     """Hash of the decode-step kernels' code, comments and layout excluded, so
     that recorded DRAM counters stay tied to the code they were taken on."""
     h = hashlib.sha256()
-    for f in ("traverse.cu", "attend.cu", "zha_device.cuh"):
+    for f in ("decode_dense.cu", "attend.cu", "zha_device.cuh"):
         with open(os.path.join(ROOT, "tree_indexed_sparse_zha_b200", "csrc", f), encoding="utf-8") as fh:
             h.update(strip_c_comments(fh.read()).encode())
             h.update(b"\0")
@@ -725,19 +725,22 @@ def run_zha(args, rank, world, dev):
     h2d = kv_host[0].numel() * kv_host.element_size() + q_host[0].numel() * q_host.element_size()
     d2h = out_host[0].numel() * out_host.element_size()
 
-    # ---- roofline of the dominant kernel group ----
+    # ---- roofline of both kernel groups; the line's `roofline` is the one
+    # that takes longer. Traffic is ncu's DRAM bytes per launch from the
+    # committed record, while it matches these kernels' sources ----
     traffic = recorded_traffic() if args.n_tokens is None else None  # taken at full size
-    if ms_att >= ms_sel:
-        roof = {"kernel": "attend_mma_kernel + combine (zha_decode_attend)", "bound": "hbm",
-                "achieved": att_bytes / (ms_att / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
-                "peak_kind": peak_kind}
-        roof["traffic"] = float(traffic["attend_dram_bytes_per_launch"]) if traffic else None
-    else:
-        roof = {"kernel": "traverse_kernel (zha_decode_select)", "bound": "hbm",
-                "achieved": sel_bytes / (ms_sel / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
-                "peak_kind": peak_kind}
-        roof["traffic"] = float(traffic["traverse_dram_bytes_per_launch"]) if traffic else None
-    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof_att = {"kernel": "attend_mma_kernel + combine_kernel (zha_decode_attend)",
+                "bound": "hbm", "achieved": att_bytes / (ms_att / 1e3) / 1e9, "peak": peak,
+                "unit": "GB/s", "peak_kind": peak_kind,
+                "traffic": float(traffic["attend_dram_bytes_per_step"]) if traffic else None}
+    roof_sel = {"kernel": "dense_score_kernel + head_cut_kernel + union_kernel "
+                          "(zha_decode_select)",
+                "bound": "hbm", "achieved": sel_bytes / (ms_sel / 1e3) / 1e9, "peak": peak,
+                "unit": "GB/s", "peak_kind": peak_kind,
+                "traffic": float(traffic["select_dram_bytes_per_step"]) if traffic else None}
+    for r_ in (roof_att, roof_sel):
+        r_["frac"] = r_["achieved"] / r_["peak"]
+    roof = dict(roof_att if ms_att >= ms_sel else roof_sel)
 
     res = {
         "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world,
@@ -753,6 +756,7 @@ def run_zha(args, rank, world, dev):
                       "kv_rows_read": kv_rows,
                       "kv_fraction_read": kv_rows / (B * Hkv * n_last), **per_query},
         "roofline": roof,
+        "roofline_by_phase": {"select": roof_sel, "attend": roof_att},
         "dense": {"ms_per_step": dense_ms, "queries_per_s": queries_per_step * world / (dense_ms / 1e3),
                   "hbm_gbs": dense_bytes / (dense_ms / 1e3) / 1e9,
                   "hbm_frac": dense_bytes / (dense_ms / 1e3) / 1e9 / peak},
@@ -762,7 +766,7 @@ def run_zha(args, rank, world, dev):
                        "tokens": n_tok},
         "e2e": {"value": queries_per_step * world / (e2e_ms / 1e3), "unit": "queries/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 6 * args.steps,  # extend, score, cut, union, attention, combine
         "clocks": clocks,
     }
     if args.n_tokens is None:  # the other workloads at their full sizes

@@ -214,6 +214,44 @@ def test_zero_query_all_ties():
         _decode_parity(wl, q, p, c.n_tokens)
 
 
+def test_decode_clustered_keys_narrowed_groups():
+    """Decode (B = 1, 131K context) over keys that form one tight cluster
+    (a common vector plus 0.01 noise) with one far-off key every 256 tokens:
+    the far keys stretch each level's score range, so the cluster's
+    candidates crowd into a few first-pass buckets and, at level 1, the
+    crossing bucket holds thousands of them with distinct keys. The cut then
+    narrows it by key digits before ranking. Counts and attended sets must
+    equal the oracle's for every head."""
+    wl = W.make("decode-deep-32k", n_tokens=131072)
+    c = wl.cfg
+    g = torch.Generator().manual_seed(3)
+    n = c.n_tokens
+    for kvh in range(c.n_kv_heads):
+        v = torch.randn(c.head_dim, generator=g)
+        keys = v + 0.01 * torch.randn(n, c.head_dim, generator=g)
+        keys[::256] = 3.0 * torch.randn(keys[::256].shape, generator=g)
+        wl.K[0, kvh, :n] = keys.to(c.torch_dtype)
+    gpu = Gpu(wl)
+    ref = Ref(wl, c.n_tokens)
+    _decode_parity.gpu, _decode_parity.ref = gpu, ref
+    for p in (0.5, 0.95):
+        _decode_parity(wl, wl.queries(0), p, c.n_tokens)
+
+
+def test_decode_long_context_large_frontier():
+    """Decode at 400K context (B = 1) with p = 0.999: the level-1 frontier of a
+    head exceeds what the cut keeps bucket bytes for in shared memory, and the
+    kept list one level up exceeds its shared copy, so the cut streams its
+    parents and scores from global memory. Checked head by head against the
+    oracle."""
+    wl = W.make("decode-deep-32k", n_tokens=400000)
+    c = wl.cfg
+    gpu = Gpu(wl)
+    ref = Ref(wl, c.n_tokens)
+    _decode_parity.gpu, _decode_parity.ref = gpu, ref
+    _decode_parity(wl, wl.queries(0), 0.999, c.n_tokens)
+
+
 def test_select_one_cta_narrowed_groups():
     """148 queries (one CTA per (query, KV head) unit, as a prefill tile runs)
     at 131K context, small-norm queries and p = 0.5 / 0.95: the crossing
