@@ -454,7 +454,9 @@ def workload_config(args, c):
     return {"workload": args.workload, "batch": c.batch, "context": c.n_tokens,
             "heads": f"{c.n_q_heads}q/{c.n_kv_heads}kv", "head_dim": c.head_dim,
             "tree": f"b={c.block},L={c.levels}", "p": c.p,
-            "queries_per_step": c.batch * c.n_q_heads, "l2": l2_note(kv_gb)}
+            "queries_per_step": c.batch * c.n_q_heads, "l2": l2_note(kv_gb),
+            "step": "CUDA graph of zha_extend_tree + zha_decode, replayed after the step's "
+                    "lengths and queries are copied into its input buffers"}
 
 
 def tree_build_work(n_tokens: int, b: int, L: int, D: int, units: int, elem: int = 2):
@@ -607,31 +609,51 @@ def run_zha(args, rank, world, dev):
         s = (i % n_steps_cap) + 1  # wrap: rebuilt nodes are identical
         return s, lens[s - 1], lens[s], queries[s - 1]
 
-    def one_step(i, ev=None):
-        s, old, new, q = step_inputs(i)
-        cache.seq_len = new
-        if ev:
-            ev[0].record(stream)
-        z.zha_extend_tree(cfg, cache, old, 1)
-        if ev:
-            ev[1].record(stream)
-        z.zha_decode_select(cfg, cache, q, c.p, None, ws, st)
-        if ev:
-            ev[2].record(stream)
-        z.zha_decode_attend(cfg, cache, q, out, ws)
-        if ev:
-            ev[3].record(stream)
+    # The timed step is one CUDA graph of zha_extend_tree + zha_decode (the
+    # decode's unit groups on the library's own streams, joined back), fed
+    # through static buffers: each step copies its lengths and queries into
+    # them (inside the timed region) and replays the graph.
+    old_st, len_st = lens[0].clone(), lens[0].clone()
+    q_st = torch.empty_like(queries[0])
+    cache.seq_len = len_st
 
-    # reset the tree to the initial length, then warm up
-    cache.seq_len = lens[0]
+    def load_inputs(i):
+        _, old, new, q = step_inputs(i)
+        old_st.copy_(old)
+        len_st.copy_(new)
+        q_st.copy_(q)
+
+    def decode_body():
+        z.zha_extend_tree(cfg, cache, old_st, 1)
+        z.zha_decode(cfg, cache, q_st, c.p, out, None, ws, st)
+
+    # reset the tree to the initial length, then warm up (eagerly, which also
+    # creates the library's streams), capture and warm up the graph
+    len_st.copy_(lens[0])
+    z.zha_build_tree(cfg, cache)
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for i in range(args.warmup):
+            load_inputs(i)
+            decode_body()
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    load_inputs(args.warmup)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph):
+        decode_body()
+    torch.cuda.synchronize()
+    len_st.copy_(lens[0])
     z.zha_build_tree(cfg, cache)
     for i in range(args.warmup):
-        one_step(i)
+        load_inputs(i)
+        graph.replay()
     torch.cuda.synchronize()
     if int(st.item()) != 0:
         raise RuntimeError(f"device status {z.status_string(int(st.item()))}")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(True), torch.cuda.Event(True)
     sampler = ClockSampler(dev.index if dev.index is not None else 0)
     if world > 1:
@@ -641,17 +663,16 @@ def run_zha(args, rank, world, dev):
     time.sleep(0.3)
     t_start.record(stream)
     for i in range(args.steps):
-        one_step(args.warmup + i, evs[i])
+        load_inputs(args.warmup + i)
+        graph.replay()
     t_end.record(stream)
     torch.cuda.synchronize()
     clocks = sampler.stop()
     if world > 1:
         torch.distributed.barrier()
     ms_total = t_start.elapsed_time(t_end)
-    ms_ext = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
-    ms_sel = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
-    ms_att = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
     ms_total = max_over_ranks(ms_total, dev)
+    n_after = args.warmup + args.steps  # steps appended so far (for the phase loop below)
     ms_step = ms_total / args.steps
     queries_per_step = B * Hq
     value = throughput(queries_per_step, args.steps, world, ms_total)
@@ -675,6 +696,24 @@ def run_zha(args, rank, world, dev):
     z.zha_decode_select(cfg, cache, step_inputs(args.warmup + args.steps - 1)[3], c.p, lc, ws, st)
     torch.cuda.synchronize()
     per_query = selection_per_query(lc.cpu(), b, L, n_last, D * 2)
+
+    # ---- phase split: the same steps eagerly on one stream, select and attend
+    # apart (the roofline of each kernel group; not the headline) ----
+    nph = min(20, args.steps)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nph)]
+    for i in range(nph):
+        load_inputs(n_after + i)
+        ev = evs[i]
+        ev[0].record(stream)
+        z.zha_extend_tree(cfg, cache, old_st, 1)
+        ev[1].record(stream)
+        z.zha_decode_select(cfg, cache, q_st, c.p, None, ws, st)
+        ev[2].record(stream)
+        z.zha_decode_attend(cfg, cache, q_st, out, ws)
+        ev[3].record(stream)
+    torch.cuda.synchronize()
+    ms_ext, ms_sel, ms_att = (sum(e[a].elapsed_time(e[a + 1]) for e in evs) / nph
+                              for a in range(3))
     ext_bytes = 0
     step_bytes = sel_bytes + att_bytes + ext_bytes
     peak, peak_kind = measured_peaks()
@@ -766,7 +805,10 @@ def run_zha(args, rank, world, dev):
                        "tokens": n_tok},
         "e2e": {"value": queries_per_step * world / (e2e_ms / 1e3), "unit": "queries/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": 6 * args.steps,  # extend, score, cut, union, attention, combine
+        # per step: the extension, and per unit group (the library forms up to 4
+        # groups of at least 2 (sequence, KV head) units) score, cut, union,
+        # attention and combine
+        "gpu_launches": (1 + 5 * min(4, max(1, B * Hkv // 2))) * args.steps,
         "clocks": clocks,
     }
     if args.n_tokens is None:  # the other workloads at their full sizes

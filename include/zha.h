@@ -30,9 +30,11 @@
  * Conventions for every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller (for example
  *     PyTorch tensors), contiguous, 16-byte aligned. The library never
- *     allocates, never synchronises the device and keeps no state between
- *     calls; it is re-entrant (zha_decode_noalloc, which works in a static
- *     device array instead of a caller workspace, is the one exception).
+ *     allocates device memory and never synchronises the device. The only
+ *     state it keeps between calls is, per device, the streams and events
+ *     zha_decode forks its unit groups onto (created on its first call there)
+ *     and zha_decode_noalloc's static array. Every entry point is re-entrant
+ *     except zha_decode_noalloc (one array per device).
  *   - `stream` is a cudaStream_t passed as void*; every call is asynchronous on
  *     it.
  *   - Argument errors return synchronously before any launch
@@ -171,7 +173,16 @@ zha_status zha_attend(const zha_config* cfg, const zha_cache* cache, const void*
  * The query heads sharing a KV head are traversed together and their
  * selections are read from HBM once (per-head masks). level_counts is
  * nullable. The tree must already contain every node complete at seq_len
- * (call zha_extend_tree after appending tokens). ws: ZHA_OP_DECODE workspace. */
+ * (call zha_extend_tree after appending tokens). ws: ZHA_OP_DECODE workspace.
+ * Streams: the (sequence, KV head) units are split into up to 4 groups whose
+ * kernels run on streams of decreasing priority that the library creates
+ * once per device (forked from `stream` by an event and joined back into it
+ * before the call returns), so that one group's cut overlaps the other
+ * groups' scoring and attention. Work queued on `stream` after the call
+ * waits for all of it, and the call can be captured into a CUDA graph; the
+ * streams are created by the first call on a device that is not being
+ * captured (until then the call runs on `stream` alone). Outputs equal those
+ * of zha_decode_select followed by zha_decode_attend bit for bit. */
 zha_status zha_decode(const zha_config* cfg, const zha_cache* cache, const void* q, double p,
                       void* out, int32_t* level_counts, void* ws, size_t ws_bytes,
                       int32_t* dev_status, void* stream);
@@ -273,7 +284,8 @@ zha_status zha_decode_kept_lists(const zha_config* cfg, const zha_cache* cache, 
  * device memory instead of ws; nothing is allocated by the call.
  *   - Limit: geometries whose ZHA_OP_DECODE workspace (zha_workspace_bytes)
  *     exceeds 64 MiB are rejected with ZHA_ERR_WORKSPACE before any launch
- *     (for example B = 1, Hkv = 2, G = 8, b = 4 fits up to about 180K tokens).
+ *     (for example B = 1, Hkv = 2, G = 8, b = 4, L = 6 fits up to about 2.19M
+ *     tokens).
  *   - Set-up: the first call on each device looks up the array's device
  *     address (this loads its module on that device); make that first call
  *     with the device current and outside any stream capture. The address is
@@ -284,6 +296,8 @@ zha_status zha_decode_kept_lists(const zha_config* cfg, const zha_cache* cache, 
  *     ran on hold them; with CUDA_MODULE_LOADING=EAGER every process that
  *     loads libzha holds them on every device it uses.
  *   - The scratch needs no clearing: every word is written before it is read.
+ *   - Every launch runs on `stream` itself: unlike zha_decode, this call uses
+ *     no streams or events of the library's own.
  *   - Unlike the other entry points this one is NOT re-entrant: every call on
  *     a device shares the one array, so two calls whose executions overlap
  *     (different streams, or different host threads, without ordering between

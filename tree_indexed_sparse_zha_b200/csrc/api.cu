@@ -5,6 +5,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "zha_internal.h"
 
 namespace zha {
@@ -86,7 +88,22 @@ struct DecodeLayout {
   size_t trav, kept, n_kept, stats, part, total;
   int64_t units;
   bool dense;  // selection by decode_dense (decode steps), else the frontier traversal
+  int groups;  // unit groups of a decode step
 };
+
+// Unit groups of a decode step on the dense path (see run_decode_step).
+#ifndef ZHA_DECODE_GROUPS
+#define ZHA_DECODE_GROUPS 4
+#endif
+constexpr int kDecodeGroups = ZHA_DECODE_GROUPS;
+constexpr int kMinUnitsPerGroup = 2;
+
+static int decode_groups(bool dense, int64_t units) {
+  if (!dense) return 1;
+  int64_t k = units / kMinUnitsPerGroup;
+  if (k > kDecodeGroups) k = kDecodeGroups;
+  return k < 1 ? 1 : (int)k;
+}
 
 // dense: the caller is a decode step (one query per sequence at seq_len - 1)
 static DecodeLayout decode_layout(const Geometry& g, int64_t nq, int kind, int sms,
@@ -94,6 +111,7 @@ static DecodeLayout decode_layout(const Geometry& g, int64_t nq, int kind, int s
   DecodeLayout L{};
   L.units = nq * g.Hkv;
   L.dense = decode && decode_dense_ok(g, L.units);
+  L.groups = decode_groups(L.dense, L.units);
   size_t off = 0;
   L.trav = off;
   off = align256(off + (L.dense ? decode_dense_ws_bytes(g, L.units)
@@ -353,6 +371,123 @@ static zha_status run_tree_decode(const Geometry& g, const zha_cache* cache, con
   return run_tree_attend(g, cache, q, q_seq, q_pos, nq, out, ws, L, sms, s);
 }
 
+// ---- decode step over groups of units on concurrent streams -----------------
+//
+// A decode step's cut runs one CTA per query head and is bound by its chain of
+// dependent passes, not by the SM count; the scoring and the attention around
+// it are bound by HBM. So the units of a step are cut into groups, each with a
+// stream of its own, at decreasing priorities (group 0 highest): a group
+// scores, cuts, merges and attends, and the block scheduler serves the
+// earlier groups first, so one group's cut overlaps the later groups' scoring
+// and the earlier groups' attention. Every kernel computes per unit exactly
+// what the single-stream order computes (the attention keeps the split count
+// of the whole step), so the outputs are the same bit for bit.
+constexpr int kPipeDevices = 64;
+
+struct DecodePipe {
+  bool ready;
+  cudaStream_t s[kDecodeGroups];
+  cudaEvent_t fork, done[kDecodeGroups];
+};
+static std::mutex g_pipe_mutex;  // held while a step's launches are enqueued
+static DecodePipe g_pipe[kPipeDevices];
+
+// Streams and events of the current device, created on first use and kept for
+// the life of the process (nullptr when they cannot be had, or when they would
+// have to be created while `s` is being captured into a graph).
+static DecodePipe* decode_pipe(cudaStream_t s) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kPipeDevices) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  DecodePipe& P = g_pipe[dev];
+  if (P.ready) return &P;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  int least = 0, greatest = 0;
+  if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  bool ok = cudaEventCreateWithFlags(&P.fork, cudaEventDisableTiming) == cudaSuccess;
+  for (int k = 0; ok && k < kDecodeGroups; ++k) {
+    const int prio = greatest + k < least ? greatest + k : least;
+    ok = cudaStreamCreateWithPriority(&P.s[k], cudaStreamNonBlocking, prio) == cudaSuccess &&
+         cudaEventCreateWithFlags(&P.done[k], cudaEventDisableTiming) == cudaSuccess;
+  }
+  if (!ok) {  // what was created stays (a few handles); the step runs on one stream
+    cudaGetLastError();
+    return nullptr;
+  }
+  P.ready = true;
+  return &P;
+}
+
+static zha_status run_dense_decode_grouped(const Geometry& g, const zha_cache* cache,
+                                           const void* q, uint64_t p_q, void* out,
+                                           int32_t* level_counts, unsigned char* ws,
+                                           const DecodeLayout& L, int32_t* dev_status, int sms,
+                                           cudaStream_t s, int K, DecodePipe& P) {
+  AttendArgs a{};
+  a.kind = kStreamTree;
+  a.k = cache->k;
+  a.v = cache->v;
+  a.q = q;
+  a.out = out;
+  a.seq_len = cache->seq_len;
+  a.nq = g.B;
+  a.kept = reinterpret_cast<const uint32_t*>(ws + L.kept);
+  a.n_kept = reinterpret_cast<const int32_t*>(ws + L.n_kept);
+  a.kept_stride = traverse_kept_stride(g);
+  a.kept_segs = traverse_cluster_size(g, L.units, sms);
+  cudaError_t err = cudaEventRecord(P.fork, s);
+  int launched = 0;  // groups whose stream joined the step
+  for (int k = 0; k < K && err == cudaSuccess; ++k) {
+    const int64_t u0 = L.units * k / K, u1 = L.units * (k + 1) / K;
+    cudaStream_t sk = P.s[k];
+    err = cudaStreamWaitEvent(sk, P.fork, 0);
+    if (err != cudaSuccess) break;
+    launched = k + 1;
+    err = launch_decode_dense(g, cache->tree, q, cache->seq_len, p_q, ws + L.trav, level_counts,
+                              reinterpret_cast<int32_t*>(ws + L.stats),
+                              reinterpret_cast<uint32_t*>(ws + L.kept),
+                              reinterpret_cast<int32_t*>(ws + L.n_kept), a.kept_stride,
+                              a.kept_segs, dev_status, sms, sk, u0, u1 - u0);
+    if (err != cudaSuccess) break;
+    a.unit0 = u0;
+    a.n_units = u1 - u0;
+    err = launch_attend(g, a, ws + L.part, L.total - L.part, sms, sk);
+  }
+  // join every stream that took part, also after a failed launch
+  for (int k = 0; k < launched; ++k) {
+    const cudaError_t e1 = cudaEventRecord(P.done[k], P.s[k]);
+    const cudaError_t e2 = e1 == cudaSuccess ? cudaStreamWaitEvent(s, P.done[k], 0) : e1;
+    if (err == cudaSuccess) err = e2;
+  }
+  return cuda_status(err);
+}
+
+// A decode step: the grouped form when the selection takes the dense path and
+// the streams can be had, else select then attend on the caller's stream.
+static zha_status run_decode_step(const Geometry& g, const zha_cache* cache, const void* q,
+                                  uint64_t p_q, void* out, int32_t* level_counts,
+                                  unsigned char* ws, const DecodeLayout& L, int32_t* dev_status,
+                                  int sms, cudaStream_t s, bool concurrent) {
+  const int K = concurrent ? L.groups : 1;
+  if (K > 1) {
+    std::lock_guard<std::mutex> lock(g_pipe_mutex);
+    DecodePipe* P = decode_pipe(s);
+    if (P) return run_dense_decode_grouped(g, cache, q, p_q, out, level_counts, ws, L, dev_status,
+                                           sms, s, K, *P);
+  }
+  return run_tree_decode(g, cache, q, nullptr, nullptr, g.B, p_q, out, level_counts, ws, L,
+                         dev_status, sms, s);
+}
+
 __global__ void decode_stats_kernel(const int32_t* stats, const int32_t* n_kept, int units, int L,
                                     int segs, int32_t* out) {
   const int u = blockIdx.x * blockDim.x + threadIdx.x;
@@ -363,9 +498,9 @@ __global__ void decode_stats_kernel(const int32_t* stats, const int32_t* n_kept,
   out[(int64_t)u * (L + 1) + L] = kept;
 }
 
-zha_status zha_decode(const zha_config* cfg, const zha_cache* cache, const void* q, double p,
-                      void* out, int32_t* level_counts, void* ws, size_t ws_bytes,
-                      int32_t* dev_status, void* stream) {
+static zha_status decode_impl(const zha_config* cfg, const zha_cache* cache, const void* q,
+                              double p, void* out, int32_t* level_counts, void* ws,
+                              size_t ws_bytes, int32_t* dev_status, void* stream, bool concurrent) {
   Geometry g;
   zha_status st = make_geometry(cfg, &g);
   if (st != ZHA_OK) return st;
@@ -375,9 +510,14 @@ zha_status zha_decode(const zha_config* cfg, const zha_cache* cache, const void*
   const int sms = device_sm_count();
   const DecodeLayout L = decode_layout(g, g.B, kStreamTree, sms, true);
   if (ws_bytes < L.total) return ZHA_ERR_WORKSPACE;
-  return run_tree_decode(g, cache, q, nullptr, nullptr, g.B, p_q, out, level_counts,
-                         static_cast<unsigned char*>(ws), L, dev_status, sms,
-                         (cudaStream_t)stream);
+  return run_decode_step(g, cache, q, p_q, out, level_counts, static_cast<unsigned char*>(ws), L,
+                         dev_status, sms, (cudaStream_t)stream, concurrent);
+}
+
+zha_status zha_decode(const zha_config* cfg, const zha_cache* cache, const void* q, double p,
+                      void* out, int32_t* level_counts, void* ws, size_t ws_bytes,
+                      int32_t* dev_status, void* stream) {
+  return decode_impl(cfg, cache, q, p, out, level_counts, ws, ws_bytes, dev_status, stream, true);
 }
 
 zha_status zha_decode_select(const zha_config* cfg, const zha_cache* cache, const void* q,
@@ -558,3 +698,13 @@ zha_status zha_dense_decode(const zha_config* cfg, const zha_cache* cache, const
 }
 
 }  // extern "C"
+
+namespace zha {
+
+zha_status decode_one_stream(const zha_config* cfg, const zha_cache* cache, const void* q,
+                             double p, void* out, int32_t* level_counts, void* ws,
+                             size_t ws_bytes, int32_t* dev_status, void* stream) {
+  return decode_impl(cfg, cache, q, p, out, level_counts, ws, ws_bytes, dev_status, stream, false);
+}
+
+}  // namespace zha

@@ -56,6 +56,7 @@ struct AttParams {
   int64_t idx_cap;
   const int32_t* n_idx;
   int S;                   // splits per unit
+  int unit0;               // first unit of this launch (grid: its units x S)
   float* part;             // [units][S][G][D + 2]
 };
 
@@ -160,7 +161,7 @@ __global__ void __launch_bounds__(Cfg<T, D>::kThreads, 1) attend_kernel(AttParam
   unsigned char* my = wbase + warp * C::kWarpBytes;
   float2* pbuf = reinterpret_cast<float2*>(my + 2 * C::kStageBytes);  // [32][8]
 
-  const int unit = blockIdx.x / p.S;
+  const int unit = p.unit0 + (int)(blockIdx.x / p.S);
   const int split = blockIdx.x % p.S;
   const uint32_t all = (1u << G) - 1u;
 
@@ -488,7 +489,7 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads, 1) attend_mma_kernel(AttP
   unsigned char* my = smem + warp * C::kWarpBytes;
   uint8_t* rmask = my + C::kStages * C::kStageBytes;  // [stage][32]
 
-  const int unit = blockIdx.x / p.S;
+  const int unit = p.unit0 + (int)(blockIdx.x / p.S);
   const int split = blockIdx.x % p.S;
   const uint32_t all = (1u << G) - 1u;
 
@@ -744,7 +745,7 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads, 1) attend_mma_kernel(AttP
 // Merge the S split partials of each (unit, head) and write the output row.
 template <typename T, int D, int G>
 __global__ void combine_kernel(AttParams p, void* out_v) {
-  const int unit = blockIdx.x / G;
+  const int unit = p.unit0 + (int)(blockIdx.x / G);
   const int h = blockIdx.x % G;
   const int i = threadIdx.x;
   const float* base = p.part + (int64_t)unit * p.S * G * (D + 2);
@@ -863,8 +864,11 @@ cudaError_t launch_attend(const Geometry& g, const AttendArgs& a, void* ws, size
   p.n_idx = a.n_idx;
   p.S = splits_of(g, a.kind, a.nq, num_sms);
   p.part = static_cast<float*>(ws);
-  const int64_t units = units_of(g, a.kind, a.nq);
+  const int64_t all_units = units_of(g, a.kind, a.nq);
+  const int64_t units = a.n_units > 0 ? a.n_units : all_units;
+  p.unit0 = (int)a.unit0;
   if (units <= 0) return cudaSuccess;
+  if (a.unit0 < 0 || a.unit0 + units > all_units) return cudaErrorInvalidValue;
   if (g.dtype == ZHA_BF16) {
     if (g.d == 128) return launch_g<__nv_bfloat16, 128>(p.G, p, units, a.out, stream);
     return launch_g<__nv_bfloat16, 64>(p.G, p, units, a.out, stream);

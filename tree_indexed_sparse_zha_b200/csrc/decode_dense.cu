@@ -15,11 +15,14 @@
 //      levels top-down: its frontier at a level is the children of the nodes it
 //      kept one level up, and the canonical top-p cut of the frontier (exact
 //      fixed-point masses, ties to the lower node) is found from the stored
-//      scores with CTA-local passes only. The descent is exactly the method's;
-//      scores of nodes outside the frontier are computed but never read.
-//   3. union_kernel -- the heads' kept level-1 nodes of a (sequence, KV head)
-//      are merged into one ascending list with an 8-bit head mask per node, in
-//      the segments the decode attention reads.
+//      scores with CTA-local passes only, as a threshold (key*, node*) on the
+//      frontier's (score desc, node asc) order. The descent is exactly the
+//      method's; scores of nodes outside the frontier are computed but never
+//      read. Levels L..2 list their kept nodes; level 1 stops at its threshold.
+//   3. union_kernel -- many CTAs per (sequence, KV head) apply every head's
+//      level-1 threshold to the children of that head's kept level-2 nodes and
+//      merge the heads' kept level-1 nodes into one ascending list with an
+//      8-bit head mask per node, in the segments the decode attention reads.
 // Reading every row under the complete top nodes costs the same bytes as
 // reading the union of the heads' frontiers whenever that union covers the
 // tree (as on diffuse queries), and it removes the per-level dependence of
@@ -58,8 +61,9 @@ struct DenseParams {
   int keep_all;
   int32_t* klist;          // [units][G][2][klcap] kept nodes, ascending
   int64_t klcap;
-  uint32_t* bitmap;        // [units][G][bmw] kept level-1 nodes
+  uint32_t* bitmap;        // [units][G][bmw] kept level-2 nodes (L >= 2)
   int64_t bmw;
+  uint4* cutpar;           // [units][G] level-1 cut: mode, key*, node*, kept count
   int32_t* level_counts;   // [B][Hq][L] (nullable)
   int32_t* status;
   // union
@@ -67,6 +71,7 @@ struct DenseParams {
   int32_t* n_kept;         // [units][segs]
   int64_t kept_stride;
   int segs;
+  int unit0;               // first unit of this launch (grid y: its units)
 };
 
 // Complete top nodes visible to the decode query of sequence `seq` (at
@@ -128,7 +133,7 @@ __global__ void __launch_bounds__(kSThreads, 3) dense_score_kernel(const __grid_
   constexpr int kPer = C::kPer, kSteps = C::kSteps;
   extern __shared__ __align__(16) unsigned char sm[];
   float* qs = reinterpret_cast<float*>(sm + 2 * kSStageBytes);  // [D][8]
-  const int unit = blockIdx.y;
+  const int unit = p.unit0 + (int)blockIdx.y;
   const int seq = unit / p.Hkv, kvh = unit % p.Hkv;
   const int tid = threadIdx.x;
   const int64_t T_top = decode_top(p, seq);
@@ -312,7 +317,7 @@ struct CutSmem {
   unsigned int thr_key, thr_node, tie_n, rank_hit;
   int ok;
 };
-// the level-1 bitmap of the head follows the struct (bmw words)
+// the head's level-2 kept bitmap follows the struct (bmw words)
 
 enum CutMode : unsigned { kCutAll = 0, kCutThr = 1, kCutTie = 2 };
 
@@ -613,24 +618,84 @@ __device__ void rank_group(CutSmem& S, int n, float zmax, unsigned long long abo
   __syncthreads();
 }
 
+// The candidates of one iteration (as load_slots gives them) with their keep
+// bits -- key > key*, or key == key* and node <= node*; every candidate in
+// kCutAll -- and their exact-tie bits (key == key*). by_bytes: every candidate
+// outside the crossing bucket beta is decided by its bucket byte, and scores
+// are loaded only for the items that hold members of beta.
+__device__ __forceinline__ void classify(const CutSmem& S, const Frontier& V, int64_t base,
+                                         bool by_bytes, const uint32_t* qbw, unsigned mode,
+                                         uint32_t thr_key, uint32_t thr_node, uint32_t beta,
+                                         Slots& q, uint32_t* keepm, uint32_t* tiem) {
+  uint32_t km = 0, tm = 0;
+  if (by_bytes) {
+    const int64_t i0 = base + (int64_t)threadIdx.x * V.U;
+    uint32_t n0[kCU];
+    int cnt[kCU];
+    uint32_t qw[kCU];
+    load_item_nodes(V, i0, n0, cnt);
+#pragma unroll
+    for (int u = 0; u < kCU; ++u) qw[u] = cnt[u] ? qbw[i0 + u] : 0u;
+    const uint32_t bpat = beta * 0x01010101u;
+    float4 zz[kCU];
+#pragma unroll
+    for (int u = 0; u < kCU; ++u)
+      zz[u] = (cnt[u] && __vcmpeq4(qw[u], bpat)) ? load_z4(V.zl, n0[u])
+                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    q.valid = 0;
+#pragma unroll
+    for (int u = 0; u < kCU; ++u)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int sl = 4 * u + c;
+        q.nd[sl] = n0[u] + c;
+        if (c >= cnt[u]) continue;
+        q.valid |= 1u << sl;
+        const uint32_t d = (qw[u] >> (8 * c)) & 0xffu;
+        if (d > beta) {
+          km |= 1u << sl;
+        } else if (d == beta) {
+          const uint32_t key = order_key(f4get(zz[u], c));
+          const bool gt = key > thr_key, eq = key == thr_key;
+          km |= (gt || (eq && mode == kCutThr && q.nd[sl] <= thr_node) ? 1u : 0u) << sl;
+          tm |= (eq ? 1u : 0u) << sl;
+        }
+      }
+  } else {
+    load_slots(S, V, base, q);
+#pragma unroll
+    for (int sl = 0; sl < 4 * kCU; ++sl) {
+      if (!((q.valid >> sl) & 1u)) continue;
+      const uint32_t key = order_key(q.z[sl]);
+      const bool gt = key > thr_key, eq = key == thr_key;
+      km |= (mode == kCutAll || gt || (eq && mode == kCutThr && q.nd[sl] <= thr_node) ? 1u : 0u)
+            << sl;
+      tm |= (eq ? 1u : 0u) << sl;
+    }
+  }
+  *keepm = km;
+  *tiem = tm;
+}
+
 __global__ void __launch_bounds__(kCThreads, 1) head_cut_kernel(const __grid_constant__ DenseParams p) {
   extern __shared__ __align__(16) unsigned char smc[];
   CutSmem& S = *reinterpret_cast<CutSmem*>(smc);
-  uint32_t* bm1 = reinterpret_cast<uint32_t*>(smc + ((sizeof(CutSmem) + 15) & ~(size_t)15));
-  const int h = blockIdx.x, unit = blockIdx.y;
+  uint32_t* bm2 = reinterpret_cast<uint32_t*>(smc + ((sizeof(CutSmem) + 15) & ~(size_t)15));
+  const int h = blockIdx.x, unit = p.unit0 + (int)blockIdx.y;
   const int G = p.G, b = p.b, L = p.L;
   const int seq = unit / p.Hkv, kvh = unit % p.Hkv;
   const int tid = threadIdx.x;
   const int64_t T_top = decode_top(p, seq);
-  const int64_t n1 = T_top * p.span[L - 1];  // level-1 nodes under complete top nodes
-  const int64_t words = (n1 + 31) / 32;
+  // level-2 nodes under complete top nodes, kept ones as bits
+  const int64_t words2 = L >= 2 ? (T_top * p.span[L - 2] + 31) / 32 : 0;
   int32_t* lc = p.level_counts && seq >= 0 && seq < p.B
                     ? p.level_counts + ((int64_t)seq * p.Hq + (int64_t)kvh * G + h) * L
                     : nullptr;
   uint32_t* gbm = p.bitmap + ((int64_t)unit * G + h) * p.bmw;
-  for (int64_t w = tid; w < words; w += kCThreads) bm1[w] = 0u;
+  for (int64_t w = tid; w < words2; w += kCThreads) bm2[w] = 0u;
   if (T_top == 0) {
     if (lc && tid < L) lc[tid] = 0;
+    if (tid == 0) p.cutpar[(int64_t)unit * G + h] = make_uint4(kCutAll, 0u, 0u, 0u);
     return;
   }
   // kept nodes in global memory, two buffers: a streamed level reads its
@@ -751,13 +816,16 @@ __global__ void __launch_bounds__(kCThreads, 1) head_cut_kernel(const __grid_con
           S.ok = ok;
           S.beta = beta;
           S.above = ab;
+          S.cabove = 0u;  // counted by the gather below (this pass counts no members)
           S.bmass = ok ? S.bm[beta] : 0ull;
         }
       }
       __syncthreads();
-      // -- the crossing bucket's members into the list (counted past its end) --
+      // -- the crossing bucket's members into the list (counted past its end),
+      //    and the count of the candidates in the buckets above it --
       if (S.ok) {
         const unsigned beta = S.beta;
+        unsigned n_above = 0;
         if (qb_ok) {  // from the bucket bytes; scores only for the members
           const uint32_t bpat = beta * 0x01010101u;
           for (int64_t base = 0; base < V.nItems; base += stride) {
@@ -769,7 +837,9 @@ __global__ void __launch_bounds__(kCThreads, 1) head_cut_kernel(const __grid_con
 #pragma unroll
             for (int u = 0; u < kCU; ++u) {
               const bool in = u < V.U && i0 + u < V.nItems;
-              eqm[u] = in ? __vcmpeq4(qbw[i0 + u], bpat) : 0u;
+              const uint32_t w = in ? qbw[i0 + u] : 0u;  // absent candidates hold byte 0
+              eqm[u] = in ? __vcmpeq4(w, bpat) : 0u;
+              n_above += (unsigned)__popc(__vcmpgtu4(w, bpat)) >> 3;
               anym |= eqm[u] != 0u;
             }
             if (!anym) continue;
@@ -795,13 +865,19 @@ __global__ void __launch_bounds__(kCThreads, 1) head_cut_kernel(const __grid_con
             load_slots(S, V, base, q);
 #pragma unroll
             for (int sl = 0; sl < 4 * kCU; ++sl) {
-              if (!((q.valid >> sl) & 1u) || quant_bucket(q.z[sl], zlo, zscale) != beta) continue;
+              if (!((q.valid >> sl) & 1u)) continue;
+              const uint32_t d = quant_bucket(q.z[sl], zlo, zscale);
+              n_above += d > beta ? 1u : 0u;
+              if (d != beta) continue;
               const unsigned slot = atomicAdd(&S.n_list, 1u);
               if (slot < (unsigned)kCList)
                 S.list[slot] = ((unsigned long long)order_key(q.z[sl]) << 32) | (0xffffffffu - q.nd[sl]);
             }
           }
         }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) n_above += __shfl_xor_sync(0xffffffffu, n_above, off);
+        if ((tid & 31) == 0 && n_above) atomicAdd(&S.cabove, n_above);
       }
       __syncthreads();
       // -- a group too large to rank: narrow it by key digits, then gather again --
@@ -849,6 +925,7 @@ __global__ void __launch_bounds__(kCThreads, 1) head_cut_kernel(const __grid_con
                 const uint32_t dlo = topb | (dig << sh);
                 const uint32_t dhi = dlo | (uint32_t)((1ull << sh) - 1ull);
                 S.above = ab;
+                S.cabove += ca;
                 S.bcnt = S.bc[dig];
                 S.bmass = S.bm[dig];
                 S.kgmin = dlo > kgmin ? dlo : kgmin;
@@ -890,6 +967,7 @@ __global__ void __launch_bounds__(kCThreads, 1) head_cut_kernel(const __grid_con
             S.mode = kCutThr;
             S.thr_key = (uint32_t)(S.srt[r] >> 32);
             S.thr_node = 0xffffffffu - (uint32_t)S.srt[r];
+            S.count = S.cabove + r + 1u;
           }
         }
       } else if (S.ok && S.kgmin == S.kgmax) {
@@ -900,6 +978,7 @@ __global__ void __launch_bounds__(kCThreads, 1) head_cut_kernel(const __grid_con
           S.mode = kCutTie;
           S.tie_n = (unsigned)(tn < S.bcnt ? tn : S.bcnt);
           S.thr_key = S.kgmin;
+          S.count = S.cabove + S.tie_n;
         }
       } else if (tid == 0) {
         S.ok = 0;
@@ -914,107 +993,78 @@ __global__ void __launch_bounds__(kCThreads, 1) head_cut_kernel(const __grid_con
       }
       __syncthreads();
     }
-    // -- emit the kept nodes in frontier (= node) order: key > key*, or key ==
-    //    key* and node <= node* (exact ties: the first tie_n in node order) --
-    const unsigned mode = S.mode;
-    const unsigned thr_key = S.thr_key, thr_node = S.thr_node, tie_n = S.tie_n, beta = S.beta;
-    const bool by_bytes = qb_ok && mode != kCutAll;
-    unsigned run = 0, tie_run = 0;
-    for (int64_t base = 0; base < V.nItems; base += stride) {
-      Slots q;
-      uint32_t keepm = 0, tiem = 0;  // bit = slot
-      if (by_bytes) {
-        // bucket bytes decide every candidate outside the crossing bucket;
-        // scores are loaded only for the items holding members of it
-        const int64_t i0 = base + (int64_t)tid * V.U;
-        uint32_t n0[kCU];
-        int cnt[kCU];
-        uint32_t qw[kCU];
-        load_item_nodes(V, i0, n0, cnt);
-#pragma unroll
-        for (int u = 0; u < kCU; ++u) qw[u] = cnt[u] ? qbw[i0 + u] : 0u;
-        const uint32_t bpat = beta * 0x01010101u;
-        float4 zz[kCU];
-#pragma unroll
-        for (int u = 0; u < kCU; ++u)
-          zz[u] = (cnt[u] && __vcmpeq4(qw[u], bpat)) ? load_z4(V.zl, n0[u])
-                                                     : make_float4(0.f, 0.f, 0.f, 0.f);
-        q.valid = 0;
-#pragma unroll
-        for (int u = 0; u < kCU; ++u)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int sl = 4 * u + c;
-            q.nd[sl] = n0[u] + c;
-            if (c >= cnt[u]) continue;
-            q.valid |= 1u << sl;
-            const uint32_t d = (qw[u] >> (8 * c)) & 0xffu;
-            if (d > beta) {
-              keepm |= 1u << sl;
-            } else if (d == beta) {
-              const uint32_t key = order_key(f4get(zz[u], c));
-              const bool gt = key > thr_key, eq = key == thr_key;
-              const bool k = gt || (eq && mode == kCutThr && q.nd[sl] <= thr_node);
-              keepm |= (k ? 1u : 0u) << sl;
-              tiem |= (eq && mode == kCutTie ? 1u : 0u) << sl;
-            }
-          }
-      } else {
-        load_slots(S, V, base, q);
-#pragma unroll
-        for (int sl = 0; sl < 4 * kCU; ++sl) {
-          if (!((q.valid >> sl) & 1u)) continue;
-          const uint32_t key = order_key(q.z[sl]);
-          const bool gt = key > thr_key, eq = key == thr_key;
-          const bool k = mode == kCutAll || gt || (eq && mode == kCutThr && q.nd[sl] <= thr_node);
-          keepm |= (k ? 1u : 0u) << sl;
-          tiem |= (eq && mode == kCutTie ? 1u : 0u) << sl;
-        }
-      }
-      if (mode == kCutTie) {  // exact ties: the first tie_n in node order
+    // -- exact ties (one key, too many members to rank): the tie_n-th of them
+    //    in frontier (= node) order becomes the node threshold --
+    if (S.mode == kCutTie) {
+      const unsigned thr_key = S.thr_key, tie_n = S.tie_n, beta = S.beta;
+      unsigned tie_run = 0;
+      for (int64_t base = 0; base < V.nItems && tie_run < tie_n; base += stride) {
+        Slots q;
+        uint32_t keepm, tiem;
+        classify(S, V, base, qb_ok, qbw, kCutTie, thr_key, 0u, beta, q, &keepm, &tiem);
         unsigned tot;
         unsigned rk = tie_run + block_scan(S, __popc(tiem), &tot, 1);
 #pragma unroll
         for (int sl = 0; sl < 4 * kCU; ++sl)
           if ((tiem >> sl) & 1u) {
-            keepm |= (rk < tie_n ? 1u : 0u) << sl;
-            ++rk;
+            if (++rk == tie_n) S.thr_node = q.nd[sl];
           }
         tie_run += tot;
       }
+      __syncthreads();
+      if (tid == 0) S.mode = kCutThr;
+      __syncthreads();
+    }
+    // the level's kept count: the candidates above the group and the group's
+    // members up to the threshold (every candidate when nothing is cut)
+    const unsigned kept_n = S.mode == kCutAll ? (unsigned)nF : S.count;
+    if (level == 1) {  // the union kernel applies the threshold to the level-1 frontier
+      if (tid == 0) {
+        p.cutpar[(int64_t)unit * G + h] = make_uint4(S.mode, S.thr_key, S.thr_node, kept_n);
+        if (lc) lc[L - 1] = (int32_t)kept_n;
+      }
+      break;
+    }
+    // -- emit the kept nodes in frontier (= node) order: key > key*, or key ==
+    //    key* and node <= node* (the level-2 ones also as bits) --
+    const unsigned mode = S.mode;
+    const unsigned thr_key = S.thr_key, thr_node = S.thr_node, beta = S.beta;
+    unsigned run = 0;
+    for (int64_t base = 0; base < V.nItems; base += stride) {
+      Slots q;
+      uint32_t keepm, tiem;
+      classify(S, V, base, qb_ok && mode != kCutAll, qbw, mode, thr_key, thr_node, beta, q,
+               &keepm, &tiem);
       unsigned tot;
       unsigned pos = run + block_scan(S, __popc(keepm), &tot, 0);
-      if (level > 1) {
+      uint32_t cw = 0xffffffffu, acc = 0;  // level 2: a bitmap word OR-ed while it stays
 #pragma unroll
-        for (int sl = 0; sl < 4 * kCU; ++sl)
-          if ((keepm >> sl) & 1u) {
-            kg_out[pos] = (int32_t)q.nd[sl];
-            // a cached frontier never reads S.ks, so it can take the list at once
-            if (cached && pos < (unsigned)kKCap) S.ks[pos] = (int32_t)q.nd[sl];
-            ++pos;
-          }
-      } else {  // level 1: bitmap words, OR-ed in a register while the word stays
-        uint32_t cw = 0xffffffffu, acc = 0;
-#pragma unroll
-        for (int sl = 0; sl < 4 * kCU; ++sl)
-          if ((keepm >> sl) & 1u) {
+      for (int sl = 0; sl < 4 * kCU; ++sl)
+        if ((keepm >> sl) & 1u) {
+          kg_out[pos] = (int32_t)q.nd[sl];
+          // a cached frontier never reads S.ks, so it can take the list at once
+          if (cached && pos < (unsigned)kKCap) S.ks[pos] = (int32_t)q.nd[sl];
+          ++pos;
+          if (level == 2) {
             const uint32_t w = q.nd[sl] >> 5;
             if (w != cw) {
-              if (acc) atomicOr(&bm1[cw], acc);
+              if (acc) atomicOr(&bm2[cw], acc);
               cw = w;
               acc = 0;
             }
             acc |= 1u << (q.nd[sl] & 31);
           }
-        if (acc) atomicOr(&bm1[cw], acc);
-      }
+        }
+      if (acc) atomicOr(&bm2[cw], acc);
       run += tot;
     }
-    if (tid == 0 && lc) lc[L - level] = (int32_t)run;
+    if (tid == 0) {
+      if (lc) lc[L - level] = (int32_t)run;
+      if (run != kept_n) raise_status(p.status, ZHA_ERR_INTERNAL);  // the count rule above
+    }
     n_prev = run;
     gsel ^= 1;
     __syncthreads();  // kept list complete
-    if (level == 1) break;
     if (!cached && run <= (unsigned)kKCap) {  // a streamed level's list into shared memory
       for (int64_t j = tid; j < run; j += kCThreads) S.ks[j] = __ldcg(kg_out + j);
       __syncthreads();
@@ -1055,45 +1105,87 @@ __global__ void __launch_bounds__(kCThreads, 1) head_cut_kernel(const __grid_con
     }
     __syncthreads();
   }
-  for (int64_t w = tid; w < words; w += kCThreads) gbm[w] = bm1[w];
+  __syncthreads();  // every level-2 bit is set
+  for (int64_t w = tid; w < words2; w += kCThreads) gbm[w] = bm2[w];
 }
 
 // ---------------------------------------------------------------------------
-// 3. union of the heads' kept level-1 nodes, in the decode attention's format
+// 3. the level-1 cut of every head applied, and the heads' kept level-1 nodes
+//    merged, in the decode attention's format
 // ---------------------------------------------------------------------------
-constexpr int kUThreads = 256;
+constexpr int kUThreads = 512;
+constexpr int kUNodes = 8;  // consecutive level-1 nodes per thread and iteration
 
-// One thread per 32-node bitmap word: the G heads' words are loaded at once,
-// the nodes any head keeps are counted, a block scan places them, and each
-// is written with the mask of the heads that keep it.
+// A thread takes 8 consecutive level-1 nodes n (starting at a multiple of 8,
+// within the CTA's share [lo, hi) of the unit): head h keeps n when h kept
+// its parent at level 2 (every node is a candidate when the tree has one
+// level) and its score passes h's level-1 threshold (key > key*, or key ==
+// key* and n <= node*; every candidate in kCutAll). The 8 nodes' parents lie
+// in one 32-bit word of each head's level-2 bitmap (b >= 2). Nodes any head
+// keeps are placed by a block scan, staged in shared memory and written in
+// node order as (head mask << 24) | n.
 __global__ void __launch_bounds__(kUThreads) union_kernel(const __grid_constant__ DenseParams p) {
   __shared__ unsigned int s_warp[kUThreads / 32];
-  __shared__ uint32_t s_out[32 * kUThreads];  // one iteration's entries, written out coalesced
-  const int r = blockIdx.x, unit = blockIdx.y;
+  __shared__ uint4 s_par[kMaxGroup];
+  __shared__ uint32_t s_out[kUThreads * kUNodes];
+  const int r = blockIdx.x, unit = p.unit0 + (int)blockIdx.y;
   const int seq = unit / p.Hkv;
   const int G = p.G;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t n1 = decode_top(p, seq) * p.span[p.L - 1];
   const int64_t lo = n1 * r / p.segs, hi = n1 * (r + 1) / p.segs;
   uint32_t* out = p.kept + ((int64_t)unit * p.segs + r) * p.kept_stride;
-  const uint32_t* bms = p.bitmap + (int64_t)unit * G * p.bmw;
-  const int64_t w_lo = lo / 32, w_hi = (hi + 31) / 32;
+  if (tid < G) s_par[tid] = p.cutpar[(int64_t)unit * G + tid];
+  __syncthreads();
+  const float* z1 = p.z + (int64_t)unit * G * p.zrows + p.zoff[0];
+  const uint32_t* bm2 = p.bitmap + (int64_t)unit * G * p.bmw;
+  const bool one_level = p.L == 1;
+  // b <= 32 is a power of two (parent = n >> bsh); a larger b is a multiple
+  // of 32, so the 8 nodes share one parent
+  const int bsh = p.b <= 32 ? __ffs(p.b) - 1 : -1;
   unsigned run = 0;
-  for (int64_t wb = w_lo; wb < w_hi; wb += kUThreads) {
-    const int64_t w = wb + tid;
-    uint32_t words[kMaxGroup];
-    uint32_t any = 0;
-    const int64_t n0 = w * 32;
+  for (int64_t nb = lo & ~(int64_t)(kUNodes - 1); nb < hi; nb += (int64_t)kUThreads * kUNodes) {
+    const int64_t n0 = nb + (int64_t)tid * kUNodes;
+    const uint32_t u0 = (uint32_t)n0;  // node ids fit in 24 bits
+    const uint32_t par0 = bsh >= 0 ? u0 >> bsh : u0 / (uint32_t)p.b;
+    uint32_t m[kUNodes];
 #pragma unroll
-    for (int h = 0; h < kMaxGroup; ++h) {
-      words[h] = (h < G && w < w_hi) ? __ldcg(bms + (int64_t)h * p.bmw + w) : 0u;
-      any |= words[h];
+    for (int j = 0; j < kUNodes; ++j) m[j] = 0u;
+    if (n0 < hi) {
+      // scores of the 8 nodes (the level's score vector is padded to 64 rows)
+      // and the parents' bitmap word, for every head at once
+      float4 za[kMaxGroup], zb[kMaxGroup];
+      uint32_t pw[kMaxGroup];
+#pragma unroll
+      for (int h = 0; h < kMaxGroup; ++h) {
+        const bool live = h < G && s_par[h].x != kCutAll;
+        const float4* zp = reinterpret_cast<const float4*>(z1 + (int64_t)h * p.zrows + n0);
+        za[h] = live ? __ldcg(zp) : make_float4(0.f, 0.f, 0.f, 0.f);
+        zb[h] = live ? __ldcg(zp + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+        pw[h] = h < G && !one_level ? __ldcg(bm2 + (int64_t)h * p.bmw + (par0 >> 5)) : 0xffffffffu;
+      }
+#pragma unroll
+      for (int h = 0; h < kMaxGroup; ++h) {
+        if (h >= G) continue;
+        const uint4 c = s_par[h];
+        const float zz[kUNodes] = {za[h].x, za[h].y, za[h].z, za[h].w,
+                                   zb[h].x, zb[h].y, zb[h].z, zb[h].w};
+#pragma unroll
+        for (int j = 0; j < kUNodes; ++j) {
+          const uint32_t par = bsh >= 0 ? (u0 + j) >> bsh : par0;
+          const bool cand = (pw[h] >> (par & 31)) & 1u;
+          const uint32_t key = order_key(zz[j]);
+          const bool keep = cand && (c.x == kCutAll || key > c.y || (key == c.y && u0 + j <= c.z));
+          m[j] |= (keep ? 1u : 0u) << h;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kUNodes; ++j)
+        if (n0 + j < lo || n0 + j >= hi) m[j] = 0u;  // outside the share
     }
-    if (w < w_hi) {  // keep the nodes of [lo, hi) only
-      if (n0 < lo) any &= ~0u << (uint32_t)(lo - n0);
-      if (n0 + 32 > hi) any &= (1u << (uint32_t)(hi - n0)) - 1u;
-    }
-    const unsigned f = __popc(any);
+    unsigned f = 0;
+#pragma unroll
+    for (int j = 0; j < kUNodes; ++j) f += m[j] ? 1u : 0u;
     unsigned x = f;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -1109,14 +1201,9 @@ __global__ void __launch_bounds__(kUThreads) union_kernel(const __grid_constant_
       tot += s_warp[w2];
     }
     unsigned pos = wbase + x - f;  // within this iteration's entries
-    while (any) {
-      const int i = __ffs(any) - 1;
-      any &= any - 1u;
-      uint32_t mask = 0;
 #pragma unroll
-      for (int h = 0; h < kMaxGroup; ++h) mask |= ((words[h] >> i) & 1u) << h;
-      s_out[pos++] = (mask << 24) | (uint32_t)(n0 + i);
-    }
+    for (int j = 0; j < kUNodes; ++j)
+      if (m[j]) s_out[pos++] = (m[j] << 24) | (u0 + (uint32_t)j);
     __syncthreads();
     for (unsigned e = tid; e < tot; e += kUThreads) out[run + e] = s_out[e];
     run += tot;
@@ -1149,7 +1236,7 @@ cudaError_t launch_score_g(const DenseParams& p, int units, int sms, cudaStream_
 }
 
 struct DenseLayout {
-  size_t z, klist, bitmap, total;
+  size_t z, klist, bitmap, cutpar, total;
   int64_t zrows, klcap, bmw;
   int64_t zoff[kMaxLevels];
 };
@@ -1163,7 +1250,7 @@ DenseLayout dense_layout(const Geometry& g, int64_t units) {
   }
   D.zrows = off + 64;  // the last level's vector loads may read 3 rows past its end
   D.klcap = (g.level_rows[0] + 63) / 64 * 64;
-  D.bmw = (g.level_rows[0] + 31) / 32 + 1;
+  D.bmw = g.L >= 2 ? (g.level_rows[1] + 31) / 32 + 1 : 1;
   auto a256 = [](size_t x) { return (x + 255) & ~(size_t)255; };
   size_t o = 0;
   D.z = o;
@@ -1172,6 +1259,8 @@ DenseLayout dense_layout(const Geometry& g, int64_t units) {
   o = a256(o + sizeof(int32_t) * (size_t)units * g.G * 2 * D.klcap);
   D.bitmap = o;
   o = a256(o + sizeof(uint32_t) * (size_t)units * g.G * D.bmw);
+  D.cutpar = o;
+  o = a256(o + sizeof(uint4) * (size_t)units * g.G);
   D.total = o;
   return D;
 }
@@ -1183,7 +1272,7 @@ size_t cut_smem_bytes(const Geometry& g) {
 }  // namespace
 
 bool decode_dense_ok(const Geometry& g, int64_t units) {
-  // the level-1 bitmap of a head lives in shared memory next to the cut state
+  // the level-2 bitmap of a head lives in shared memory next to the cut state
   if (cut_smem_bytes(g) > 227 * 1024) return false;
   // every row under the complete top nodes is read: keep that prefix within
   // what the frontier traversal's latency costs anyway (a few hundred us)
@@ -1200,9 +1289,11 @@ cudaError_t launch_decode_dense(const Geometry& g, const void* tree, const void*
                                 const int32_t* seq_len, uint64_t p_q, void* ws,
                                 int32_t* level_counts, int32_t* stats, uint32_t* kept,
                                 int32_t* n_kept, int64_t kept_stride, int segs, int32_t* status,
-                                int num_sms, cudaStream_t stream) {
-  const int64_t units = (int64_t)g.B * g.Hkv;
-  const DenseLayout Ly = dense_layout(g, units);
+                                int num_sms, cudaStream_t stream, int64_t unit0, int64_t n_units) {
+  const int64_t all_units = (int64_t)g.B * g.Hkv;
+  const int64_t units = n_units > 0 ? n_units : all_units;
+  if (unit0 < 0 || unit0 + units > all_units) return cudaErrorInvalidValue;
+  const DenseLayout Ly = dense_layout(g, all_units);
   unsigned char* w = static_cast<unsigned char*>(ws);
   DenseParams p{};
   p.tree = tree;
@@ -1232,12 +1323,14 @@ cudaError_t launch_decode_dense(const Geometry& g, const void* tree, const void*
   p.klcap = Ly.klcap;
   p.bitmap = reinterpret_cast<uint32_t*>(w + Ly.bitmap);
   p.bmw = Ly.bmw;
+  p.cutpar = reinterpret_cast<uint4*>(w + Ly.cutpar);
   p.level_counts = level_counts;
   p.status = status;
   p.kept = kept;
   p.n_kept = n_kept;
   p.kept_stride = kept_stride;
   p.segs = segs;
+  p.unit0 = (int)unit0;
   cudaError_t e;
   if (g.dtype == ZHA_BF16)
     e = g.d == 128 ? launch_score_g<__nv_bfloat16, 128>(p, (int)units, num_sms, stream)

@@ -16,10 +16,9 @@
 
 namespace {
 
-// Largest ZHA_OP_DECODE workspace this entry point serves. A decode of B
-// sequences at context n needs about B * Hkv * 16 * (n / b) * (8 + 4 G) bytes
-// (per-CTA frontier segments sized for the worst case), so this covers e.g.
-// B = 1, Hkv = 2, G = 8 up to about 180K tokens with b = 4.
+// Largest ZHA_OP_DECODE workspace this entry point serves (zha_workspace_bytes
+// gives a geometry's need): e.g. B = 1, Hkv = 2, G = 8, b = 4, L = 6 fits up
+// to about 2.19M tokens of context.
 constexpr size_t kStaticScratchBytes = size_t(64) << 20;
 
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
@@ -67,11 +66,12 @@ zha_status zha_decode_noalloc(const zha_config* cfg, const zha_cache* cache, con
   if (need > kStaticScratchBytes) return ZHA_ERR_WORKSPACE;  // geometry beyond the static size
   void* ws = nullptr;
   if ((st = static_scratch(&ws)) != ZHA_OK) return st;
-  // Nothing in the decode workspace has to start at zero: the traversal writes
-  // every candidate, score, keep-bit word, kept-list entry and counter before
-  // it is read, so no clearing pass is needed between calls.
-  return zha_decode(cfg, cache, q, p, out, level_counts, ws, kStaticScratchBytes, dev_status,
-                    stream);
+  // Nothing in the decode workspace has to start at zero: the selection writes
+  // every score, kept-list entry, bitmap word and counter before it is read,
+  // so no clearing pass is needed between calls. Every launch stays on the
+  // caller's stream: this entry point creates no streams or events either.
+  return zha::decode_one_stream(cfg, cache, q, p, out, level_counts, ws, kStaticScratchBytes,
+                                dev_status, stream);
 }
 
 }  // extern "C"

@@ -84,11 +84,13 @@ size_t decode_dense_ws_bytes(const Geometry& g, int64_t units);
 // Decode mode only (query of sequence s at seq_len[s] - 1): writes the kept
 // level-1 union with per-head masks in `segs` ordered segments per unit, the
 // per-head level counts (nullable) and the rows scored per level (stats).
+// Units [unit0, unit0 + n_units) only when n_units > 0.
 cudaError_t launch_decode_dense(const Geometry& g, const void* tree, const void* q,
                                 const int32_t* seq_len, uint64_t p_q, void* ws,
                                 int32_t* level_counts, int32_t* stats, uint32_t* kept,
                                 int32_t* n_kept, int64_t kept_stride, int segs, int32_t* status,
-                                int num_sms, cudaStream_t stream);
+                                int num_sms, cudaStream_t stream, int64_t unit0 = 0,
+                                int64_t n_units = 0);
 
 // ---- prefill top level on the tensor cores ----------------------------------
 // Top nodes per (sequence, KV head): ncap / b^L.
@@ -128,6 +130,10 @@ struct AttendArgs {
   const int32_t* idx;
   int64_t idx_cap;
   const int32_t* n_idx;
+  // units [unit0, unit0 + n_units) only (n_units 0: all); the split count
+  // stays that of the whole launch, so a range's outputs equal the whole's
+  int64_t unit0;
+  int64_t n_units;
 };
 
 size_t attend_ws_bytes(const Geometry& g, int kind, int64_t nq, int num_sms);
@@ -157,5 +163,11 @@ cudaError_t launch_kept_lists(const Geometry& g, const uint32_t* kept, const int
                               cudaStream_t stream);
 
 int device_sm_count();
+
+// zha_decode with every launch on the caller's stream (no streams or events of
+// the library's own); the same outputs as zha_decode.
+zha_status decode_one_stream(const zha_config* cfg, const zha_cache* cache, const void* q,
+                             double p, void* out, int32_t* level_counts, void* ws,
+                             size_t ws_bytes, int32_t* dev_status, void* stream);
 
 }  // namespace zha
