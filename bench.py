@@ -594,14 +594,8 @@ def run_zha(args, rank, world, dev):
     stream = torch.cuda.current_stream()
 
     # ---- tree build (rate reported; not part of a decode step) ----
-    z.zha_build_tree(cfg, cache)
-    torch.cuda.synchronize()
+    build_ms = time_tree_build(cfg, cache, stream)
     e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
-    e0.record()
-    z.zha_build_tree(cfg, cache)
-    e1.record()
-    torch.cuda.synchronize()
-    build_ms = e0.elapsed_time(e1)
     n_tok = B * Hkv * c.n_tokens
     build_bytes, build_flops = tree_build_work(c.n_tokens, b, L, D, B * Hkv)
 
@@ -843,13 +837,7 @@ def run_prefill(args, rank, world, dev):
     e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
 
     # ---- tree over the cached context (rate reported; not part of a step) ----
-    z.zha_build_tree(cfg, cache)
-    torch.cuda.synchronize()
-    e0.record(stream)
-    z.zha_build_tree(cfg, cache)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    build_ms = e0.elapsed_time(e1)
+    build_ms = time_tree_build(cfg, cache, stream)
 
     def one_step():
         cache.seq_len = len1

@@ -146,8 +146,9 @@ __device__ void node_small_b(const TreeParams& p, const float* Rt, float* abuf, 
 // ---------------------------------------------------------------------------
 // Level kernel for b <= 32: a CTA takes tiles of kTileRows consecutive child
 // rows (kTileRows / b whole nodes) of one unit. The rows are staged in shared
-// memory by cp.async, double-buffered so that the next tile's rows stream in
-// while the current one is reduced, in four phases:
+// memory by cp.async in one stage (49 KB of shared memory per CTA, so four
+// CTAs share an SM and overlap one another's loads), then reduced in four
+// phases:
 //   1. logits: thread (cg, rg) runs the 16 canonical chains of children
 //      4cg..4cg+3 against reference queries 4rg..4rg+3 -- every staged x
 //      chunk feeds 4 reference queries and every R value 4 children;
@@ -168,7 +169,7 @@ struct TileCfg {
   static constexpr int kStageBytes = kTileRows * D * (int)sizeof(T);
   static constexpr int kRtBytes = kNRef * D * 4;
   static constexpr int kWBytes = kTileRows * kNRef * 4;
-  static constexpr int kSmem = 2 * kStageBytes + kRtBytes + kWBytes + kTileRows * 4;
+  static constexpr int kSmem = kStageBytes + kRtBytes + kWBytes + kTileRows * 4;
 };
 
 // Chunk ch of staged row r sits at chunk ch ^ ((r >> 2) & 7): the 8 rows one
@@ -192,8 +193,8 @@ __global__ void __launch_bounds__(kTileThreads) tree_level_tiled(const __grid_co
   using C = TileCfg<T, D>;
   constexpr int kPer = C::kPer, kNch = C::kNch;
   extern __shared__ __align__(16) float sm[];
-  unsigned char* X0 = reinterpret_cast<unsigned char*>(sm);  // two stages of staged rows
-  float* Rt = reinterpret_cast<float*>(X0 + 2 * C::kStageBytes);  // [D][16]
+  unsigned char* X = reinterpret_cast<unsigned char*>(sm);  // the tile's staged rows
+  float* Rt = reinterpret_cast<float*>(X + C::kStageBytes);  // [D][16]
   float* W = Rt + kNRef * D;                                // [tile rows][16]
   float* A = W + kTileRows * kNRef;                         // [tile rows]
   const int tid = threadIdx.x;
@@ -214,25 +215,12 @@ __global__ void __launch_bounds__(kTileThreads) tree_level_tiled(const __grid_co
   const int rg = tid & 3, cg = tid >> 2;  // phase-1 block: 4 children x 4 reference queries
   const float inv_sqrt_d = p.inv_sqrt_d;
 
-  int64_t tile = blockIdx.x;
-  {
+  for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
     const int64_t r0 = tile * kTileRows;
     const int rows = (int)(rows_total - r0 < kTileRows ? rows_total - r0 : kTileRows);
-    stage_tile<T, D>(cb + r0 * D, rows, X0);
-  }
-  cp_async_commit();
-  for (int it = 0; tile < n_tiles; ++it, tile += gridDim.x) {
-    unsigned char* X = X0 + (it & 1) * C::kStageBytes;
-    const int64_t r0 = tile * kTileRows;
-    const int rows = (int)(rows_total - r0 < kTileRows ? rows_total - r0 : kTileRows);
-    const int64_t next = tile + gridDim.x;
-    if (next < n_tiles) {  // the other stage was last read before the previous iteration's end
-      const int64_t n0 = next * kTileRows;
-      const int nrows = (int)(rows_total - n0 < kTileRows ? rows_total - n0 : kTileRows);
-      stage_tile<T, D>(cb + n0 * D, nrows, X0 + ((it + 1) & 1) * C::kStageBytes);
-    }
+    stage_tile<T, D>(cb + r0 * D, rows, X);
     cp_async_commit();
-    cp_async_wait<1>();  // this tile's rows have landed (this thread's copies)
+    cp_async_wait<0>();  // this thread's copies have landed
     __syncthreads();     // ... and every thread's
     // ---- 1. logits of children 4cg..4cg+3 against queries 4rg..4rg+3 ----
     {
@@ -305,9 +293,8 @@ __global__ void __launch_bounds__(kTileThreads) tree_level_tiled(const __grid_co
       }
       *reinterpret_cast<uint4*>(ob + (r0 / b + n) * D + ch * kPer) = Elem<T>::pack(s);
     }
-    __syncthreads();  // this stage is refilled two iterations on
+    __syncthreads();  // the stage is refilled by the next tile
   }
-  cp_async_wait<0>();
 }
 
 // One CTA per unit walks every level; for small growth (decode steps).
@@ -431,9 +418,12 @@ cudaError_t launch_tree_t(const Geometry& g, const TreeParams& p, int64_t max_ne
       e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tree_level_tiled<T, D>,
                                                         kTileThreads, C::kSmem);
       if (e != cudaSuccess) return e;
-      // enough CTAs for one full wave over all units, each looping over tiles
+      // at most one wave (a partial second wave would run a whole CTA's share
+      // of tiles after the first): the resident slots shared evenly by the
+      // units, each CTA looping over its unit's tiles
       const int64_t tiles = (nodes * g.b + kTileRows - 1) / kTileRows;
-      int64_t per_unit = ((int64_t)device_sm_count() * (per_sm > 0 ? per_sm : 1) + units - 1) / units;
+      int64_t per_unit = ((int64_t)device_sm_count() * (per_sm > 0 ? per_sm : 1)) / units;
+      if (per_unit < 1) per_unit = 1;
       if (per_unit > tiles) per_unit = tiles;
       dim3 grid((unsigned)per_unit, (unsigned)units);
       tree_level_tiled<T, D><<<grid, kTileThreads, C::kSmem, stream>>>(p, level);
