@@ -98,6 +98,8 @@ def lib():
                                     ctypes.c_int64, ctypes.c_double, _i32p, ctypes.c_int64, _i32p,
                                     _f64p]
         L.zo_select_f64.restype = ctypes.c_int64
+        L.zo_fp4_round_rows.argtypes = [_f32p, ctypes.c_int64, ctypes.c_int, _f32p, _i32p]
+        L.zo_fp4_round_rows.restype = None
         L.zo_attend_f64.argtypes = [_f32p, ctypes.c_int, _f32p, _f32p, _i32p, ctypes.c_int64,
                                     _f64p]
         L.zo_attend_f64.restype = None
@@ -258,6 +260,23 @@ def select_f64(q, tree: Tree, t: int, p: float):
 # ---------------------------------------------------------------------------
 # attention
 # ---------------------------------------------------------------------------
+
+def fp4_round_rows(rows) -> Tuple[np.ndarray, np.ndarray]:
+    """Block-scaled 4-bit rounding of [n][d] rows (zo_fp4_round_rows): the
+    rounded fp32 values and the per-32-element exponents [n][d / 32]."""
+    x = np.ascontiguousarray(rows, dtype=np.float32)
+    n, d = x.shape
+    assert d % 32 == 0
+    out = np.empty_like(x)
+    exps = np.empty((n, d // 32), dtype=np.int32)
+    lib().zo_fp4_round_rows(_ptr(x, _f32p), n, d, _ptr(out, _f32p), _ptr(exps, _i32p))
+    return out, exps
+
+
+def fp4_tree(tree: "Tree") -> "Tree":
+    """The tree with every stored summary row rounded by fp4_round_rows."""
+    return Tree(fp4_round_rows(tree.rows)[0], tree.offs, tree.b, tree.L, tree.d)
+
 
 def attend(q, K, V, idx) -> np.ndarray:
     """fp64 softmax attention of q over rows idx of (K, V)."""

@@ -535,3 +535,47 @@ int64_t zo_select_f64(const float* q, int d, const float* tree, const int64_t* l
   free(c);
   return n_sel;
 }
+
+/* ------------------------------------------------------------------------ */
+/* block-scaled 4-bit summary rows (the FP4 router variant)                  */
+/* ------------------------------------------------------------------------ */
+
+/* [lefilia] par. 4 reports that a 4-bit (FP4) variant of the router was
+ * tried; the pages give no format. This library's reading: every block of 32
+ * consecutive elements of a summary row is stored as e2m1 magnitudes
+ * {0, 0.5, 1, 1.5, 2, 3, 4, 6} (codes 0..7 in that order) with a sign, times
+ * one power of two 2^e per block, e the smallest integer with
+ * max|x| <= 6 * 2^e (e = 0 for an all-zero block). Each |x| / 2^e goes to the
+ * nearest magnitude, an exact tie to the even code. The rounded values are
+ * written to out (zero as +0) and e to exps[row * d/32 + block]. The router
+ * then scores these values with the canonical arithmetic. */
+void zo_fp4_round_rows(const float* in, int64_t n_rows, int d, float* out, int32_t* exps) {
+  static const float mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+  static const float mid[7] = {0.25f, 0.75f, 1.25f, 1.75f, 2.5f, 3.5f, 5.0f};
+  const int nb = d / 32;
+  for (int64_t r = 0; r < n_rows; ++r)
+    for (int blk = 0; blk < nb; ++blk) {
+      const float* x = in + r * d + blk * 32;
+      float* y = out + r * d + blk * 32;
+      float amax = 0.0f;
+      for (int i = 0; i < 32; ++i)
+        if (fabsf(x[i]) > amax) amax = fabsf(x[i]);
+      int e = 0;
+      if (amax > 0.0f) {
+        /* amax = m 2^E with m in [0.5, 1); 6 2^e = 0.75 2^(e+3) */
+        int E = 0;
+        const float m = frexpf(amax, &E);
+        e = m <= 0.75f ? E - 3 : E - 2;
+      }
+      exps[r * nb + blk] = e;
+      for (int i = 0; i < 32; ++i) {
+        const float a = ldexpf(fabsf(x[i]), -e); /* exact: a power-of-two scaling */
+        int k = 0;
+        while (k < 7 && a > mid[k]) ++k;
+        if (k < 7 && a == mid[k] && (k & 1)) ++k;
+        const float v = ldexpf(mag[k], e);
+        y[i] = k == 0 ? 0.0f : (x[i] < 0.0f ? -v : v);
+      }
+    }
+}
+
