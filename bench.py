@@ -454,9 +454,7 @@ def workload_config(args, c):
     return {"workload": args.workload, "batch": c.batch, "context": c.n_tokens,
             "heads": f"{c.n_q_heads}q/{c.n_kv_heads}kv", "head_dim": c.head_dim,
             "tree": f"b={c.block},L={c.levels}", "p": c.p,
-            "queries_per_step": c.batch * c.n_q_heads, "l2": l2_note(kv_gb),
-            "step": "CUDA graph of zha_extend_tree + zha_decode, replayed after the step's "
-                    "lengths and queries are copied into its input buffers"}
+            "queries_per_step": c.batch * c.n_q_heads, "l2": l2_note(kv_gb)}
 
 
 def tree_build_work(n_tokens: int, b: int, L: int, D: int, units: int, elem: int = 2):
@@ -518,6 +516,90 @@ def tree_builds_other_workloads(dev, peak_gbs: float) -> dict:
         del wl, cache
         torch.cuda.empty_cache()
     return out
+
+
+def fp4_router_leg(z, cfg, cache, c, ws, st, queries, peak: float, steps: int = 20,
+                   warmup: int = 3) -> dict:
+    """The FP4 router variant on the headline cache as it stands (tree and
+    lengths of the last timed step): the 4-bit copy's quantization time, then
+    zha_decode_fp4 against zha_decode on the same queries (eager, no extend),
+    the bytes each touches, and the drift of the variant's attended sets from
+    the canonical ones (recall of the canonical set, size ratio), per
+    (sequence, query head) of the last query set."""
+    dev = queries.device
+    B, Hq, Hkv, D, b, L = c.batch, c.n_q_heads, c.n_kv_heads, c.head_dim, c.block, c.levels
+    fp4 = z.alloc_fp4_tree(cfg, dev)
+    z.zha_fp4_quantize_tree(cfg, cache, fp4)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+    e0.record()
+    z.zha_fp4_quantize_tree(cfg, cache, fp4)
+    e1.record()
+    torch.cuda.synchronize()
+    quant_ms = e0.elapsed_time(e1)
+    out = torch.empty_like(queries[0])
+    n_q = queries.shape[0]
+
+    def timed(fn):
+        for i in range(warmup):
+            fn(queries[i % n_q])
+        torch.cuda.synchronize()
+        e0.record()
+        for i in range(steps):
+            fn(queries[i % n_q])
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    canon_ms = timed(lambda q: z.zha_decode(cfg, cache, q, c.p, out, None, ws, st))
+    fp4_ms = timed(lambda q: z.zha_decode_fp4(cfg, cache, fp4, q, c.p, out, None, ws, st))
+    n = int(cache.seq_len.max().item())
+    tail = n - b ** L * (n // b ** L)
+    row = D * 2
+    lists = {}
+    bytes_ = {}
+    for name, fn in (("canonical", lambda q: z.zha_decode(cfg, cache, q, c.p, out, None, ws, st)),
+                     ("fp4", lambda q: z.zha_decode_fp4(cfg, cache, fp4, q, c.p, out, None, ws,
+                                                        st))):
+        fn(queries[(steps - 1) % n_q])
+        stats = torch.zeros(B * Hkv, L + 1, dtype=torch.int32, device=dev)
+        z.zha_decode_stats(cfg, ws, stats)
+        idx = torch.empty(B, Hq, n + 2, dtype=torch.int32, device=dev)
+        n_idx = torch.zeros(B, Hq, dtype=torch.int32, device=dev)
+        z.zha_decode_kept_lists(cfg, cache, ws, idx, n_idx, st)
+        torch.cuda.synchronize()
+        stats = stats.cpu()
+        cand, kept = int(stats[:, :L].sum()), int(stats[:, L].sum())
+        srow = row if name == "canonical" else D // 2 + 2 * (D // 32)
+        sel, att, _ = decode_step_bytes(cand, kept, b, tail, B * Hkv, B * Hq, row)
+        sel += cand * (srow - row)
+        bytes_[name] = (sel, att)
+        lists[name] = (idx, n_idx.cpu())
+    if int(st.item()) != 0:
+        raise RuntimeError(f"fp4 leg: device status {z.status_string(int(st.item()))}")
+    recall, ratio = [], []
+    (ci, cn), (fi, fn_) = lists["canonical"], lists["fp4"]
+    for s in range(B):
+        for h in range(Hq):
+            a = ci[s, h, :int(cn[s, h])]
+            f = fi[s, h, :int(fn_[s, h])]
+            recall.append(torch.isin(a, f).sum().item() / a.numel())
+            ratio.append(f.numel() / a.numel())
+    sel4, att4 = bytes_["fp4"]
+    selc, attc = bytes_["canonical"]
+    return {
+        "format": "e2m1 codes, one int16 power-of-two exponent per 32 elements (72 B per "
+                  "d=128 row instead of 256 B)",
+        "quantize_ms": quant_ms,
+        "decode_ms": {"fp4": fp4_ms, "canonical": canon_ms},
+        "queries_per_s": {"fp4": B * Hq / (fp4_ms / 1e3), "canonical": B * Hq / (canon_ms / 1e3)},
+        "select_bytes_per_step": {"fp4": sel4, "canonical": selc},
+        "bytes_per_step": {"fp4": sel4 + att4, "canonical": selc + attc},
+        "hbm_frac": {"fp4": (sel4 + att4) / (fp4_ms / 1e3) / 1e9 / peak,
+                     "canonical": (selc + attc) / (canon_ms / 1e3) / 1e9 / peak},
+        "recall_of_canonical_set": {"mean": sum(recall) / len(recall), "min": min(recall)},
+        "set_size_ratio_mean": sum(ratio) / len(ratio),
+    }
 
 
 def wide_p_sweep(dev, peak: float, steps: int = 20, warmup: int = 3) -> list:
@@ -781,6 +863,8 @@ def run_zha(args, rank, world, dev):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded Gaussian-mixture keys, planted needles; no dataset)",
         "config": workload_config(args, c),
+        "timed_step": "a CUDA graph of zha_extend_tree + zha_decode, replayed after the "
+                      "step's lengths and queries are copied into its input buffers",
         "hbm_frac": hbm_frac,
         "hbm_frac_of_nominal_8tbs": step_bytes / (ms_step / 1e3) / 8e12,
         "bytes_touched_per_step": step_bytes,
@@ -805,6 +889,7 @@ def run_zha(args, rank, world, dev):
         "gpu_launches": (1 + 5 * min(4, max(1, B * Hkv // 2))) * args.steps,
         "clocks": clocks,
     }
+    res["fp4_router"] = fp4_router_leg(z, cfg, cache, c, ws, st, queries, peak)
     if args.n_tokens is None:  # the other workloads at their full sizes
         res["decode_wide_p_sweep"] = wide_p_sweep(dev, peak)
         res["tree_build_other_workloads"] = tree_builds_other_workloads(dev, peak)

@@ -275,6 +275,48 @@ zha_status zha_decode_kept_lists(const zha_config* cfg, const zha_cache* cache, 
                                  size_t ws_bytes, int32_t* idx, int64_t idx_cap, int32_t* n_idx,
                                  int32_t* dev_status, void* stream);
 
+/* ---- FP4 router variant (lefilia.fr page, par. 4: a 4-bit variant of the
+ * router was tried; the page gives no format) ----------------------------
+ * A block-scaled 4-bit copy of the summary tree, scored in place of the
+ * tree's rows by the decode selection; everything else of the step (cut,
+ * union, attention over the raw K/V) is unchanged. Format: every block of
+ * 32 consecutive elements of a stored summary row becomes 4-bit codes --
+ * bit 3 the sign, bits 0-2 the index k of the magnitude in
+ * {0, 0.5, 1, 1.5, 2, 3, 4, 6} (the e2m1 encoding) -- and one exponent e:
+ * value = sign * mag[k] * 2^e, with e the smallest integer such that the
+ * block's largest magnitude is at most 6 * 2^e (0 for an all-zero block),
+ * each |x| / 2^e rounded to the nearest magnitude, an exact tie to the even
+ * k, zeros stored with sign 0. A 256-byte bf16 row (d = 128) becomes 64
+ * bytes of codes and 8 bytes of exponents. The selection this gives is a
+ * labelled variant of the canonical one (it scores rounded summaries);
+ * scoring itself is the canonical fp32 chain over the exact 4-bit values.
+ * Layout of the copy: the code of tree element i (element order and
+ * level_off as zha_tree_layout) in byte i/2, the low nibble for even i; the
+ * int16 exponent of block i/32 at byte codes_bytes + 2*(i/32), codes_bytes =
+ * tree_elems/2 rounded up to a multiple of 256. */
+
+/* Bytes of the FP4 copy of a tree of this configuration. */
+zha_status zha_fp4_tree_bytes(const zha_config* cfg, size_t* bytes);
+
+/* Writes the FP4 copy (device buffer of zha_fp4_tree_bytes) of the rows of
+ * every node complete at seq_len, or, with old_len (device int32 [B],
+ * nullable), of the nodes completed in (old_len[b], seq_len[b]] -- call it
+ * after zha_build_tree / zha_extend_tree with the same old_len. The tree
+ * itself is read only. Asynchronous on stream. */
+zha_status zha_fp4_quantize_tree(const zha_config* cfg, const zha_cache* cache, void* fp4_tree,
+                                 const int32_t* old_len, void* stream);
+
+/* zha_decode with the selection scored on the FP4 copy fp4_tree (kept up to
+ * date with zha_fp4_quantize_tree): same arguments, workspace
+ * (ZHA_OP_DECODE), streams, outputs and errors as zha_decode, plus
+ * ZHA_ERR_UNSUPPORTED unless head_dim is 128 and the step takes the dense
+ * decode selection (the tree prefix under the complete top nodes is at
+ * most 1.5 GB and a head's cut state fits shared memory). zha_decode_stats
+ * and zha_decode_kept_lists read its workspace as after zha_decode. */
+zha_status zha_decode_fp4(const zha_config* cfg, const zha_cache* cache, const void* fp4_tree,
+                          const void* q, double p, void* out, int32_t* level_counts, void* ws,
+                          size_t ws_bytes, int32_t* dev_status, void* stream);
+
 /* zha_decode without a caller workspace. The pages describe no counterpart of
  * this call; it exists for callers that cannot hand the library a workspace --
  * plugins loaded by a host that owns the device allocator and exposes none of

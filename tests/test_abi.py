@@ -28,7 +28,7 @@ def z():
 
 def test_exports_every_declared_symbol(z):
     names = _declared_functions()
-    assert len(names) == 16, names
+    assert len(names) == 19, names
     lib = z.lib()
     for n in names:
         assert hasattr(lib, n), n
@@ -93,6 +93,27 @@ def test_bad_arguments_rejected_before_launch(z):
     assert L.zha_dense_decode(ctypes.byref(cfg), ctypes.byref(c), ctypes.c_void_p(16),
                               ctypes.c_void_p(16), ctypes.c_void_p(16), 1, None) == \
         z.ZHA_ERR_WORKSPACE
+
+
+def test_fp4_router_host_side(z):
+    cfg = z.make_config(128, 4, 6, 16, 2, 8, 262400, torch.bfloat16)
+    nbytes, _ = z.zha_tree_layout(cfg)
+    elems = nbytes // 2
+    # 4-bit codes (rounded up to 256 bytes), then one int16 exponent per 32 elements
+    assert z.zha_fp4_tree_bytes(cfg) == (elems // 2 + 255) // 256 * 256 + 2 * (elems // 32)
+    L = z.lib()
+    c = z.zha_cache(16, 16, 16, 16, 16)  # non-null dummies: never dereferenced here
+    ws_need = z.zha_workspace_bytes(cfg, z.ZHA_OP_DECODE)
+    args = (ctypes.c_void_p(16), 0.95, ctypes.c_void_p(16), None, ctypes.c_void_p(16), ws_need,
+            None, None)
+    # no FP4 copy, and head_dim 64 (the 4-bit scoring is written for 128)
+    assert L.zha_decode_fp4(ctypes.byref(cfg), ctypes.byref(c), None, *args) == \
+        z.ZHA_ERR_INVALID_ARG
+    cfg64 = z.make_config(64, 4, 6, 16, 2, 8, 262400, torch.bfloat16)
+    assert L.zha_decode_fp4(ctypes.byref(cfg64), ctypes.byref(c), ctypes.c_void_p(16), *args) == \
+        z.ZHA_ERR_UNSUPPORTED
+    assert L.zha_fp4_quantize_tree(ctypes.byref(cfg), ctypes.byref(c), None, None, None) == \
+        z.ZHA_ERR_INVALID_ARG
 
 
 def test_prefill_top_scores_rejected_before_launch(z):

@@ -43,6 +43,7 @@ EXPORTS = (
     "zha_extend_tree", "zha_select", "zha_attend", "zha_decode", "zha_decode_select",
     "zha_decode_attend", "zha_decode_stats", "zha_prefill_chunk", "zha_dense_decode",
     "zha_decode_noalloc", "zha_prefill_top_scores", "zha_decode_kept_lists",
+    "zha_fp4_tree_bytes", "zha_fp4_quantize_tree", "zha_decode_fp4",
 )
 
 
@@ -108,6 +109,9 @@ def lib() -> ctypes.CDLL:
             "zha_dense_decode": ([c_cfg, c_cache, vp, vp, vp, sz, vp], i32),
             "zha_decode_noalloc": ([c_cfg, c_cache, vp, d, vp, vp, vp, vp], i32),
             "zha_decode_kept_lists": ([c_cfg, c_cache, vp, sz, vp, i64, vp, vp, vp], i32),
+            "zha_fp4_tree_bytes": ([c_cfg, P(sz)], i32),
+            "zha_fp4_quantize_tree": ([c_cfg, c_cache, vp, vp, vp], i32),
+            "zha_decode_fp4": ([c_cfg, c_cache, vp, vp, d, vp, vp, vp, sz, vp, vp], i32),
             "zha_prefill_top_scores": ([c_cfg, c_cache, vp, i32, i64, i64, d, vp, vp, vp, sz, vp,
                                         vp], i32),
         }
@@ -200,6 +204,16 @@ def alloc_tree(cfg: zha_config, device="cuda") -> torch.Tensor:
     return torch.zeros(max(nbytes // dt.itemsize, 1), dtype=dt, device=device)
 
 
+def zha_fp4_tree_bytes(cfg: zha_config) -> int:
+    n = ctypes.c_size_t(0)
+    _check("zha_fp4_tree_bytes", lib().zha_fp4_tree_bytes(ctypes.byref(cfg), ctypes.byref(n)))
+    return n.value
+
+
+def alloc_fp4_tree(cfg: zha_config, device="cuda") -> torch.Tensor:
+    return torch.zeros(zha_fp4_tree_bytes(cfg), dtype=torch.uint8, device=device)
+
+
 def alloc_workspace(cfg: zha_config, op: int, max_queries: int = 0, device="cuda") -> torch.Tensor:
     return torch.empty(zha_workspace_bytes(cfg, op, max_queries), dtype=torch.uint8, device=device)
 
@@ -251,6 +265,22 @@ def zha_decode(cfg: zha_config, cache: Cache, q: torch.Tensor, p: float, out: to
     _check("zha_decode", lib().zha_decode(
         ctypes.byref(cfg), ctypes.byref(c), _ptr(q), float(p), _ptr(out), _ptr(level_counts),
         _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream)))
+
+
+def zha_fp4_quantize_tree(cfg: zha_config, cache: Cache, fp4_tree: torch.Tensor,
+                          old_len: Optional[torch.Tensor] = None, stream=None):
+    c = cache.c()
+    _check("zha_fp4_quantize_tree", lib().zha_fp4_quantize_tree(
+        ctypes.byref(cfg), ctypes.byref(c), _ptr(fp4_tree), _ptr(old_len), _stream(stream)))
+
+
+def zha_decode_fp4(cfg: zha_config, cache: Cache, fp4_tree: torch.Tensor, q: torch.Tensor,
+                   p: float, out: torch.Tensor, level_counts: Optional[torch.Tensor],
+                   ws: torch.Tensor, dev_status: Optional[torch.Tensor] = None, stream=None):
+    c = cache.c()
+    _check("zha_decode_fp4", lib().zha_decode_fp4(
+        ctypes.byref(cfg), ctypes.byref(c), _ptr(fp4_tree), _ptr(q), float(p), _ptr(out),
+        _ptr(level_counts), _ptr(ws), ws.numel(), _ptr(dev_status), _stream(stream)))
 
 
 def zha_decode_select(cfg: zha_config, cache: Cache, q: torch.Tensor, p: float,
@@ -329,5 +359,6 @@ def zha_decode_noalloc(cfg: zha_config, cache: Cache, q: torch.Tensor, p: float,
 
 
 __all__ = [n for n in globals() if n.startswith("zha_")] + [
-    "lib", "Cache", "make_config", "alloc_tree", "alloc_workspace", "ZhaError", "EXPORTS",
+    "lib", "Cache", "make_config", "alloc_tree", "alloc_fp4_tree", "alloc_workspace", "ZhaError",
+    "EXPORTS",
 ]

@@ -323,13 +323,15 @@ static zha_status run_tree_select(const Geometry& g, const zha_cache* cache, con
                                   const int32_t* q_seq, const int32_t* q_pos, int64_t nq,
                                   uint64_t p_q, int32_t* level_counts, unsigned char* ws,
                                   const DecodeLayout& L, int32_t* dev_status, int sms,
-                                  cudaStream_t s, const TopSeeds* seeds = nullptr) {
+                                  cudaStream_t s, const TopSeeds* seeds = nullptr,
+                                  const void* fp4 = nullptr) {
   if (L.dense && !q_pos && !seeds)
     return cuda_status(launch_decode_dense(
         g, cache->tree, q, cache->seq_len, p_q, ws + L.trav, level_counts,
         reinterpret_cast<int32_t*>(ws + L.stats), reinterpret_cast<uint32_t*>(ws + L.kept),
         reinterpret_cast<int32_t*>(ws + L.n_kept), traverse_kept_stride(g),
-        traverse_cluster_size(g, L.units, sms), dev_status, sms, s));
+        traverse_cluster_size(g, L.units, sms), dev_status, sms, s, 0, 0, fp4));
+  if (fp4) return ZHA_ERR_UNSUPPORTED;  // the FP4 rows are read by the dense decode path only
   TraverseOut to{};
   to.kept = reinterpret_cast<uint32_t*>(ws + L.kept);
   to.n_kept = reinterpret_cast<int32_t*>(ws + L.n_kept);
@@ -364,9 +366,10 @@ static zha_status run_tree_decode(const Geometry& g, const zha_cache* cache, con
                                   const int32_t* q_seq, const int32_t* q_pos, int64_t nq,
                                   uint64_t p_q, void* out, int32_t* level_counts,
                                   unsigned char* ws, const DecodeLayout& L, int32_t* dev_status,
-                                  int sms, cudaStream_t s, const TopSeeds* seeds = nullptr) {
+                                  int sms, cudaStream_t s, const TopSeeds* seeds = nullptr,
+                                  const void* fp4 = nullptr) {
   zha_status st = run_tree_select(g, cache, q, q_seq, q_pos, nq, p_q, level_counts, ws, L,
-                                  dev_status, sms, s, seeds);
+                                  dev_status, sms, s, seeds, fp4);
   if (st != ZHA_OK) return st;
   return run_tree_attend(g, cache, q, q_seq, q_pos, nq, out, ws, L, sms, s);
 }
@@ -431,7 +434,7 @@ static zha_status run_dense_decode_grouped(const Geometry& g, const zha_cache* c
                                            const void* q, uint64_t p_q, void* out,
                                            int32_t* level_counts, unsigned char* ws,
                                            const DecodeLayout& L, int32_t* dev_status, int sms,
-                                           cudaStream_t s, int K, DecodePipe& P) {
+                                           cudaStream_t s, int K, DecodePipe& P, const void* fp4) {
   AttendArgs a{};
   a.kind = kStreamTree;
   a.k = cache->k;
@@ -456,7 +459,7 @@ static zha_status run_dense_decode_grouped(const Geometry& g, const zha_cache* c
                               reinterpret_cast<int32_t*>(ws + L.stats),
                               reinterpret_cast<uint32_t*>(ws + L.kept),
                               reinterpret_cast<int32_t*>(ws + L.n_kept), a.kept_stride,
-                              a.kept_segs, dev_status, sms, sk, u0, u1 - u0);
+                              a.kept_segs, dev_status, sms, sk, u0, u1 - u0, fp4);
     if (err != cudaSuccess) break;
     a.unit0 = u0;
     a.n_units = u1 - u0;
@@ -476,16 +479,17 @@ static zha_status run_dense_decode_grouped(const Geometry& g, const zha_cache* c
 static zha_status run_decode_step(const Geometry& g, const zha_cache* cache, const void* q,
                                   uint64_t p_q, void* out, int32_t* level_counts,
                                   unsigned char* ws, const DecodeLayout& L, int32_t* dev_status,
-                                  int sms, cudaStream_t s, bool concurrent) {
+                                  int sms, cudaStream_t s, bool concurrent,
+                                  const void* fp4 = nullptr) {
   const int K = concurrent ? L.groups : 1;
   if (K > 1) {
     std::lock_guard<std::mutex> lock(g_pipe_mutex);
     DecodePipe* P = decode_pipe(s);
     if (P) return run_dense_decode_grouped(g, cache, q, p_q, out, level_counts, ws, L, dev_status,
-                                           sms, s, K, *P);
+                                           sms, s, K, *P, fp4);
   }
   return run_tree_decode(g, cache, q, nullptr, nullptr, g.B, p_q, out, level_counts, ws, L,
-                         dev_status, sms, s);
+                         dev_status, sms, s, nullptr, fp4);
 }
 
 __global__ void decode_stats_kernel(const int32_t* stats, const int32_t* n_kept, int units, int L,
@@ -500,7 +504,8 @@ __global__ void decode_stats_kernel(const int32_t* stats, const int32_t* n_kept,
 
 static zha_status decode_impl(const zha_config* cfg, const zha_cache* cache, const void* q,
                               double p, void* out, int32_t* level_counts, void* ws,
-                              size_t ws_bytes, int32_t* dev_status, void* stream, bool concurrent) {
+                              size_t ws_bytes, int32_t* dev_status, void* stream, bool concurrent,
+                              const void* fp4 = nullptr) {
   Geometry g;
   zha_status st = make_geometry(cfg, &g);
   if (st != ZHA_OK) return st;
@@ -509,15 +514,43 @@ static zha_status decode_impl(const zha_config* cfg, const zha_cache* cache, con
   if (!q || !out || !ws || !check_p(p, &p_q)) return ZHA_ERR_INVALID_ARG;
   const int sms = device_sm_count();
   const DecodeLayout L = decode_layout(g, g.B, kStreamTree, sms, true);
+  if (fp4 && (!L.dense || g.d != 128)) return ZHA_ERR_UNSUPPORTED;
   if (ws_bytes < L.total) return ZHA_ERR_WORKSPACE;
   return run_decode_step(g, cache, q, p_q, out, level_counts, static_cast<unsigned char*>(ws), L,
-                         dev_status, sms, (cudaStream_t)stream, concurrent);
+                         dev_status, sms, (cudaStream_t)stream, concurrent, fp4);
 }
 
 zha_status zha_decode(const zha_config* cfg, const zha_cache* cache, const void* q, double p,
                       void* out, int32_t* level_counts, void* ws, size_t ws_bytes,
                       int32_t* dev_status, void* stream) {
   return decode_impl(cfg, cache, q, p, out, level_counts, ws, ws_bytes, dev_status, stream, true);
+}
+
+zha_status zha_fp4_tree_bytes(const zha_config* cfg, size_t* bytes) {
+  Geometry g;
+  zha_status st = make_geometry(cfg, &g);
+  if (st != ZHA_OK) return st;
+  if (!bytes) return ZHA_ERR_INVALID_ARG;
+  *bytes = fp4_tree_bytes(g);
+  return ZHA_OK;
+}
+
+zha_status zha_fp4_quantize_tree(const zha_config* cfg, const zha_cache* cache, void* fp4_tree,
+                                 const int32_t* old_len, void* stream) {
+  Geometry g;
+  zha_status st = make_geometry(cfg, &g);
+  if (st != ZHA_OK) return st;
+  if (!cache || !cache->tree || !cache->seq_len || !fp4_tree) return ZHA_ERR_INVALID_ARG;
+  return cuda_status(launch_fp4_quantize(g, cache->tree, fp4_tree, cache->seq_len, old_len,
+                                         device_sm_count(), (cudaStream_t)stream));
+}
+
+zha_status zha_decode_fp4(const zha_config* cfg, const zha_cache* cache, const void* fp4_tree,
+                          const void* q, double p, void* out, int32_t* level_counts, void* ws,
+                          size_t ws_bytes, int32_t* dev_status, void* stream) {
+  if (!fp4_tree) return ZHA_ERR_INVALID_ARG;
+  return decode_impl(cfg, cache, q, p, out, level_counts, ws, ws_bytes, dev_status, stream, true,
+                     fp4_tree);
 }
 
 zha_status zha_decode_select(const zha_config* cfg, const zha_cache* cache, const void* q,

@@ -29,6 +29,7 @@
 // the reads on the cuts. The host uses this path when that prefix is small
 // enough (decode_dense_ok) and the frontier traversal otherwise.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "zha_device.cuh"
@@ -72,6 +73,10 @@ struct DenseParams {
   int64_t kept_stride;
   int segs;
   int unit0;               // first unit of this launch (grid y: its units)
+  // FP4 router variant (nullable): block-scaled 4-bit summary rows scored in
+  // place of the tree's rows (d = 128)
+  const unsigned char* fp4_codes;
+  const int16_t* fp4_exps;
 };
 
 // Complete top nodes visible to the decode query of sequence `seq` (at
@@ -261,6 +266,221 @@ __global__ void __launch_bounds__(kSThreads, 3) dense_score_kernel(const __grid_
       cur_r0 = nxt_r0;
       cur_n = nxt_n;
     }
+  }
+  cp_async_wait<0>();
+}
+
+// ---------------------------------------------------------------------------
+// 1b. scoring the FP4 router variant's rows (d = 128): 64 bytes of 4-bit codes
+//     per row, one stage per tile, and the row's four block exponents (8
+//     bytes, loaded while the codes land). Each code becomes its exact fp32
+//     value sign * mag[k] * 2^e (k the e2m1 magnitude index), which enters the
+//     same canonical chains as a bf16 or fp32 element would.
+// ---------------------------------------------------------------------------
+
+// The two e2m1 codes of byte `byte` (bits 0-7) as exact fp32 values (the
+// low nibble in .x), by the sm_100 hardware conversion to f16x2.
+__device__ __forceinline__ float2 e2m1x2_to_f2(uint32_t byte) {
+  uint32_t h2;
+  asm("{\n .reg .b8 t;\n cvt.u8.u32 t, %1;\n cvt.rn.f16x2.e2m1x2 %0, t;\n}" : "=r"(h2) : "r"(byte));
+  const __half2 h = *reinterpret_cast<const __half2*>(&h2);
+  return __half22float2(h);
+}
+
+// The fp32 value of code `nib` times 2^e for any e (exact ldexpf scaling):
+// the path of blocks whose scale 2^e is not a normal float.
+__device__ __forceinline__ float fp4_value_any(uint32_t nib, int e) {
+  const uint32_t k = nib & 7u;
+  const float m = k <= 4u ? 0.5f * (float)k : (k == 5u ? 3.0f : (k == 6u ? 4.0f : 6.0f));
+  const float v = ldexpf(m, e);
+  return k == 0u ? 0.0f : ((nib & 8u) ? -v : v);
+}
+
+// One canonical chain step for the 4 rows of a thread: acc_h += q_h[i] * x_k.
+template <int G>
+__device__ __forceinline__ void chain_step(const float* qv, const float* x, float2 (&acc)[4][(G + 1) / 2],
+                                           float (&acc1)[4]) {
+  if constexpr (G == 1) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc1[k] = __fmaf_rn(qv[0], x[k], acc1[k]);
+  } else if constexpr (G == 2) {
+    const float2 q2 = *reinterpret_cast<const float2*>(qv);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[k][0] = ffma2(q2, make_float2(x[k], x[k]), acc[k][0]);
+  } else {
+    float4 q4[G / 4];
+#pragma unroll
+    for (int jj = 0; jj < G / 4; ++jj) q4[jj] = *reinterpret_cast<const float4*>(qv + 4 * jj);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 xx = make_float2(x[k], x[k]);
+#pragma unroll
+      for (int jj = 0; jj < G / 4; ++jj) {
+        acc[k][2 * jj] = ffma2(make_float2(q4[jj].x, q4[jj].y), xx, acc[k][2 * jj]);
+        acc[k][2 * jj + 1] = ffma2(make_float2(q4[jj].z, q4[jj].w), xx, acc[k][2 * jj + 1]);
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t word_of(const uint4& v, int w) {
+  return w == 0 ? v.x : (w == 1 ? v.y : (w == 2 ? v.z : v.w));
+}
+
+__device__ __forceinline__ void stage_fp4_rows(const unsigned char* lvl, int64_t r0, int n,
+                                               unsigned char* dst) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = lane & 3;
+#pragma unroll 4
+  for (int m = 0; m < 16; ++m) {
+    const int row = warp * 128 + m * 8 + (lane >> 2);
+    if (row < n)
+      cp_async16(dst + row * 64 + sswz(c, row) * 16,
+                 reinterpret_cast<const uint4*>(lvl + (r0 + row) * 64) + c);
+  }
+}
+
+template <typename T, int G>
+__global__ void __launch_bounds__(kSThreads, 3)
+    dense_score_fp4_kernel(const __grid_constant__ DenseParams p) {
+  constexpr int D = 128;
+  extern __shared__ __align__(16) unsigned char sm[];
+  float* qs = reinterpret_cast<float*>(sm + 2 * kSStageBytes);  // [D][8]
+  const int unit = p.unit0 + (int)blockIdx.y;
+  const int seq = unit / p.Hkv, kvh = unit % p.Hkv;
+  const int tid = threadIdx.x;
+  const int64_t T_top = decode_top(p, seq);
+  int64_t n_tiles = 0;
+  for (int l = p.L; l >= 1; --l) n_tiles += (level_prefix_rows(p, T_top, l) + kSTile - 1) / kSTile;
+  if (p.stats && blockIdx.x == 0 && tid < p.L)
+    p.stats[(int64_t)unit * p.L + tid] = (int32_t)level_prefix_rows(p, T_top, p.L - tid);
+  if ((int64_t)blockIdx.x >= n_tiles) return;  // uniform over the CTA
+  for (int e = tid; e < D * kMaxGroup; e += kSThreads) {
+    const int i = e / kMaxGroup, h = e % kMaxGroup;
+    qs[e] = h < G ? Elem<T>::to_f(static_cast<const T*>(p.q)[((int64_t)seq * p.Hq + kvh * G + h) * D + i])
+                  : 0.0f;
+  }
+  auto locate = [&](int64_t tile, int* level, int64_t* r0, int* n) {
+    int64_t t = tile;
+    for (int l = p.L; l >= 1; --l) {
+      const int64_t rows = level_prefix_rows(p, T_top, l);
+      const int64_t nt = (rows + kSTile - 1) / kSTile;
+      if (t < nt) {
+        *level = l;
+        *r0 = t * kSTile;
+        *n = (int)(rows - *r0 < kSTile ? rows - *r0 : kSTile);
+        return;
+      }
+      t -= nt;
+    }
+    *level = 0;
+    *r0 = 0;
+    *n = 0;
+  };
+  // element offset of the unit's level `level` in the tree's element order
+  auto elem0 = [&](int level) {
+    return p.level_off[level - 1] + (int64_t)unit * p.level_rows[level - 1] * D;
+  };
+  const int64_t my_tiles = (n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x;
+  int cur_level;
+  int64_t cur_r0;
+  int cur_n;
+  locate(blockIdx.x, &cur_level, &cur_r0, &cur_n);
+  stage_fp4_rows(p.fp4_codes + elem0(cur_level) / 2, cur_r0, cur_n, sm);
+  cp_async_commit();
+  for (int64_t it = 0; it < my_tiles; ++it) {
+    const int64_t tile = blockIdx.x + it * gridDim.x;
+    int nxt_level = 0;
+    int64_t nxt_r0 = 0;
+    int nxt_n = 0;
+    if (it + 1 < my_tiles) {  // prefetch the next tile into the other stage
+      locate(tile + gridDim.x, &nxt_level, &nxt_r0, &nxt_n);
+      stage_fp4_rows(p.fp4_codes + elem0(nxt_level) / 2, nxt_r0, nxt_n,
+                     sm + ((it + 1) & 1) * kSStageBytes);
+    }
+    cp_async_commit();
+    uint2 ex[4];  // the 4 block exponents of each of the thread's rows
+    {
+      const int16_t* el = p.fp4_exps + elem0(cur_level) / 32;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int row = tid + k * kSThreads;
+        ex[k] = row < cur_n ? __ldg(reinterpret_cast<const uint2*>(el + (cur_r0 + row) * 4))
+                            : make_uint2(0u, 0u);
+      }
+    }
+    cp_async_wait<1>();
+    __syncthreads();
+    const unsigned char* st = sm + (it & 1) * kSStageBytes;
+    float2 acc[4][(G + 1) / 2];
+    float acc1[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      acc1[k] = 0.0f;
+#pragma unroll
+      for (int j = 0; j < (G + 1) / 2; ++j) acc[k][j] = make_float2(0.0f, 0.0f);
+    }
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {  // block c: elements 32c .. 32c + 31
+      uint4 cw[4];
+      int eb[4];
+      float sc[4];
+      bool fast = true;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int row = tid + k * kSThreads;
+        cw[k] = lds128(st + row * 64 + sswz(c, row) * 16);
+        const uint32_t pair = c < 2 ? ex[k].x : ex[k].y;
+        eb[k] = (int)(int16_t)((c & 1) ? (pair >> 16) : (pair & 0xffffu));
+        fast = fast && eb[k] >= -126 && eb[k] <= 127;
+        sc[k] = __int_as_float((eb[k] + 127) << 23);  // 2^e while it is a normal float
+      }
+      if (fast) {  // value = e2m1 value * 2^e, an exact product
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+#pragma unroll
+          for (int jb = 0; jb < 4; ++jb) {
+            float x0[4], x1[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float2 v = e2m1x2_to_f2((word_of(cw[k], w) >> (8 * jb)) & 0xffu);
+              x0[k] = __fmul_rn(v.x, sc[k]);
+              x1[k] = __fmul_rn(v.y, sc[k]);
+            }
+            const int i = 32 * c + 8 * w + 2 * jb;
+            chain_step<G>(qs + i * kMaxGroup, x0, acc, acc1);
+            chain_step<G>(qs + (i + 1) * kMaxGroup, x1, acc, acc1);
+          }
+      } else {
+#pragma unroll 1
+        for (int j = 0; j < 32; ++j) {
+          float x[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            x[k] = fp4_value_any((word_of(cw[k], j >> 3) >> (4 * (j & 7))) & 15u, eb[k]);
+          chain_step<G>(qs + (32 * c + j) * kMaxGroup, x, acc, acc1);
+        }
+      }
+    }
+    {  // the rows' chains are complete: store their scores
+      const float lns = p.lnsize[cur_level - 1];
+      float* zl = p.z + (int64_t)unit * G * p.zrows + p.zoff[cur_level - 1] + cur_r0;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int row = tid + k * kSThreads;
+        if (row < cur_n) {
+#pragma unroll
+          for (int h = 0; h < G; ++h) {
+            const float raw = (G == 1) ? acc1[k] : ((h & 1) ? acc[k][h / 2].y : acc[k][h / 2].x);
+            zl[(int64_t)h * p.zrows + row] = __fadd_rn(__fmul_rn(raw, p.inv_sqrt_d), lns);
+          }
+        }
+      }
+    }
+    __syncthreads();  // this stage is refilled by the next iteration's prefetch
+    cur_level = nxt_level;
+    cur_r0 = nxt_r0;
+    cur_n = nxt_n;
   }
   cp_async_wait<0>();
 }
@@ -1224,8 +1444,33 @@ cudaError_t launch_score(const DenseParams& p, int units, int sms, cudaStream_t 
   return cudaGetLastError();
 }
 
+template <typename T, int G>
+cudaError_t launch_score_fp4(const DenseParams& p, int units, int sms, cudaStream_t s) {
+  auto kern = dense_score_fp4_kernel<T, G>;
+  const int smem = 2 * kSStageBytes + 128 * kMaxGroup * 4;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  int per = 3 * sms / units;  // three CTAs per SM
+  if (per < 1) per = 1;
+  kern<<<dim3((unsigned)per, (unsigned)units), kSThreads, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
 template <typename T, int D>
 cudaError_t launch_score_g(const DenseParams& p, int units, int sms, cudaStream_t s) {
+  if constexpr (D == 128) {
+    if (p.fp4_codes) {
+      switch (p.G) {
+        case 1: return launch_score_fp4<T, 1>(p, units, sms, s);
+        case 2: return launch_score_fp4<T, 2>(p, units, sms, s);
+        case 4: return launch_score_fp4<T, 4>(p, units, sms, s);
+        case 8: return launch_score_fp4<T, 8>(p, units, sms, s);
+        default: return cudaErrorInvalidValue;
+      }
+    }
+  } else {
+    if (p.fp4_codes) return cudaErrorInvalidValue;
+  }
   switch (p.G) {
     case 1: return launch_score<T, D, 1>(p, units, sms, s);
     case 2: return launch_score<T, D, 2>(p, units, sms, s);
@@ -1289,7 +1534,8 @@ cudaError_t launch_decode_dense(const Geometry& g, const void* tree, const void*
                                 const int32_t* seq_len, uint64_t p_q, void* ws,
                                 int32_t* level_counts, int32_t* stats, uint32_t* kept,
                                 int32_t* n_kept, int64_t kept_stride, int segs, int32_t* status,
-                                int num_sms, cudaStream_t stream, int64_t unit0, int64_t n_units) {
+                                int num_sms, cudaStream_t stream, int64_t unit0, int64_t n_units,
+                                const void* fp4_tree) {
   const int64_t all_units = (int64_t)g.B * g.Hkv;
   const int64_t units = n_units > 0 ? n_units : all_units;
   if (unit0 < 0 || unit0 + units > all_units) return cudaErrorInvalidValue;
@@ -1331,6 +1577,11 @@ cudaError_t launch_decode_dense(const Geometry& g, const void* tree, const void*
   p.kept_stride = kept_stride;
   p.segs = segs;
   p.unit0 = (int)unit0;
+  if (fp4_tree) {
+    p.fp4_codes = static_cast<const unsigned char*>(fp4_tree);
+    p.fp4_exps = reinterpret_cast<const int16_t*>(static_cast<const unsigned char*>(fp4_tree) +
+                                                  fp4_codes_bytes(g));
+  }
   cudaError_t e;
   if (g.dtype == ZHA_BF16)
     e = g.d == 128 ? launch_score_g<__nv_bfloat16, 128>(p, (int)units, num_sms, stream)

@@ -84,13 +84,25 @@ size_t decode_dense_ws_bytes(const Geometry& g, int64_t units);
 // Decode mode only (query of sequence s at seq_len[s] - 1): writes the kept
 // level-1 union with per-head masks in `segs` ordered segments per unit, the
 // per-head level counts (nullable) and the rows scored per level (stats).
-// Units [unit0, unit0 + n_units) only when n_units > 0.
+// Units [unit0, unit0 + n_units) only when n_units > 0. fp4_tree (nullable,
+// d = 128): score the FP4 router variant's 4-bit rows instead of the tree's.
 cudaError_t launch_decode_dense(const Geometry& g, const void* tree, const void* q,
                                 const int32_t* seq_len, uint64_t p_q, void* ws,
                                 int32_t* level_counts, int32_t* stats, uint32_t* kept,
                                 int32_t* n_kept, int64_t kept_stride, int segs, int32_t* status,
                                 int num_sms, cudaStream_t stream, int64_t unit0 = 0,
-                                int64_t n_units = 0);
+                                int64_t n_units = 0, const void* fp4_tree = nullptr);
+
+// ---- FP4 router variant: block-scaled 4-bit copy of the tree ------------------
+// Layout: codes of tree element i in byte i / 2 (low nibble for even i), then
+// at fp4_codes_bytes the int16 exponent of block i / 32 (32 elements).
+size_t fp4_codes_bytes(const Geometry& g);
+size_t fp4_tree_bytes(const Geometry& g);
+// Quantizes the rows of every node complete at seq_len (old_len null) or
+// completed in (old_len, seq_len].
+cudaError_t launch_fp4_quantize(const Geometry& g, const void* tree, void* fp4,
+                                const int32_t* seq_len, const int32_t* old_len, int num_sms,
+                                cudaStream_t stream);
 
 // ---- prefill top level on the tensor cores ----------------------------------
 // Top nodes per (sequence, KV head): ncap / b^L.
