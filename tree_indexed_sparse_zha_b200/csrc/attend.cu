@@ -528,28 +528,16 @@ __global__ void __launch_bounds__(MmaCfg<D>::kThreads, 1) attend_mma_kernel(AttP
     s.t1 = tail_len * (split + 1) / p.S;
     s.rows = s.tok0 + (s.n1 - s.n0) * p.b + (s.t1 - s.t0);
     if (s.n1 - s.n0 <= C::kKeptCap) {  // stage this CTA's kept entries in smem once
-      // four entries per thread and batch, their global loads in flight
-      // together: the streaming below waits for this prologue
+      // every entry's 4-byte asynchronous copy is issued before the one wait:
+      // the streaming below waits for this prologue
       uint32_t* kl = reinterpret_cast<uint32_t*>(smem + C::kWarps * C::kWarpBytes);
-      constexpr int kB = 4;
       int r = 0;  // segment cursor: this thread's entries only grow
-      for (int64_t j0 = s.n0 + tid; j0 < s.n1; j0 += kB * C::kThreads) {
-        uint32_t v[kB];
-#pragma unroll
-        for (int u = 0; u < kB; ++u) {
-          const int64_t j = j0 + (int64_t)u * C::kThreads;
-          v[u] = 0u;
-          if (j < s.n1) {
-            while ((int64_t)s_segbase[r + 1] <= j) ++r;
-            v[u] = __ldg(s.kept + r * s.stride + (j - s_segbase[r]));
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < kB; ++u) {
-          const int64_t j = j0 + (int64_t)u * C::kThreads;
-          if (j < s.n1) kl[j - s.n0] = v[u];
-        }
+      for (int64_t j = s.n0 + tid; j < s.n1; j += C::kThreads) {
+        while ((int64_t)s_segbase[r + 1] <= j) ++r;
+        cp_async4(kl + (j - s.n0), s.kept + r * s.stride + (j - s_segbase[r]));
       }
+      cp_async_commit();
+      cp_async_wait<0>();
       s.kept_local = kl;
       __syncthreads();
     }
