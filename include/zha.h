@@ -170,8 +170,12 @@ zha_status zha_attend(const zha_config* cfg, const zha_cache* cache, const void*
  * top-p descent at p = 0.95 followed by exact attention over the selected raw
  * keys, token 0 and the causal tail): selection at position seq_len[b] - 1
  * followed by attention over the selected keys, q [B][Hq][d] -> out [B][Hq][d].
- * The query heads sharing a KV head are traversed together and their
- * selections are read from HBM once (per-head masks). level_counts is
+ * The query heads sharing a KV head share every read: each summary row is
+ * scored for all of them in one pass (every row under the complete top nodes,
+ * while that prefix is at most 1.5 GB; above it the cluster traversal of
+ * zha_select scores the union of their frontiers), each head then cuts its own
+ * frontier, and the K/V rows of their kept nodes are read once with per-head
+ * masks. level_counts is
  * nullable. The tree must already contain every node complete at seq_len
  * (call zha_extend_tree after appending tokens). ws: ZHA_OP_DECODE workspace.
  * Streams: the (sequence, KV head) units are split into up to 4 groups whose
@@ -187,11 +191,12 @@ zha_status zha_decode(const zha_config* cfg, const zha_cache* cache, const void*
                       void* out, int32_t* level_counts, void* ws, size_t ws_bytes,
                       int32_t* dev_status, void* stream);
 
-/* The two halves of zha_decode, for callers that schedule or time them
- * separately. zha_decode_select runs the traversal for every sequence and
- * leaves the kept level-1 nodes (union over the query heads of each KV head,
- * with per-head masks) in ws; zha_decode_attend then attends over them. Both
- * must get the same cfg, cache, q and ws; nothing may touch ws in between. */
+/* The two halves of zha_decode on `stream` alone, for callers that schedule
+ * or time them separately. zha_decode_select runs the selection for every
+ * sequence and leaves the kept level-1 nodes (union over the query heads of
+ * each KV head, with per-head masks) in ws; zha_decode_attend then attends
+ * over them. Both must get the same cfg, cache, q and ws; nothing may touch
+ * ws in between. */
 zha_status zha_decode_select(const zha_config* cfg, const zha_cache* cache, const void* q,
                              double p, int32_t* level_counts, void* ws, size_t ws_bytes,
                              int32_t* dev_status, void* stream);
