@@ -170,6 +170,7 @@ struct TileCfg {
   static constexpr int kRtBytes = kNRef * D * 4;
   static constexpr int kWBytes = kTileRows * kNRef * 4;
   static constexpr int kSmem = kStageBytes + kRtBytes + kWBytes + kTileRows * 4;
+  static constexpr int kSmemB4 = kStageBytes + kRtBytes + kTileRows * 4;  // no logit buffer
 };
 
 // Chunk ch of staged row r sits at chunk ch ^ ((r >> 2) & 7): the 8 rows one
@@ -187,7 +188,13 @@ __device__ __forceinline__ void stage_tile(const T* src, int rows, unsigned char
   }
 }
 
-template <typename T, int D>
+// B4 (b == 4): a thread's 4 children are exactly one node, so phases 2 and 3
+// run in its registers: the softmax over the node's children for its 4
+// reference queries, then each child's weight sum in r order, handed from
+// the lane holding r = 0..3 to the one holding r = 12..15 (the 4 lanes of a
+// node are adjacent). The same rounded operations in the same order as the
+// shared-memory phases, without the logit buffer and two barriers.
+template <typename T, int D, bool B4>
 __global__ void __launch_bounds__(kTileThreads) tree_level_tiled(const __grid_constant__ TreeParams p,
                                                                  int level) {
   using C = TileCfg<T, D>;
@@ -195,8 +202,8 @@ __global__ void __launch_bounds__(kTileThreads) tree_level_tiled(const __grid_co
   extern __shared__ __align__(16) float sm[];
   unsigned char* X = reinterpret_cast<unsigned char*>(sm);  // the tile's staged rows
   float* Rt = reinterpret_cast<float*>(X + C::kStageBytes);  // [D][16]
-  float* W = Rt + kNRef * D;                                // [tile rows][16]
-  float* A = W + kTileRows * kNRef;                         // [tile rows]
+  float* W = Rt + kNRef * D;                                // [tile rows][16] (not B4)
+  float* A = B4 ? W : W + kTileRows * kNRef;                // [tile rows]
   const int tid = threadIdx.x;
   const int unit = blockIdx.y;
   const int seq = unit / p.Hkv;
@@ -246,15 +253,65 @@ __global__ void __launch_bounds__(kTileThreads) tree_level_tiled(const __grid_co
           }
         }
       }
+      if constexpr (B4) {
+        float l[4][4];  // [child][reference query 4rg + j]
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
-        *reinterpret_cast<float4*>(W + (4 * cg + k) * kNRef + 4 * rg) =
-            make_float4(__fmul_rn(acc[k][0].x, inv_sqrt_d), __fmul_rn(acc[k][0].y, inv_sqrt_d),
-                        __fmul_rn(acc[k][1].x, inv_sqrt_d), __fmul_rn(acc[k][1].y, inv_sqrt_d));
+        for (int k = 0; k < 4; ++k) {
+          l[k][0] = __fmul_rn(acc[k][0].x, inv_sqrt_d);
+          l[k][1] = __fmul_rn(acc[k][0].y, inv_sqrt_d);
+          l[k][2] = __fmul_rn(acc[k][1].x, inv_sqrt_d);
+          l[k][3] = __fmul_rn(acc[k][1].y, inv_sqrt_d);
+        }
+        // ---- 2. softmax over the node's children, per reference query ----
+        float w[4][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float mu = l[0][j];
+#pragma unroll
+          for (int k = 1; k < 4; ++k) mu = fmaxf(mu, l[k][j]);
+          float e[4], Z = 0.0f;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            e[k] = exp_canon(__fsub_rn(l[k][j], mu));
+            Z = __fadd_rn(Z, e[k]);
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k) w[k][j] = __fdiv_rn(e[k], Z);
+        }
+        // ---- 3. child weights a_c: r = 0..15 in order across the node's lanes ----
+        float part[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int step = 0; step < 4; ++step) {
+          if (rg == step) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+#pragma unroll
+              for (int j = 0; j < 4; ++j) part[k] = __fadd_rn(part[k], w[k][j]);
+          }
+          if (step < 3) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float v = __shfl_up_sync(0xffffffffu, part[k], 1);
+              if (rg == step + 1) part[k] = v;
+            }
+          }
+        }
+        if (rg == 3) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) A[4 * cg + k] = __fmul_rn(part[k], 0.0625f);
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          *reinterpret_cast<float4*>(W + (4 * cg + k) * kNRef + 4 * rg) =
+              make_float4(__fmul_rn(acc[k][0].x, inv_sqrt_d), __fmul_rn(acc[k][0].y, inv_sqrt_d),
+                          __fmul_rn(acc[k][1].x, inv_sqrt_d), __fmul_rn(acc[k][1].y, inv_sqrt_d));
+      }
     }
     __syncthreads();
-    // ---- 2. softmax over each node's children, per reference query ----
     const int nodes = rows / b;
+    if constexpr (!B4) {
+    // ---- 2. softmax over each node's children, per reference query ----
     for (int task = tid; task < nodes * kNRef; task += kTileThreads) {
       const int n = task / kNRef, r = task % kNRef;
       float* w = W + (n * b) * kNRef + r;
@@ -277,6 +334,7 @@ __global__ void __launch_bounds__(kTileThreads) tree_level_tiled(const __grid_co
       A[c] = __fmul_rn(a, 0.0625f);
     }
     __syncthreads();
+    }
     // ---- 4. weighted sums, one 16-byte output chunk per task ----
     for (int task = tid; task < nodes * kNch; task += kTileThreads) {
       const int n = task / kNch, ch = task % kNch;
@@ -411,12 +469,13 @@ cudaError_t launch_tree_t(const Geometry& g, const TreeParams& p, int64_t max_ne
     if (nodes <= 0) break;
     if (small_b) {
       using C = TileCfg<T, D>;
-      cudaError_t e = cudaFuncSetAttribute(tree_level_tiled<T, D>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+      const bool b4 = g.b == 4;
+      auto kern = b4 ? tree_level_tiled<T, D, true> : tree_level_tiled<T, D, false>;
+      const int smem = b4 ? C::kSmemB4 : C::kSmem;
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       if (e != cudaSuccess) return e;
       int per_sm = 0;
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tree_level_tiled<T, D>,
-                                                        kTileThreads, C::kSmem);
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kTileThreads, smem);
       if (e != cudaSuccess) return e;
       // at most one wave (a partial second wave would run a whole CTA's share
       // of tiles after the first): the resident slots shared evenly by the
@@ -426,7 +485,7 @@ cudaError_t launch_tree_t(const Geometry& g, const TreeParams& p, int64_t max_ne
       if (per_unit < 1) per_unit = 1;
       if (per_unit > tiles) per_unit = tiles;
       dim3 grid((unsigned)per_unit, (unsigned)units);
-      tree_level_tiled<T, D><<<grid, kTileThreads, C::kSmem, stream>>>(p, level);
+      kern<<<grid, kTileThreads, smem, stream>>>(p, level);
     } else {
       const size_t smem = sizeof(float) * (kNRef * D + kNRef * g.b + g.b + 32 * kNRef + kNRef);
       cudaError_t e = cudaFuncSetAttribute(tree_level_large_b<T, D>,
