@@ -188,12 +188,13 @@ __device__ __forceinline__ void stage_tile(const T* src, int rows, unsigned char
   }
 }
 
-// B4 (b == 4): a thread's 4 children are exactly one node, so phases 2 and 3
+// B4 (b == 4): a thread's 4 children are exactly one node, so phases 2 to 4
 // run in its registers: the softmax over the node's children for its 4
-// reference queries, then each child's weight sum in r order, handed from
-// the lane holding r = 0..3 to the one holding r = 12..15 (the 4 lanes of a
-// node are adjacent). The same rounded operations in the same order as the
-// shared-memory phases, without the logit buffer and two barriers.
+// reference queries, each child's weight sum in r order, handed from the lane
+// holding r = 0..3 to the one holding r = 12..15 (the 4 lanes of a node are
+// adjacent), then a quarter of the node's output chunks. The same rounded
+// operations in the same order as the shared-memory phases, without the
+// logit buffer and with one barrier per tile instead of four.
 template <typename T, int D, bool B4>
 __global__ void __launch_bounds__(kTileThreads) tree_level_tiled(const __grid_constant__ TreeParams p,
                                                                  int level) {
@@ -296,9 +297,29 @@ __global__ void __launch_bounds__(kTileThreads) tree_level_tiled(const __grid_co
             }
           }
         }
-        if (rg == 3) {
+        // ---- 4. the node's weighted sum: chunks rg, rg + 4, ... of its output
+        //    row, each element a chain over the 4 children in order ----
+        float a[4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) A[4 * cg + k] = __fmul_rn(part[k], 0.0625f);
+        for (int k = 0; k < 4; ++k)
+          a[k] = __shfl_sync(0xffffffffu, __fmul_rn(part[k], 0.0625f), ((tid & 31) & ~3) | 3);
+        if (4 * cg < rows) {
+#pragma unroll
+          for (int m = 0; m < kNch / 4; ++m) {
+            const int ch = rg + 4 * m;
+            float sum[kPer];
+#pragma unroll
+            for (int e = 0; e < kPer; ++e) sum[e] = 0.0f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int r = 4 * cg + k;
+              float x[kPer];
+              Elem<T>::unpack(lds128(X + ((int64_t)r * kNch + tswz(ch, r)) * 16), x);
+#pragma unroll
+              for (int e = 0; e < kPer; ++e) sum[e] = __fmaf_rn(a[k], x[e], sum[e]);
+            }
+            *reinterpret_cast<uint4*>(ob + (r0 / 4 + cg) * D + ch * kPer) = Elem<T>::pack(sum);
+          }
         }
       } else {
 #pragma unroll
@@ -308,9 +329,9 @@ __global__ void __launch_bounds__(kTileThreads) tree_level_tiled(const __grid_co
                           __fmul_rn(acc[k][1].x, inv_sqrt_d), __fmul_rn(acc[k][1].y, inv_sqrt_d));
       }
     }
+    if constexpr (!B4) {
     __syncthreads();
     const int nodes = rows / b;
-    if constexpr (!B4) {
     // ---- 2. softmax over each node's children, per reference query ----
     for (int task = tid; task < nodes * kNRef; task += kTileThreads) {
       const int n = task / kNRef, r = task % kNRef;
@@ -334,7 +355,6 @@ __global__ void __launch_bounds__(kTileThreads) tree_level_tiled(const __grid_co
       A[c] = __fmul_rn(a, 0.0625f);
     }
     __syncthreads();
-    }
     // ---- 4. weighted sums, one 16-byte output chunk per task ----
     for (int task = tid; task < nodes * kNch; task += kTileThreads) {
       const int n = task / kNch, ch = task % kNch;
@@ -350,6 +370,7 @@ __global__ void __launch_bounds__(kTileThreads) tree_level_tiled(const __grid_co
         for (int e = 0; e < kPer; ++e) s[e] = __fmaf_rn(a, x[e], s[e]);
       }
       *reinterpret_cast<uint4*>(ob + (r0 / b + n) * D + ch * kPer) = Elem<T>::pack(s);
+    }
     }
     __syncthreads();  // the stage is refilled by the next tile
   }
