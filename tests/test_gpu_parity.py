@@ -280,3 +280,44 @@ def test_select_one_cta_narrowed_groups():
                 assert n_idx[i, h] == len(e_idx), (p, i, h, n_idx[i, h], len(e_idx))
                 assert np.array_equal(rows[h, :n_idx[i, h]], e_idx), (p, i, h)
         del idx
+
+
+@pytest.mark.parametrize("dtype,d,b,L,n", [
+    ("f32", 64, 64, 2, 64 * 64 * 3 + 70),     # two levels, ragged tail
+    ("bf16", 128, 96, 1, 96 * 40 + 5),        # b not a power of two
+    ("bf16", 64, 128, 2, 128 * 128 + 300),
+    ("f32", 128, 256, 1, 256 * 30 + 17),      # the widest staged kernel, fp32 rows
+    ("bf16", 128, 512, 1, 512 * 9 + 100),     # one CTA of b threads per node
+])
+def test_tree_wide_blocks_ragged_and_extend(dtype, d, b, L, n):
+    """Summary trees with wide blocks against the oracle, bit for bit: built
+    over ragged lengths (3 sequences, 2 KV heads), then extended by a few
+    hundred tokens per sequence (nodes completed by the new tokens only)."""
+    import oracle
+    import tree_indexed_sparse_zha_b200 as z
+    cfg = W.WorkloadConfig(f"tree-b{b}", 5, dtype, 3, 4, 2, d, n, b, L, 0.95, (1, 2), steps=600)
+    wl = W.Workload(cfg)
+    gpu = Gpu(wl, build=False)
+    lens0 = [n - 3 * b - 1, n, b ** L - 1]
+    gpu.cache.seq_len.copy_(torch.tensor(lens0, dtype=torch.int32))
+    z.zha_build_tree(gpu.cfg, gpu.cache)
+    K = wl.K.float().numpy()
+    R = wl.R.numpy()
+
+    def check(lens):
+        torch.cuda.synchronize()
+        for s in range(cfg.batch):
+            for kvh in range(cfg.n_kv_heads):
+                got = gpu.tree_unit(s, kvh)
+                exp = oracle.build_tree(K[s, kvh], lens[s], R, b, L, dtype == "bf16", cfg.capacity)
+                for l in range(1, L + 1):
+                    m = lens[s] // b ** l
+                    a, e = got[l - 1][:m], exp.level(l)[:m]
+                    assert np.array_equal(a.view(np.uint32), e.view(np.uint32)), (s, kvh, l)
+
+    check(lens0)
+    old = gpu.cache.seq_len.clone()
+    lens1 = [x + 600 for x in lens0]
+    gpu.cache.seq_len.copy_(torch.tensor(lens1, dtype=torch.int32))
+    z.zha_extend_tree(gpu.cfg, gpu.cache, old, 600)
+    check(lens1)

@@ -11,10 +11,12 @@
 //     w_rc = e_rc / Z_r ; a_c = (sum_r w_rc, r order) * 1/16
 //     s_i  = sum_c fmaf(a_c, x_ci, .) in c order from +0, stored RNE in the I/O type
 //
-// Layout: one thread per child row computes its 16 logits (16 independent
-// chains, packed two per fp32x2 FMA); the b threads of a node exchange values
-// by warp shuffles (b <= 32) or through shared memory (b = 64..1024, one CTA
-// per node). The work is FP32-ALU bound: 16 d FMAs per child row.
+// Layout: the level kernels stage child rows in shared memory and give each
+// thread a 4 x 4 block of (child, reference query) logit chains, packed two
+// per fp32x2 FMA: tiles of whole nodes for b <= 32, one node per CTA
+// iteration for b = 64..256; wider blocks take one CTA of b threads per node,
+// one child row per thread. The work is FP32-ALU bound: 16 d FMAs per child
+// row.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -472,6 +474,200 @@ __global__ void __launch_bounds__(1024) tree_level_large_b(TreeParams p, int lev
   }
 }
 
+// ---------------------------------------------------------------------------
+// Level kernel for 64 <= b <= 256 (b a multiple of 32): a CTA takes one node
+// at a time, its b child rows staged in shared memory by cp.async (swizzled
+// as in the tiled kernel), then
+//   1. thread (cg, rg) runs the 16 canonical logit chains of children
+//      4cg..4cg+3 against reference queries 4rg..4rg+3 (b threads busy);
+//      its maxima over its 4 children go through warp shuffles and one
+//      shared slot per warp to the node maxima mu_r;
+//   2. the exponentials stay in the thread's registers; one copy goes to
+//      shared memory, where 16 threads form Z_r over the children in order;
+//   3. w_rc = e_rc / Z_r in registers, and a_c = (sum_r w_rc in r order) / 16
+//      handed along the 4 lanes of a child group (r = 0..3 first);
+//   4. thread i runs output element i's chain over the children in order.
+// The same rounded operations in the same order as the per-node form
+// (tree_level_large_b), so the stored summaries are bit-identical.
+// ---------------------------------------------------------------------------
+constexpr int kBigThreads = 256;
+constexpr int kBigMaxB = 256;  // one 4x4 logit block per thread and node
+
+template <typename T, int D>
+size_t big_b_smem(int b) {
+  // rows [b][D], Rt [D][16], E [16][b + 4], warp maxima [8][16], a [b], Z [16]
+  return (size_t)b * D * sizeof(T) +
+         sizeof(float) * ((size_t)kNRef * D + (size_t)kNRef * (b + 4) + 8 * kNRef + b + kNRef);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kBigThreads) tree_level_big_b(const __grid_constant__ TreeParams p,
+                                                                int level) {
+  constexpr int kPer = Elem<T>::kPerChunk;
+  constexpr int kNch = D * (int)sizeof(T) / 16;  // chunks per row
+  extern __shared__ __align__(16) float sm[];
+  const int b = p.b;
+  const int es = b + 4;  // row stride of E: 16-byte rows, a quarter-warp's float4 stores spread
+  unsigned char* X = reinterpret_cast<unsigned char*>(sm);             // [b][kNch] chunks
+  float* Rt = reinterpret_cast<float*>(X + (size_t)b * D * sizeof(T));  // [D][16]
+  float* E = Rt + kNRef * D;                                           // [16][es]
+  float* red = E + kNRef * es;                                         // [8][16]
+  float* A = red + 8 * kNRef;                                          // [b]
+  float* Zs = A + b;                                                   // [16]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int rg = tid & 3, cg = tid >> 2;  // logit block: 4 children x 4 reference queries
+  const bool blk = tid < b;               // whole warps (b is a multiple of 32)
+  const int nw = b >> 5;                  // warps holding a block
+  const int unit = blockIdx.y;
+  const int seq = unit / p.Hkv;
+  const int64_t span = p.span[level];
+  const int64_t n_new = clamp_len(p.seq_len[seq], p.ncap);
+  const int64_t n_old = p.old_len ? clamp_len(p.old_len[seq], p.ncap) : 0;
+  const int64_t lo = (n_old < n_new ? n_old : n_new) / span;
+  const int64_t hi = n_new / span;
+  if (lo + blockIdx.x >= hi) return;  // uniform over the CTA
+  const T* cb = child_base<T, D>(p, level, unit);
+  T* ob = level_base<T, D>(p, level, unit);
+  load_rt<D>(p.r, Rt);
+  const float inv_sqrt_d = p.inv_sqrt_d;
+  for (int64_t node = lo + blockIdx.x; node < hi; node += gridDim.x) {
+    const T* rows = cb + node * b * D;
+    for (int e = tid; e < b * kNch; e += kBigThreads) {
+      const int r = e / kNch, ch = e % kNch;
+      cp_async16(X + ((int64_t)r * kNch + tswz(ch, r)) * 16,
+                 reinterpret_cast<const uint4*>(rows + (int64_t)r * D) + ch);
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();  // the rows (and, the first time, R) are in place
+    float l[4][4];    // [child 4cg + k][reference query 4rg + j]
+    // ---- 1. logits, then the block's maxima per reference query ----
+    if (blk) {
+      float2 acc[4][2];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) acc[k][0] = acc[k][1] = make_float2(0.0f, 0.0f);
+#pragma unroll 2
+      for (int ch = 0; ch < kNch; ++ch) {
+        float x[4][kPer];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int r = 4 * cg + k;
+          Elem<T>::unpack(lds128(X + ((int64_t)r * kNch + tswz(ch, r)) * 16), x[k]);
+        }
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) {
+          const float4 rv = *reinterpret_cast<const float4*>(Rt + (ch * kPer + e) * kNRef + 4 * rg);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 xx = make_float2(x[k][e], x[k][e]);
+            acc[k][0] = ffma2(make_float2(rv.x, rv.y), xx, acc[k][0]);
+            acc[k][1] = ffma2(make_float2(rv.z, rv.w), xx, acc[k][1]);
+          }
+        }
+      }
+      float m[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        l[k][0] = __fmul_rn(acc[k][0].x, inv_sqrt_d);
+        l[k][1] = __fmul_rn(acc[k][0].y, inv_sqrt_d);
+        l[k][2] = __fmul_rn(acc[k][1].x, inv_sqrt_d);
+        l[k][3] = __fmul_rn(acc[k][1].y, inv_sqrt_d);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        m[j] = fmaxf(fmaxf(l[0][j], l[1][j]), fmaxf(l[2][j], l[3][j]));
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1)  // lanes of the same rg
+          m[j] = fmaxf(m[j], __shfl_xor_sync(0xffffffffu, m[j], off));
+      }
+      if (lane < 4) *reinterpret_cast<float4*>(red + warp * kNRef + 4 * rg) = make_float4(m[0], m[1], m[2], m[3]);
+    }
+    __syncthreads();
+    // ---- 2. exponentials against the node maxima; E for the Z chains ----
+    if (blk) {
+      float4 mu = *reinterpret_cast<const float4*>(red + 4 * rg);
+      for (int w = 1; w < nw; ++w) {
+        const float4 v = *reinterpret_cast<const float4*>(red + w * kNRef + 4 * rg);
+        mu = make_float4(fmaxf(mu.x, v.x), fmaxf(mu.y, v.y), fmaxf(mu.z, v.z), fmaxf(mu.w, v.w));
+      }
+      const float muj[4] = {mu.x, mu.y, mu.z, mu.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) l[k][j] = exp_canon(__fsub_rn(l[k][j], muj[j]));
+        *reinterpret_cast<float4*>(E + (4 * rg + j) * es + 4 * cg) =
+            make_float4(l[0][j], l[1][j], l[2][j], l[3][j]);
+      }
+    }
+    __syncthreads();
+    if (tid < kNRef) {  // Z_r: the children in order
+      const float* e = E + tid * es;
+      float Z = 0.0f;
+      for (int c = 0; c < b; c += 8) {
+        const float4 v0 = *reinterpret_cast<const float4*>(e + c);
+        const float4 v1 = *reinterpret_cast<const float4*>(e + c + 4);
+        Z = __fadd_rn(Z, v0.x);
+        Z = __fadd_rn(Z, v0.y);
+        Z = __fadd_rn(Z, v0.z);
+        Z = __fadd_rn(Z, v0.w);
+        Z = __fadd_rn(Z, v1.x);
+        Z = __fadd_rn(Z, v1.y);
+        Z = __fadd_rn(Z, v1.z);
+        Z = __fadd_rn(Z, v1.w);
+      }
+      Zs[tid] = Z;
+    }
+    __syncthreads();
+    // ---- 3. child weights a_c: r = 0..15 in order across the group's lanes ----
+    if (blk) {
+      const float4 z = *reinterpret_cast<const float4*>(Zs + 4 * rg);
+      const float zj[4] = {z.x, z.y, z.z, z.w};
+      float part[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+      for (int step = 0; step < 4; ++step) {
+        if (rg == step) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) part[k] = __fadd_rn(part[k], __fdiv_rn(l[k][j], zj[j]));
+        }
+        if (step < 3) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float v = __shfl_up_sync(0xffffffffu, part[k], 1);
+            if (rg == step + 1) part[k] = v;
+          }
+        }
+      }
+      if (rg == 3)
+        *reinterpret_cast<float4*>(A + 4 * cg) =
+            make_float4(__fmul_rn(part[0], 0.0625f), __fmul_rn(part[1], 0.0625f),
+                        __fmul_rn(part[2], 0.0625f), __fmul_rn(part[3], 0.0625f));
+    }
+    __syncthreads();
+    // ---- 4. output element tid: a chain over the children in order ----
+    if (tid < D) {
+      const int ch = tid / kPer, pos = tid % kPer;
+      float s = 0.0f;
+      for (int c = 0; c < b; c += 8) {
+        const float4 a0 = *reinterpret_cast<const float4*>(A + c);
+        const float4 a1 = *reinterpret_cast<const float4*>(A + c + 4);
+        const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        float xv[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int cc = c + u;
+          xv[u] = Elem<T>::to_f(*(reinterpret_cast<const T*>(X + ((int64_t)cc * kNch + tswz(ch, cc)) * 16) + pos));
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) s = __fmaf_rn(av[u], xv[u], s);
+      }
+      ob[node * D + tid] = Elem<T>::from_f(s);
+    }
+    __syncthreads();  // the rows are restaged for the next node
+  }
+}
+
 template <typename T, int D>
 cudaError_t launch_tree_t(const Geometry& g, const TreeParams& p, int64_t max_new_tokens,
                           cudaStream_t stream) {
@@ -507,6 +703,19 @@ cudaError_t launch_tree_t(const Geometry& g, const TreeParams& p, int64_t max_ne
       if (per_unit > tiles) per_unit = tiles;
       dim3 grid((unsigned)per_unit, (unsigned)units);
       kern<<<grid, kTileThreads, smem, stream>>>(p, level);
+    } else if (g.b <= kBigMaxB) {
+      const size_t smem = big_b_smem<T, D>(g.b);
+      auto kern = tree_level_big_b<T, D>;
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      int per_sm = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kBigThreads, smem);
+      if (e != cudaSuccess) return e;
+      // one wave of resident CTAs shared by the units, each looping over nodes
+      int64_t per_unit = ((int64_t)device_sm_count() * (per_sm > 0 ? per_sm : 1)) / units;
+      if (per_unit < 1) per_unit = 1;
+      if (per_unit > nodes) per_unit = nodes;
+      kern<<<dim3((unsigned)per_unit, (unsigned)units), kBigThreads, smem, stream>>>(p, level);
     } else {
       const size_t smem = sizeof(float) * (kNRef * D + kNRef * g.b + g.b + 32 * kNRef + kNRef);
       cudaError_t e = cudaFuncSetAttribute(tree_level_large_b<T, D>,
