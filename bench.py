@@ -13,6 +13,8 @@ needed between steps.
 chunk (16 query / 2 KV heads) after 1,048,576 cached tokens, one step being
 zha_prefill_chunk over the whole chunk (tree extension, tensor-core top level
 with certificates, traversal and sparse attention for all 65,536 queries).
+The default decode line also carries a short run of it (`prefill_chunk`), as
+well as the wide-tree p sweep and the other workloads' tree builds.
 
 One JSON line on rank 0. Under torchrun every rank runs an independent replica
 (weak scaling, no data-path collective); timing is the max over ranks.
@@ -652,6 +654,24 @@ def wide_p_sweep(dev, peak: float, steps: int = 20, warmup: int = 3) -> list:
     return res
 
 
+def prefill_chunk_leg(rank, world, dev, steps: int = 3, warmup: int = 3) -> dict:
+    """The chunked-prefill workload at full size, timed as `--workload
+    prefill-deep-1m-chunk4k` times it but over a few steps: one step is
+    zha_prefill_chunk over the 4096-token chunk after 1,048,576 cached tokens.
+    A failure is reported in the returned entry instead of ending the run."""
+    a = argparse.Namespace(workload="prefill-deep-1m-chunk4k", steps=steps, warmup=warmup,
+                           n_tokens=None)
+    try:
+        r, wl = run_prefill(a, rank, world, dev)
+    except Exception as e:  # noqa: BLE001 -- recorded in the JSON line
+        return {"error": f"{type(e).__name__}: {e}"[:300]}
+    del wl
+    torch.cuda.empty_cache()
+    keep = ("metric", "value", "unit", "steps", "warmup", "ms_per_step", "config",
+            "tensor_core_top_level", "roofline", "tree_build", "e2e", "gpu_launches", "clocks")
+    return {k: r[k] for k in keep}
+
+
 def run_zha(args, rank, world, dev):
     import tree_indexed_sparse_zha_b200 as z
     from tree_indexed_sparse_zha_b200 import workloads as W
@@ -893,6 +913,7 @@ def run_zha(args, rank, world, dev):
     if args.n_tokens is None:  # the other workloads at their full sizes
         res["decode_wide_p_sweep"] = wide_p_sweep(dev, peak)
         res["tree_build_other_workloads"] = tree_builds_other_workloads(dev, peak)
+        res["prefill_chunk"] = prefill_chunk_leg(rank, world, dev)
     return res, wl
 
 
