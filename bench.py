@@ -154,6 +154,20 @@ def strip_c_comments(src: str) -> str:
     return " ".join("".join(out).split())
 
 
+def prefill_selection(lc, b: int, L: int, start: int) -> dict:
+    """Per-query selection figures of a prefill chunk from kept counts lc
+    [T][Hq][L] (top level first), token i of the chunk at position start + i:
+    the mean kept nodes per level, and the mean fraction of the t + 1 visible
+    tokens a query at t selects -- b per kept level-1 node plus the tail past
+    its last complete top node (token 0 adds at most one more)."""
+    T = lc.shape[0]
+    vis = torch.arange(start + 1, start + T + 1, dtype=torch.int64)  # t + 1
+    tail = vis - b ** L * torch.div(vis, b ** L, rounding_mode="floor")
+    sel = b * lc[..., L - 1].long() + tail[:, None]
+    return {"mean_kept_per_level": [round(float(v), 3) for v in lc.double().mean(dim=(0, 1))],
+            "mean_selected_fraction": float((sel.double() / vis.double()[:, None]).mean())}
+
+
 def decode_step_bytes(cand_rows: int, kept_nodes: int, b: int, tail: int, units: int,
                       queries: int, row: int):
     """Algorithmic bytes of one decode step, counted once per unit (a sequence
@@ -637,6 +651,9 @@ def wide_p_sweep(dev, peak: float, steps: int = 20, warmup: int = 3) -> list:
         e1.record(stream)
         torch.cuda.synchronize()
         ms = e0.elapsed_time(e1) / steps
+        # kept counts per query: one more step on the same inputs, untimed
+        lc = torch.zeros(B, Hq, L, dtype=torch.int32, device=dev)
+        z.zha_decode(cfg, cache, q, p, out, lc, ws, st)
         stats = torch.zeros(B * Hkv, L + 1, dtype=torch.int32, device=dev)
         z.zha_decode_stats(cfg, ws, stats)
         stats = stats.cpu()
@@ -646,7 +663,8 @@ def wide_p_sweep(dev, peak: float, steps: int = 20, warmup: int = 3) -> list:
         res.append({"p": p, "ms_per_step": ms, "queries_per_s": B * Hq / (ms / 1e3),
                     "bytes_touched_per_step": sel_b + att_b,
                     "kv_fraction_read": kv_rows / (B * Hkv * n),
-                    "hbm_frac": (sel_b + att_b) / (ms / 1e3) / 1e9 / peak})
+                    "hbm_frac": (sel_b + att_b) / (ms / 1e3) / 1e9 / peak,
+                    **selection_per_query(lc.cpu(), b, L, n, D * 2)})
     if int(st.item()) != 0:
         raise RuntimeError(f"wide sweep: device status {z.status_string(int(st.item()))}")
     del cache, ws, wl
@@ -667,7 +685,7 @@ def prefill_chunk_leg(rank, world, dev, steps: int = 3, warmup: int = 3) -> dict
         return {"error": f"{type(e).__name__}: {e}"[:300]}
     del wl
     torch.cuda.empty_cache()
-    keep = ("metric", "value", "unit", "steps", "warmup", "ms_per_step", "config",
+    keep = ("metric", "value", "unit", "steps", "warmup", "ms_per_step", "config", "selection",
             "tensor_core_top_level", "roofline", "tree_build", "e2e", "gpu_launches", "clocks")
     return {k: r[k] for k in keep}
 
@@ -974,6 +992,13 @@ def run_prefill(args, rank, world, dev):
     queries_per_step = T * Hq
     value = throughput(queries_per_step, args.steps, world, ms_total)
 
+    # ---- kept counts per (token, head): one more step, untimed ----
+    lc = torch.zeros(T, Hq, L, dtype=torch.int32, device=dev)
+    cache.seq_len = len1
+    z.zha_prefill_chunk(cfg, cache, q, 0, start, c.p, out, lc, ws, st)
+    torch.cuda.synchronize()
+    selection = prefill_selection(lc.cpu(), b, L, start)
+
     # ---- the tensor-core top level alone (GEMM + certificates) ----
     cert = torch.full((T, Hq), -1, dtype=torch.int32, device=dev)
     z.zha_prefill_top_scores(cfg, cache, q, 0, start, c.p, None, cert, ws, st)
@@ -1039,6 +1064,7 @@ def run_prefill(args, rank, world, dev):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded Gaussian-mixture keys, planted needles; no dataset)",
         "config": workload_config(args, c),
+        "selection": selection,
         "tensor_core_top_level": {
             "ms": top_ms, "top_nodes": n_top, "gemm_flops": gemm_flops,
             "gemm_tflops_incl_certify": gemm_flops / (top_ms / 1e3) / 1e12,

@@ -269,3 +269,19 @@ def test_bench_decode_step_bytes():
     # the bytes that step reported
     sel, att, kv = bench.decode_step_bytes(1397720, 1048300, 4, 205, 16, 128, 256)
     assert kv == 4196496 and sel + att == 2514939744 - 128 * 256
+
+
+def test_bench_prefill_selection():
+    import importlib
+    import sys
+
+    sys.path.insert(0, ROOT)
+    bench = importlib.import_module("bench")
+    # by hand: b = 4, L = 2 (top nodes of 16 tokens), chunk tokens at positions
+    # 30, 31, 32 (31, 32, 33 visible tokens: tails of 15, 0 and 1), 2 heads,
+    # kept counts top level first
+    lc = torch.tensor([[[1, 2], [1, 3]], [[2, 4], [2, 0]], [[1, 1], [2, 1]]], dtype=torch.int32)
+    got = bench.prefill_selection(lc, 4, 2, 30)
+    assert got["mean_kept_per_level"] == [1.5, round(11 / 6, 3)]
+    sel_frac = [23 / 31, 27 / 31, 16 / 32, 0 / 32, 5 / 33, 5 / 33]
+    assert abs(got["mean_selected_fraction"] - sum(sel_frac) / 6) < 1e-12
