@@ -403,6 +403,44 @@ def test_traversal_tiny_p_is_argmax_descent():
     assert checked >= 5
 
 
+def test_budget_adapts_to_how_peaked_the_query_is():
+    """The budget is per query (lefilia.fr page, par. 3): the sharper a
+    query's estimated mass, the fewer nodes cover p of it. For a fixed
+    candidate set, scaling the query by a > 0 multiplies every score
+    difference by a, and the share of the mass held by the k best candidates
+    can only grow with a (its log-derivative is the tilted mean score of the
+    k best minus that of all candidates, never negative), so the top level's
+    count never grows with a; queries flagged near-tie at some a > 0 are left
+    out. Below
+    the top the candidates change with the cut above, so there only the
+    overall trend is checked: selections shrink from a flat query (a = 0,
+    the ceil(p n) lowest nodes) to a sharp one."""
+    rng = np.random.default_rng(13)
+    b, L, d, p = 4, 4, 64, 0.95
+    n = 16 * b ** L
+    K = rng.standard_normal((n, d)).astype(np.float32)
+    R = (rng.standard_normal((16, d)) / math.sqrt(d)).astype(np.float32)
+    tr = oracle.build_tree(K, n, R, b, L, False)
+    scales = (0.0, 2.0, 4.0, 8.0, 16.0, 32.0, 64.0)
+    checked = 0
+    for _ in range(6):
+        u = rng.standard_normal(d)
+        u /= np.linalg.norm(u)
+        tops, sizes = [], []
+        for a in scales:
+            idx, counts, _, tie = oracle.select((a * u).astype(np.float32), tr, n - 1, p)
+            if tie and a > 0:  # a = 0: exact ties everywhere, settled by the index rule
+                break
+            tops.append(int(counts[0]))
+            sizes.append(len(idx))
+        else:
+            assert all(x >= y for x, y in zip(tops, tops[1:])), tops
+            assert sizes[0] > sizes[3] > sizes[5] > sizes[6], sizes
+            assert sizes[6] < sizes[0] // 4, sizes
+            checked += 1
+    assert checked >= 4
+
+
 def test_no_complete_top_node_is_dense():
     rng = np.random.default_rng(11)
     K = rng.standard_normal((100, 64)).astype(np.float32)
